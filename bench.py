@@ -1,4 +1,33 @@
-"""Benchmark of one denoising step (filled in with the CUDA path)."""
+"""Benchmark: one denoising step of the active block on B200.
+
+Workload: Qwen2.5-7B shapes in bf16 (batch 4, 28 query / 4 KV heads, head dim
+128, hidden 3584, vocab 152064, per-sequence prefix lengths U[1024, 2048],
+block 32 with the sub-block of 8 active, tau 0.9), synthetic seeded inputs.
+
+``python bench.py --gpus N --steps K --warmup W`` prints one JSON line.  A
+step is one fdl_denoise_step (attention -> token-shift gather -> fused LM
+head / confidence / commit).  With N > 1 (torchrun) every rank runs its own
+batch of 4 sequences (weak scaling, no collective on the data path); the time
+is the max over ranks.  ``--impl reference`` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "qwen7b"
+METRIC = "denoise-step latency (us) & positions/s at Qwen2.5-7B shapes; % HBM roofline"
+UNIT = "positions/s"
 
 
 def roofline_seconds(bytes_moved: float, flops: float, hbm_bps: float,
@@ -6,3 +35,373 @@ def roofline_seconds(bytes_moved: float, flops: float, hbm_bps: float,
     """Lower bound on a kernel's time: the slower of moving its bytes at the
     memory bandwidth and doing its FLOPs at the arithmetic peak."""
     return max(bytes_moved / hbm_bps, flops / flops_per_s)
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def oracle_baseline(case, min_seconds: float = 10.0, max_steps: int = 50) -> dict:
+    """Time the CPU oracle (as it stands) on this workload: whole steps,
+    repeated until ``min_seconds`` have passed."""
+    import numpy as np
+    import threadpoolctl
+    from oracle import cases
+    threads = max(
+        [i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
+    n, t0 = 0, time.perf_counter()
+    while True:
+        cases.run_oracle(case)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or n >= max_steps:
+            break
+    c = case.cfg
+    pos = n * c["batch"] * c["q_len"]
+    return {"value": pos / el, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+            "sample": f"{n} whole oracle step(s) of the benchmark workload "
+                      f"({c['batch']} x {c['q_len']} positions each), {el:.1f} s, "
+                      f"numpy fp64 with {threads} BLAS threads",
+            "seconds": el, "steps": n}
+
+
+# ------------------------------------------------------------------- main
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=1002)
+    ap.add_argument("--kv-copies", type=int, default=16)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        dist.barrier(device_ids=[torch.cuda.current_device()])
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, timed on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from block_diffusion_decoding_causal_b200 import synth
+    from oracle import cases
+    case = synth.make_case(WORKLOAD, args.seed)
+    c = case.cfg
+    for _ in range(args.warmup):
+        cases.run_oracle(case)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cases.run_oracle(case)
+    el = time.perf_counter() - t0
+    import threadpoolctl
+    threads = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
+    pos = args.steps * c["batch"] * c["q_len"]
+    value = pos / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(c, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(threads),
+                         "kind": "oracle",
+                         "sample": f"{args.steps} whole oracle steps of the workload"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(c, args):
+    return {"workload": "Qwen2.5-7B-shape denoise step (bf16, batch 4, 28/4 heads, "
+                        "d 128, H 3584, V 152064, prefix U[1024,2048], block 32, "
+                        "sub-block 8, tau 0.9)",
+            "batch": c["batch"], "q_len": c["q_len"], "block_size": c["block_size"],
+            "n_q_heads": c["n_q_heads"], "n_kv_heads": c["n_kv_heads"],
+            "head_dim": c["head_dim"], "hidden": c["hidden"], "vocab": c["vocab"],
+            "prefix": list(c["prefix"]), "tau": c["tau"], "seed": args.seed,
+            "parallelism": f"replicas x{int(os.environ.get('WORLD_SIZE', '1'))}",
+            "l2": "inputs larger than L2: the 1.09 GB LM-head weight streams every "
+                  f"step; KV caches rotate over {args.kv_copies} copies"}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    from block_diffusion_decoding_causal_b200 import fdl, synth
+
+    world, rank, local = dist_setup()
+    peaks = measured_peaks()
+    case = synth.make_case(WORKLOAD, args.seed + rank)
+    c = case.cfg
+    cfg = fdl.make_cfg(c)
+    B, q_len, H, V = c["batch"], c["q_len"], c["hidden"], c["vocab"]
+    stream = torch.cuda.Stream()
+    dev = lambda t: None if t is None else t.cuda().contiguous()
+    n_copies = max(1, args.kv_copies)
+    with torch.cuda.stream(stream):
+        w = dev(case.w_lm)
+        sets = []
+        for i in range(n_copies):
+            sets.append(dict(q=dev(case.q), k_pre=dev(case.k_pre), v_pre=dev(case.v_pre),
+                             len_pre=dev(case.len_pre), k_blk=dev(case.k_blk),
+                             v_blk=dev(case.v_blk), hidden=dev(case.hidden),
+                             h_prev=dev(case.h_prev), bt=dev(case.block_tokens)))
+        out = dict(attn=torch.empty_like(sets[0]["q"]),
+                   conf=torch.empty((B, q_len), dtype=torch.float32, device="cuda"),
+                   tok=torch.empty((B, q_len), dtype=torch.int32, device="cuda"),
+                   committed=torch.empty((B, c["block_size"]), dtype=torch.uint8, device="cuda"),
+                   n_c=torch.empty(B, dtype=torch.int32, device="cuda"),
+                   n_l=torch.empty(B, dtype=torch.int32, device="cuda"))
+        ws = fdl.workspace(cfg)
+    stream.synchronize()
+
+    def step(s):
+        fdl.denoise_step(cfg, s["q"], s["k_pre"], s["v_pre"], s["len_pre"], s["k_blk"],
+                         s["v_blk"], None, None, None, s["hidden"], s["h_prev"], w,
+                         s["bt"], out["attn"], out["conf"], out["tok"], out["committed"],
+                         out["n_c"], out["n_l"], ws, stream)
+
+    def timed(fn, k):
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for i in range(k):
+            fn(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        return ev0.elapsed_time(ev1) / 1e3
+
+    for i in range(args.warmup):
+        step(sets[i % n_copies])
+    torch.cuda.synchronize()
+    assert fdl.get_status(ws, stream) == 0
+
+    with ClockSampler(_gpu_id(torch)) as clocks:
+        t_step = timed(lambda i: step(sets[i % n_copies]), args.steps)
+    t_step = max_over_ranks(t_step, world)
+    ms_per_step = t_step / args.steps * 1e3
+    pos = world * B * q_len * args.steps
+    value = pos / t_step
+
+    # Dominant kernel: the fused LM head (weight stream), timed alone on the
+    # same stream over K launches.
+    rows = sets[0]["hidden"].view(B * q_len, H)
+    lm = lambda i: fdl.lmhead_confidence(cfg, rows, w, None, out["conf"], out["tok"],
+                                         ws, stream)
+    for i in range(3):
+        lm(i)
+    t_lm = max_over_ranks(timed(lm, args.steps), world) / args.steps
+    attn = lambda i: fdl.block_attn(cfg, sets[i % n_copies]["q"], sets[i % n_copies]["k_pre"],
+                                    sets[i % n_copies]["v_pre"], sets[i % n_copies]["len_pre"],
+                                    sets[i % n_copies]["k_blk"], sets[i % n_copies]["v_blk"],
+                                    out["attn"], ws, stream)
+    for i in range(3):
+        attn(i)
+    t_attn = max_over_ranks(timed(attn, args.steps), world) / args.steps
+
+    # End to end through the public API: per step, pinned host inputs copied
+    # in, the step, and its results copied out and read on the host.
+    host_in = {k: v.cpu().pin_memory() for k, v in sets[0].items()
+               if k in ("q", "k_blk", "v_blk", "hidden", "h_prev", "bt", "len_pre")}
+    host_out = {k: torch.empty_like(out[k], device="cpu").pin_memory()
+                for k in ("conf", "tok", "committed", "n_c", "n_l")}
+    host_bt = torch.empty_like(host_in["bt"]).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values()) + \
+        host_bt.numel() * host_bt.element_size()
+    e2e_set = dict(sets[0])
+
+    def e2e_step(i):
+        with torch.cuda.stream(stream):
+            for k, t in host_in.items():
+                e2e_set[k].copy_(t, non_blocking=True)
+        step(e2e_set)
+        with torch.cuda.stream(stream):
+            for k, t in host_out.items():
+                t.copy_(out[k], non_blocking=True)
+            host_bt.copy_(e2e_set["bt"], non_blocking=True)
+        stream.synchronize()
+        _ = int(host_out["n_l"].sum())      # the host reads the result
+    for i in range(2):
+        e2e_step(i)
+    t_e2e = max_over_ranks(timed(e2e_step, args.steps), world)
+    e2e_value = pos / t_e2e
+
+    committed = float(out["n_c"].float().mean().item())
+    clk = clocks.summary()
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+
+    lm_bytes = V * H * 2 + B * q_len * H * 2 + B * q_len * 8
+    lm_gbs = lm_bytes / t_lm / 1e9
+    traffic = _profiled_traffic("lmhead")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "step_latency_us": ms_per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V/hidden, W_lm ~ N(0,1/H) x 8)",
+        "config": _config(c, args),
+        "roofline": {"bound": "hbm", "kernel": "fused LM head + confidence",
+                     "achieved": lm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": lm_gbs / peaks["hbm_gbs"],
+                     "peak_source": f"{peaks['source']} hbm_gbs (burst copy)",
+                     "traffic": traffic, "bytes_per_launch": lm_bytes,
+                     "us_per_launch": t_lm * 1e6},
+        "attention": {"us_per_launch": t_attn * 1e6},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e / args.steps * 1e3},
+        "gpu_launches": _launches_per_step(c) * args.steps,
+        "committed_per_step": committed,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_baseline(case)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def _gpu_id(torch) -> str:
+    """nvidia-smi identifier (UUID) of the current CUDA device."""
+    try:
+        u = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(torch.cuda.current_device())
+
+
+def _launches_per_step(c) -> int:
+    """Kernels one fdl_denoise_step launches: attention, (token-shift gather),
+    fused LM head + commit."""
+    return 3 if c["shift"] else 2
+
+
+def _profiled_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it covers the
+    current kernel build (see profiles/)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    return d.get(kernel)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

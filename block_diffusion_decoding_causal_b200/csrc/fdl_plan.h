@@ -1,0 +1,111 @@
+// Host-side launch plan and workspace layout of one step configuration.
+#pragma once
+
+#include <cmath>
+#include <cstddef>
+#include <string>
+
+#include "fdl.h"
+
+namespace fdl {
+
+constexpr int kAttnRowTile = 16;   // query rows per attention CTA
+constexpr int kPlanCTAs = 148;     // grid sizing unit: one B200's SM count
+constexpr int kLmMaxCTAs = 4 * kPlanCTAs;
+
+struct AttnSplit {
+  int split_keys;  // keys per split, multiple of 64
+  int n_split;
+};
+
+struct Plan {
+  int R;           // LM-head rows = batch * q_len
+  int elem;        // bytes per floating element
+  int n_row_tiles;
+  AttnSplit attn_plain, attn_dual;
+  int lm_cta, lm_rows_per_cta;
+  size_t off_ctrl, off_tickets, off_part_o, off_part_ml, off_rows, off_lm_part,
+      off_attn, total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Split the (b, kv head, row tile) key sequences so that about two CTAs per
+// SM are in flight.
+inline AttnSplit plan_split(long keys_cap, long items) {
+  AttnSplit s;
+  long want = (2L * kPlanCTAs + items - 1) / items;
+  long max_split = (keys_cap + 63) / 64;
+  if (want < 1) want = 1;
+  if (want > max_split) want = max_split;
+  long per = (keys_cap + want - 1) / want;
+  per = (per + 63) / 64 * 64;
+  s.split_keys = (int)per;
+  s.n_split = (int)((keys_cap + per - 1) / per);
+  return s;
+}
+
+inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why) {
+  if (c == nullptr) { *why = "cfg is NULL"; return false; }
+  if (c->dtype != FDL_F32 && c->dtype != FDL_BF16) { *why = "dtype must be FDL_F32 or FDL_BF16"; return false; }
+  if (c->batch < 1) { *why = "batch must be >= 1"; return false; }
+  if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads != 0) {
+    *why = "n_q_heads must be a positive multiple of n_kv_heads"; return false;
+  }
+  if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) {
+    *why = "head_dim must be 32, 64 or 128"; return false;
+  }
+  if (c->block_size < 1 || c->block_size > 64) { *why = "block_size must be in [1, 64]"; return false; }
+  if (c->q_len < 1 || c->q_len > 32) { *why = "q_len must be in [1, 32]"; return false; }
+  if (c->q_off < 0 || c->q_off + c->q_len > c->block_size) {
+    *why = "the unit [q_off, q_off+q_len) must lie inside the block"; return false;
+  }
+  if (c->cap_prefix < 0 || c->cap_suffix < 0) { *why = "cache capacities must be >= 0"; return false; }
+  if (c->hidden < 8 || c->hidden % 8 != 0) { *why = "hidden must be a positive multiple of 8"; return false; }
+  if (c->vocab < 2) { *why = "vocab must be >= 2"; return false; }
+  if (c->mask_id < 0 || c->mask_id >= c->vocab) { *why = "mask_id must be in [0, vocab)"; return false; }
+  if (c->shift != 0 && c->shift != 1) { *why = "shift must be 0 or 1"; return false; }
+  if (!std::isfinite(c->tau)) { *why = "tau must be finite"; return false; }
+  const long R = (long)c->batch * c->q_len;
+  if (R > 256) { *why = "batch * q_len must be <= 256"; return false; }
+
+  p->R = (int)R;
+  p->elem = c->dtype == FDL_BF16 ? 2 : 4;
+  const int group = c->n_q_heads / c->n_kv_heads;
+  const int rows = c->q_len * group;
+  p->n_row_tiles = (rows + kAttnRowTile - 1) / kAttnRowTile;
+  const long items = (long)c->batch * c->n_kv_heads * p->n_row_tiles;
+  const long keys_plain = (long)c->cap_prefix + c->block_size;
+  const long keys_dual = keys_plain + c->cap_suffix;
+  p->attn_plain = plan_split(keys_plain, items);
+  p->attn_dual = plan_split(keys_dual, items);
+  const long max_split = p->attn_plain.n_split > p->attn_dual.n_split
+                             ? p->attn_plain.n_split : p->attn_dual.n_split;
+
+  // LM head: contiguous vocabulary ranges (multiples of 16 rows) over about
+  // two CTAs per SM.
+  long per = ((long)c->vocab + 2 * kPlanCTAs - 1) / (2 * kPlanCTAs);
+  per = (per + 15) / 16 * 16;
+  p->lm_rows_per_cta = (int)per;
+  p->lm_cta = (int)(((long)c->vocab + per - 1) / per);
+
+  size_t off = 0;
+  p->off_ctrl = off;
+  off = align256(off + 256);
+  p->off_tickets = off;
+  off = align256(off + sizeof(unsigned int) * (size_t)items);
+  p->off_part_o = off;
+  off = align256(off + sizeof(float) * (size_t)items * max_split * kAttnRowTile * c->head_dim);
+  p->off_part_ml = off;
+  off = align256(off + 8 * (size_t)items * max_split * kAttnRowTile);
+  p->off_rows = off;
+  off = align256(off + (size_t)p->elem * R * c->hidden);
+  p->off_lm_part = off;
+  off = align256(off + 16 * (size_t)kLmMaxCTAs * R);
+  p->off_attn = off;
+  off = align256(off + (size_t)p->elem * R * c->n_q_heads * c->head_dim);
+  p->total = off;
+  return true;
+}
+
+}  // namespace fdl

@@ -146,6 +146,8 @@ def make_case(name: str, seed: int, cfg: Optional[dict] = None,
 
     lo, hi = c["prefix"]
     len_pre = _ints(seed, "len_pre", B, lo, hi).to(torch.int32)
+    if c.get("len_pre") is not None:          # explicit per-sequence lengths
+        len_pre = torch.tensor(c["len_pre"], dtype=torch.int32)
     # Prompt part of the prefix: the rest is whole finished blocks.
     n_done = (len_pre // (4 * D)).to(torch.int32)
     prompt_len = (len_pre - n_done * D).to(torch.int32)

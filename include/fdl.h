@@ -1,0 +1,211 @@
+/*
+ * fdl.h - C ABI of libfdl.so: one denoising step of the active block in
+ * block-diffusion decoding (Fast-dLLM / Fast-dLLM v2), on one NVIDIA B200.
+ *
+ * The step (pages: "Fast-dLLM v2: Efficient Block-Diffusion LLM", section 3.4
+ * "Inference Pipeline" and Figure 7b; "Fast-dLLM: Reusing Bidirectional State
+ * and Spending Confidence on Parallel Tokens", sections 2-4):
+ *   (a) attention of the active unit's queries over the block-level prefix
+ *       KV cache, the block's own K/V (bidirectional within the block) and,
+ *       for DualCache, the cached suffix of still-masked positions;
+ *   (b) the LM-head contraction over the unit's hidden states fused with a
+ *       full-vocabulary (max probability, argmax) reduction, then the
+ *       confidence-threshold commit with its single-position fallback.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers.  Every tensor pointer is a caller-owned DEVICE pointer (lengths
+ *   included), 16-byte aligned, row-major and densely packed as documented.
+ *   The library allocates no memory and keeps no state between calls: its
+ *   only scratch is the caller's workspace `ws` (see fdl_workspace_size).
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *   default stream).  All work is enqueued asynchronously on it; no entry
+ *   point synchronises except fdl_get_status.
+ * Types.  Floating tensors share cfg->dtype (FDL_F32 or FDL_BF16); conf is
+ *   always float32, token ids int32, bitmaps uint8 (0/1).
+ * Errors.  Arguments the host can check (NULL pointers, shapes, alignment,
+ *   workspace size) are checked before any launch: the call returns a
+ *   negative fdl_status with no side effects, and fdl_last_error() gives a
+ *   message (thread-local).  Launch failures return FDL_ERR_CUDA.  Values the
+ *   host cannot see (device-resident lengths outside [0, capacity]) are
+ *   detected by the kernels: the sequence is processed as if the offending
+ *   length were 0, a bit is set in the workspace status word, and
+ *   fdl_get_status reports it.  No kernel traps.
+ * Workspace.  `ws` must be at least fdl_workspace_size(cfg) bytes, 256-byte
+ *   aligned, and zero-filled before its first use (cudaMemset or
+ *   fdl_reset_workspace).  Every call leaves its counters at zero again, so
+ *   a workspace can be reused for any number of calls on one stream.  Calls
+ *   that overlap on the GPU must use different workspaces.
+ */
+#ifndef FDL_H_
+#define FDL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FDL_VERSION 1
+
+typedef enum { FDL_F32 = 0, FDL_BF16 = 1 } fdl_dtype;
+
+typedef enum {
+  FDL_OK = 0,
+  FDL_ERR_INVALID_ARG = -1,   /* bad pointer, shape, alignment or value      */
+  FDL_ERR_UNSUPPORTED = -2,   /* valid but outside what the kernels handle   */
+  FDL_ERR_WORKSPACE = -3,     /* workspace NULL, misaligned or too small     */
+  FDL_ERR_CUDA = -4,          /* a CUDA call or launch failed                */
+  FDL_ERR_DEVICE_STATUS = -5  /* fdl_get_status: a kernel flagged bad input  */
+} fdl_status;
+
+/* Device status bits (fdl_get_status). */
+#define FDL_DEV_BAD_PREFIX_LEN 1u  /* len_pre[b] outside [0, cap_prefix] */
+#define FDL_DEV_BAD_SUFFIX_LEN 2u  /* len_suf[b] outside [0, cap_suffix] */
+
+/*
+ * Geometry and decoding parameters of one step.
+ *
+ * The pages state the problem as a prompt of length P, a generation length L
+ * cut into blocks of block_size (D = 32 in all their experiments), sub-blocks
+ * of q_len (8 by default) as the thresholding unit, a threshold tau and a
+ * mask token.  One step works on block index k of the answer:
+ *   prefix length Lp = P + k*D (prompt + finished blocks, exact cache);
+ *   suffix length Ls = L - (k+1)*D (DualCache only: masked positions after
+ *     the block, whose K/V are frozen);
+ *   the active unit is block positions [q_off, q_off + q_len).
+ * Lp and Ls are per sequence and live on the device (len_pre / len_suf);
+ * cap_prefix / cap_suffix are the cache capacities (rows per (sequence, KV
+ * head)).
+ */
+typedef struct {
+  int32_t batch;       /* B >= 1                                               */
+  int32_t n_q_heads;   /* Hq; Hq % Hkv == 0                                    */
+  int32_t n_kv_heads;  /* Hkv; query head h reads KV head h / (Hq / Hkv)       */
+  int32_t head_dim;    /* d in {32, 64, 128}; softmax scale 1/sqrt(d)          */
+  int32_t block_size;  /* D, 1..64                                             */
+  int32_t q_off;       /* first block position of the active unit             */
+  int32_t q_len;       /* unit length, 1..32, q_off + q_len <= D               */
+  int32_t cap_prefix;  /* prefix cache rows per (b, kv head), >= 0             */
+  int32_t cap_suffix;  /* suffix cache rows per (b, kv head), >= 0 (DualCache) */
+  int32_t hidden;      /* H: LM-head input width                               */
+  int32_t vocab;       /* V >= 2                                               */
+  int32_t mask_id;     /* the [MASK] token id, 0 <= mask_id < V                */
+  int32_t shift;       /* 1: position p is predicted from the hidden state of
+                          p - 1 (v2 token shift); 0: from p itself             */
+  float tau;           /* commit iff confidence >= tau                         */
+  int32_t dtype;       /* fdl_dtype of every floating tensor                   */
+} fdl_step_cfg;
+
+/* Library version (FDL_VERSION) and a thread-local description of the last
+ * error returned on this thread ("" if none). */
+int fdl_version(void);
+const char* fdl_last_error(void);
+
+/* Bytes of workspace any entry point needs for this configuration; 0 if the
+ * configuration is invalid (fdl_last_error says why). */
+size_t fdl_workspace_size(const fdl_step_cfg* cfg);
+
+/* Zero a workspace (async memset on `stream`). */
+int fdl_reset_workspace(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Block-wise attention, v2 (stage a; "Fast-dLLM v2", section 3.4, Figure 7b
+ * and Level 3; attention itself is eq. (3) of the technical review).
+ *   For sequence b, query head h (KV head h / (Hq/Hkv)) and unit row r:
+ *     out[b,r,h,:] = softmax(q[b,r,h,:] . K^T / sqrt(d)) V over the keys
+ *     K = k_pre[b,kvh, 0:len_pre[b], :]  followed by  k_blk[b,kvh, 0:D, :]
+ *   i.e. every cached earlier block (causal across blocks) and every row of
+ *   the active block (bidirectional within it); later blocks do not exist.
+ *   The block rows of the active unit are the fresh K/V the caller computed
+ *   this step; the other block rows are its sub-block cache.
+ * Layouts: q, out [B, q_len, Hq, d]; k_pre, v_pre [B, Hkv, cap_prefix, d];
+ *   len_pre int32 [B]; k_blk, v_blk [B, Hkv, D, d].
+ * fp32 accumulation; out is rounded to cfg->dtype.
+ */
+int fdl_block_attn(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
+                   const void* v_pre, const int32_t* len_pre, const void* k_blk,
+                   const void* v_blk, void* out, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/*
+ * DualCache attention, v1 (stage a; technical review section 3 and its
+ * Algorithm 1, lines 6-7).  As fdl_block_attn with a third key segment,
+ * the frozen suffix cache k_suf/v_suf [B, Hkv, cap_suffix, d], rows
+ * 0:len_suf[b]; every key of prefix, block and suffix is visible (the
+ * full-attention dLLMs DualCache accelerates).
+ */
+int fdl_dualcache_attn(const fdl_step_cfg* cfg, const void* q,
+                       const void* k_pre, const void* v_pre,
+                       const int32_t* len_pre, const void* k_blk,
+                       const void* v_blk, const void* k_suf, const void* v_suf,
+                       const int32_t* len_suf, void* out, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/*
+ * LM head + confidence (stage b, first half; "Fast-dLLM v2" Level 2 and
+ * Algorithm 2 steps 1-2 of the technical review).
+ *   For each row i of rows [B*q_len, H] (already token-shifted: row
+ *   (b, i) predicts block position q_off + i):
+ *     l = w_lm . rows[i]  over the full vocabulary (w_lm [V, H] row-major),
+ *     tok[i]  = argmax_v l_v (the lowest v on a tie),
+ *     conf[i] = max softmax probability = 1 / sum_v exp(l_v - l_max).
+ *   Logits never leave the chip.  Rows with row_active[i] == 0 report
+ *   conf = -1 and tok = -1 (row_active may be NULL: all rows active).
+ * Outputs: conf float32 [B, q_len], tok int32 [B, q_len].
+ */
+int fdl_lmhead_confidence(const fdl_step_cfg* cfg, const void* rows,
+                          const void* w_lm, const uint8_t* row_active,
+                          float* conf, int32_t* tok, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/*
+ * Threshold commit (stage b, second half; technical review Algorithm 2
+ * steps 3-5; "Fast-dLLM v2" Level 2 and the sub-block paragraph).
+ *   Candidates C_b = unit positions p in [q_off, q_off+q_len) with
+ *   block_tokens[b,p] == mask_id.  S_b = {p in C_b : conf[b,p-q_off] >= tau};
+ *   if S_b is empty and C_b is not, S_b = {the p in C_b with the largest
+ *   conf, the lowest p on a tie}.  Then block_tokens[b,p] = tok[b,p-q_off]
+ *   for p in S_b (all at once).
+ * In/out: block_tokens int32 [B, D].  Out: committed uint8 [B, D] (1 on S_b,
+ *   0 elsewhere in the block), n_committed int32 [B] = |S_b|,
+ *   n_masked_left int32 [B] = unit positions still equal to mask_id.
+ */
+int fdl_threshold_commit(const fdl_step_cfg* cfg, const float* conf,
+                         const int32_t* tok, int32_t* block_tokens,
+                         uint8_t* committed, int32_t* n_committed,
+                         int32_t* n_masked_left, void* stream);
+
+/*
+ * One whole denoising step on one stream, no host synchronisation:
+ *   attention (DualCache when k_suf != NULL, else block-causal) ->
+ *   LM-head rows (hidden if given, else the attention output; then the token
+ *   shift: with cfg->shift, row i is source row i-1 and row 0 is h_prev[b],
+ *   the hidden state of the position before the unit) -> LM head +
+ *   confidence on the rows whose target is still masked -> commit.
+ * hidden: [B, q_len, H] or NULL (then H must equal Hq*d and the attention
+ *   output, rounded to cfg->dtype, is used).  h_prev: [B, H], required iff
+ *   cfg->shift.  attn_out: [B, q_len, Hq, d] or NULL (then it is kept in the
+ *   workspace).  k_suf, v_suf, len_suf: all NULL or all set.
+ * Outputs as fdl_lmhead_confidence and fdl_threshold_commit.
+ */
+int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
+                     const void* v_pre, const int32_t* len_pre,
+                     const void* k_blk, const void* v_blk, const void* k_suf,
+                     const void* v_suf, const int32_t* len_suf,
+                     const void* hidden, const void* h_prev, const void* w_lm,
+                     int32_t* block_tokens, void* attn_out, float* conf,
+                     int32_t* tok, uint8_t* committed, int32_t* n_committed,
+                     int32_t* n_masked_left, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* Synchronise `stream`, read the workspace status word into *status (bits
+ * FDL_DEV_*) and clear it.  Returns FDL_ERR_DEVICE_STATUS if any bit was
+ * set, FDL_OK otherwise. */
+int fdl_get_status(void* ws, void* stream, uint32_t* status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FDL_H_ */

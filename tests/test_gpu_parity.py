@@ -1,0 +1,190 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Bit-exact on committed token ids, argmax tokens, bitmaps and counts (inputs
+are margin-repaired so no decision sits on a rounding boundary); within
+2e-2 (bf16) or 1e-4 (fp32) relative for attention outputs and confidences.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_decoding_causal_b200 import fdl, synth
+from oracle import cases, step
+from tests import gpu_harness as gh
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+
+
+# ------------------------------------------------------------ fused step
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_tiny_fp32_step(seed):
+    case, ref, _ = cases.parity_case("tiny", seed)
+    gh.compare_step(case, gh.run_denoise_step(case), ref)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_tiny_fp32_step_attention_feeds_lm_head(seed):
+    case, ref, _ = cases.parity_case("tiny", seed, attn_as_hidden=True)
+    gh.compare_step(case, gh.run_denoise_step(case), ref)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_qwen15b_step(seed):
+    case, ref, _ = cases.parity_case("qwen1.5b", seed)
+    gh.compare_step(case, gh.run_denoise_step(case), ref)
+
+
+@pytest.mark.parametrize("tau", [0.7, 0.9])
+def test_qwen7b_step(tau):
+    case, ref, _ = cases.parity_case("qwen7b", 0, tau=tau)
+    gh.compare_step(case, gh.run_denoise_step(case), ref)
+
+
+def test_qwen7b_step_attention_feeds_lm_head():
+    case, ref, _ = cases.parity_case("qwen7b", 3, attn_as_hidden=True)
+    gh.compare_step(case, gh.run_denoise_step(case), ref)
+
+
+def test_llada_dualcache_step():
+    case, ref, _ = cases.parity_case("llada", 0)
+    gh.compare_step(case, gh.run_denoise_step(case), ref)
+
+
+# ------------------------------------------------------- ragged / edges
+
+SMALL = dict(batch=3, n_q_heads=14, n_kv_heads=2, head_dim=64, block_size=16,
+             q_len=5, q_off=None, prefix=(0, 300), cap_prefix=320, suffix=0,
+             cap_suffix=0, hidden=448, vocab=5000, mask_id=4999, shift=1,
+             tau=0.8, w_scale=8.0, dtype="bf16", masked=(1, 5))
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_ragged_shapes_step(seed):
+    """GQA group 7, q_len 5 (ragged row tiles), prefix lengths in [0, 300]
+    (empty prefix included), vocab not a multiple of the tile."""
+    lens = [0, 157, 300] if seed == 0 else None
+    case, ref, _ = cases.parity_case("small", seed, cfg=SMALL, len_pre=lens)
+    gh.compare_step(case, gh.run_denoise_step(case), ref)
+
+
+def test_unit_of_one_position_mha():
+    cfg = dict(SMALL, n_q_heads=4, n_kv_heads=4, q_len=1, masked=(1, 1), shift=0,
+               head_dim=32, hidden=128, dtype="f32")
+    case, ref, _ = cases.parity_case("one", 4, cfg=cfg)
+    gh.compare_step(case, gh.run_denoise_step(case), ref)
+
+
+def test_workspace_reuse_two_calls_in_a_row():
+    case, ref, _ = cases.parity_case("qwen1.5b", 5)
+    ws = fdl.workspace(fdl.make_cfg(case.cfg))
+    d = gh.device_case(case)
+    for _ in range(2):
+        gh.compare_step(case, gh.run_denoise_step(case, ws=ws, d=d), ref)
+
+
+def test_bad_prefix_length_sets_status_and_does_not_fault():
+    case = synth.make_case("tiny", 0)
+    case.len_pre[0] = case.cfg["cap_prefix"] + 5
+    res = gh.run_denoise_step(case)
+    assert res["status"] & fdl.DEV_BAD_PREFIX_LEN
+    # processed as an empty prefix: attention over the block rows alone
+    case.len_pre[0] = 0
+    ref = cases.run_oracle(case)
+    gh.assert_close_scaled(res["attn"].double().numpy(), ref["attn"], 1e-4, "attn")
+
+
+# ------------------------------------------------- standalone entry points
+
+def test_block_attn_entry_point():
+    case = synth.make_case("qwen7b", 7)
+    cfg = fdl.make_cfg(case.cfg)
+    d = gh.device_case(case)
+    out = torch.empty_like(d["q"])
+    ws = fdl.workspace(cfg)
+    fdl.block_attn(cfg, d["q"], d["k_pre"], d["v_pre"], d["len_pre"], d["k_blk"],
+                   d["v_blk"], out, ws)
+    ref = cases.run_oracle(case)
+    gh.assert_close_scaled(out.double().cpu().numpy(), ref["attn"], 2e-2, "attn")
+
+
+def test_dualcache_attn_entry_point():
+    case = synth.make_case("llada", 2)
+    cfg = fdl.make_cfg(case.cfg)
+    d = gh.device_case(case)
+    out = torch.empty_like(d["q"])
+    ws = fdl.workspace(cfg)
+    fdl.dualcache_attn(cfg, d["q"], d["k_pre"], d["v_pre"], d["len_pre"], d["k_blk"],
+                       d["v_blk"], d["k_suf"], d["v_suf"], d["len_suf"], out, ws)
+    ref = cases.run_oracle(case)
+    gh.assert_close_scaled(out.double().cpu().numpy(), ref["attn"], 2e-2, "attn")
+
+
+def test_lmhead_confidence_entry_point_with_row_mask():
+    case, ref, _ = cases.parity_case("qwen7b", 1)
+    cfg = fdl.make_cfg(case.cfg)
+    rows = torch.from_numpy(ref["rows"]).to(case.w_lm.dtype).cuda().contiguous()
+    active = torch.from_numpy(ref["active"].astype(np.uint8)).cuda()
+    conf = torch.empty(ref["conf"].shape, dtype=torch.float32, device="cuda")
+    tok = torch.empty(ref["conf"].shape, dtype=torch.int32, device="cuda")
+    fdl.lmhead_confidence(cfg, rows, case.w_lm.cuda(), active, conf, tok,
+                          fdl.workspace(cfg))
+    act = ref["active"]
+    assert np.array_equal(tok.cpu().numpy(), ref["tok"])
+    c = conf.cpu().numpy().astype(np.float64)
+    assert (c[~act] == -1).all()
+    np.testing.assert_allclose(c[act], ref["conf"][act], rtol=2e-2)
+
+
+def test_threshold_commit_entry_point_hand_cases():
+    """Algorithm 2 on hand-made confidences, including the fallback, an exact
+    tie, conf == tau and units with nothing masked."""
+    B, D, q_off, q_len, mask = 5, 16, 8, 8, 99
+    conf = np.array([
+        [0.95, 0.91, 0.5, 0.99, 0.1, 0.1, 0.1, 0.1],   # several above tau
+        [0.3, 0.8, 0.5, 0.8, 0.1, 0.2, 0.7, 0.6],      # fallback, tie -> lowest
+        [0.9, 0.2, 0.3, 0.4, 0.5, 0.6, 0.7, 0.8],      # conf == tau commits
+        [0.99] * 8,                                    # nothing masked
+        [0.5] * 8,                                     # masked only at the end
+    ], dtype=np.float32)
+    tok = np.arange(B * q_len, dtype=np.int32).reshape(B, q_len) + 1000
+    bt = np.full((B, D), mask, dtype=np.int32)
+    bt[:, :q_off] = 7
+    bt[3, q_off:] = 5
+    bt[4, q_off:q_off + 6] = 6
+    cfg = fdl.make_cfg(dict(batch=B, n_q_heads=1, n_kv_heads=1, head_dim=32,
+                            block_size=D, q_off=q_off, q_len=q_len, cap_prefix=0,
+                            hidden=8, vocab=2000, mask_id=mask, shift=0, tau=0.9,
+                            dtype="f32"))
+    d_bt = torch.from_numpy(bt).cuda()
+    comm = torch.empty((B, D), dtype=torch.uint8, device="cuda")
+    n_c = torch.empty(B, dtype=torch.int32, device="cuda")
+    n_l = torch.empty(B, dtype=torch.int32, device="cuda")
+    fdl.threshold_commit(cfg, torch.from_numpy(conf).cuda(), torch.from_numpy(tok).cuda(),
+                         d_bt, comm, n_c, n_l)
+    want = step.threshold_commit(bt, conf.astype(np.float64), tok, q_off, q_len, mask,
+                                 float(np.float32(0.9)))
+    assert np.array_equal(d_bt.cpu().numpy(), want[0])
+    assert np.array_equal(comm.cpu().numpy(), want[1])
+    assert np.array_equal(n_c.cpu().numpy(), want[2])
+    assert np.array_equal(n_l.cpu().numpy(), want[3])
+    assert want[2].tolist() == [3, 1, 1, 0, 1]
+
+
+# ------------------------------------------------ full-size sweep points
+
+@pytest.mark.parametrize("batch,prefix", [(16, 8192), (1, 8192)])
+def test_sweep_full_size(batch, prefix):
+    """Long-context sweep shapes at full size (prefix 8192, batch 16 = 128
+    LM-head rows): every output against the oracle."""
+    cfg = synth.sweep_config(batch, prefix, 8.0)
+    case, ref, _ = cases.parity_case("sweep", 0, cfg=cfg)
+    gpu = gh.run_denoise_step(case)
+    gh.compare_step(case, gpu, ref, check_attn=True)
