@@ -108,8 +108,9 @@ LmArgs lm_args(const fdl_step_cfg& c, const Plan& p, const void* rows,
   a.R = p.R;
   a.H = c.hidden;
   a.V = c.vocab;
-  a.n_cta = p.lm_cta;
-  a.rows_per_cta = p.lm_rows_per_cta;
+  const bool tc = c.dtype == FDL_BF16;
+  a.n_cta = tc ? p.lm_tc_cta : p.lm_cta;
+  a.rows_per_cta = tc ? p.lm_tc_rows_per_cta : p.lm_rows_per_cta;
   a.commit = 0;
   a.B = c.batch;
   a.D = c.block_size;
@@ -132,8 +133,17 @@ int run_attention(const fdl_step_cfg& c, const Plan& p, bool dual, const void* q
   return FDL_OK;
 }
 
+// bf16: tensor-core kernel (TMA + tcgen05, K in chunks of 64); fp32: the
+// CUDA-core kernel.
+int check_lmhead_supported(const fdl_step_cfg& c) {
+  if (c.dtype == FDL_BF16 && c.hidden % 64 != 0)
+    return fail(FDL_ERR_UNSUPPORTED, "bf16 LM head needs hidden %% 64 == 0 (got %d)", c.hidden);
+  return FDL_OK;
+}
+
 int run_lmhead(const LmArgs& a, const fdl_step_cfg& c, cudaStream_t s) {
-  cudaError_t e = launch_lmhead_simt(a, (fdl_dtype)c.dtype, s);
+  cudaError_t e = c.dtype == FDL_BF16 ? launch_lmhead_tc(a, s)
+                                      : launch_lmhead_simt(a, (fdl_dtype)c.dtype, s);
   if (e != cudaSuccess) return cuda_fail(e, "lm-head launch");
   return FDL_OK;
 }
@@ -226,7 +236,9 @@ int fdl_lmhead_confidence(const fdl_step_cfg* cfg, const void* rows,
   FDL_CHECK_PTR(w_lm);
   FDL_CHECK_PTR(conf);
   FDL_CHECK_PTR(tok);
-  int rc = check_ws(p, ws, ws_bytes);
+  int rc = check_lmhead_supported(*cfg);
+  if (rc != FDL_OK) return rc;
+  rc = check_ws(p, ws, ws_bytes);
   if (rc != FDL_OK) return rc;
   LmArgs a = lm_args(*cfg, p, rows, w_lm, row_active, conf, tok, ws);
   rc = run_lmhead(a, *cfg, (cudaStream_t)stream);
@@ -297,7 +309,9 @@ int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
                 c.hidden, c.n_q_heads * c.head_dim);
   if (c.shift) FDL_CHECK_PTR(h_prev);
   if (attn_out != nullptr) FDL_CHECK_PTR(attn_out);
-  int rc = check_ws(p, ws, ws_bytes);
+  int rc = check_lmhead_supported(c);
+  if (rc != FDL_OK) return rc;
+  rc = check_ws(p, ws, ws_bytes);
   if (rc != FDL_OK) return rc;
   cudaStream_t s = (cudaStream_t)stream;
 

@@ -176,6 +176,7 @@ __device__ __forceinline__ void commit_sequence_warp(
 cudaError_t launch_attn_simt(const AttnArgs& a, fdl_dtype dt, int row_tile,
                              cudaStream_t s);
 cudaError_t launch_lmhead_simt(const LmArgs& a, fdl_dtype dt, cudaStream_t s);
+cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s);
 cudaError_t launch_commit(const float* conf, const int32_t* tok,
                           int32_t* block_tokens, uint8_t* committed,
                           int32_t* n_committed, int32_t* n_masked_left, int B,

@@ -23,7 +23,8 @@ struct Plan {
   int elem;        // bytes per floating element
   int n_row_tiles;
   AttnSplit attn_plain, attn_dual;
-  int lm_cta, lm_rows_per_cta;
+  int lm_cta, lm_rows_per_cta;        // CUDA-core LM head (fp32)
+  int lm_tc_cta, lm_tc_rows_per_cta;  // tensor-core LM head (bf16): one CTA per SM
   size_t off_ctrl, off_tickets, off_part_o, off_part_ml, off_rows, off_lm_part,
       off_attn, total;
 };
@@ -88,6 +89,10 @@ inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why) {
   per = (per + 15) / 16 * 16;
   p->lm_rows_per_cta = (int)per;
   p->lm_cta = (int)(((long)c->vocab + per - 1) / per);
+  long per_tc = ((long)c->vocab + kPlanCTAs - 1) / kPlanCTAs;
+  per_tc = (per_tc + 15) / 16 * 16;
+  p->lm_tc_rows_per_cta = (int)per_tc;
+  p->lm_tc_cta = (int)(((long)c->vocab + per_tc - 1) / per_tc);
 
   size_t off = 0;
   p->off_ctrl = off;

@@ -1,0 +1,348 @@
+// LM head + confidence on the 5th-generation tensor cores (bf16, sm_100a).
+//
+// logits[v, r] = W[v, :] . X[r, :] over the full vocabulary, reduced on the
+// chip to each row's running (max logit, sum exp(l - max), argmax)
+// ("Fast-dLLM v2" Level 2: the greedy token and its probability; technical
+// review Algorithm 2 steps 1-2).  Logits never reach global memory.
+//
+// Swap-AB: the weight is the M = 128 operand (a tile of 128 vocabulary rows),
+// the <= 256 input rows are N.  Each CTA (one per SM) owns a contiguous
+// vocabulary range of ~V/148 rows and streams it once:
+//   warp 0   TMA producer: W tiles [128 x 64] (128-byte swizzle) through an
+//            A ring, X chunks [N x 64] through a B ring;
+//   warp 1   MMA issuer: tcgen05.mma kind::f16, accumulators in TMEM; tiles
+//            are processed in groups of G, K-outer inside a group so each X
+//            chunk is reused by G tiles; two TMEM buffers let the epilogue
+//            of group g overlap the MMAs of group g+1;
+//   warps 2-5  epilogue: tcgen05.ld 32 lanes x 32 columns, a warp
+//            reduce-scatter of (max, sum-exp, argmax) over the 32 vocab rows
+//            leaves column j's triple in lane j, merged into a running state.
+// The per-CTA triples go to the workspace; the last CTA to arrive merges them
+// (and, in the fused step, commits).  No thread waits on another CTA.
+#include "lm_merge.cuh"
+#include "sm100.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace fdl {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTileM = 128;                 // vocab rows per MMA tile
+constexpr int kKChunk = 64;                 // bf16 per 128-byte row
+constexpr int kStageA = kTileM * kKChunk * 2;  // 16 KB
+constexpr int kBoxPart = 16;                // rows per box of a partial tile
+constexpr int kThreads = 192;
+constexpr unsigned kDevTimeout = 4u;        // status bit: a bounded wait expired
+
+struct TcParams {
+  int npad;        // MMA N: 32, 64, 128 or 256
+  int group;       // tiles per TMEM buffer
+  int stages_a;
+  int stages_b;
+  uint32_t tmem_cols;
+};
+
+__device__ __forceinline__ void named_barrier_epilogue() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Reduce-scatter of 32 columns over the 32 lanes of a warp: on return,
+// lane j holds column j's (max, sum-exp, argmax) over all 32 lanes' rows.
+__device__ __forceinline__ MSI reduce_scatter32(MSI (&s)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool upper = (lane & w) != 0;
+#pragma unroll
+    for (int j = 0; j < w; ++j) {
+      const MSI keep = upper ? s[j + w] : s[j];
+      const MSI send = upper ? s[j] : s[j + w];
+      s[j] = msi_merge(keep, msi_shfl_xor(send, w));
+    }
+  }
+  return s[0];
+}
+
+template <int NCH>
+__global__ void __launch_bounds__(kThreads, 1)
+lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
+                 const __grid_constant__ CUtensorMap tm_w_part,
+                 const __grid_constant__ CUtensorMap tm_x, const LmArgs a,
+                 const TcParams tp) {
+  constexpr int NPAD = NCH * 32;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int SA = tp.stages_a, SB = tp.stages_b;
+  uint8_t* sa = smem;
+  uint8_t* sb = sa + SA * kStageA;
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(sb + SB * NPAD * 128);
+  uint64_t* empty_a = full_a + SA;
+  uint64_t* full_b = empty_a + SA;
+  uint64_t* empty_b = full_b + SB;
+  uint64_t* acc_full = empty_b + SB;   // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint64_t* drain = acc_empty + 2;     // [1]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  MSI* s_red = reinterpret_cast<MSI*>(tmem_holder + 4);  // [4][NPAD]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int v0 = blockIdx.x * a.rows_per_cta;
+  const int v1 = min(a.V, v0 + a.rows_per_cta);
+  const int n_rows = max(0, v1 - v0);
+  const int n_tiles = (n_rows + kTileM - 1) / kTileM;
+  const int G = tp.group;
+  const int n_groups = (n_tiles + G - 1) / G;
+  const int KC = a.H / kKChunk;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < SA; ++i) {
+      mbar_init(&full_a[i], 1);
+      mbar_init(&empty_a[i], 1);
+    }
+    for (int i = 0; i < SB; ++i) {
+      mbar_init(&full_b[i], 1);
+      mbar_init(&empty_b[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, tp.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  bool failed = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&tm_w_full);
+      tma_prefetch_desc(&tm_w_part);
+      tma_prefetch_desc(&tm_x);
+      const uint64_t pol_w = policy_evict_first();
+      int ia = 0, ib = 0;
+      for (int g = 0; g < n_groups && !failed; ++g) {
+        const int t0 = g * G, t1 = min(n_tiles, t0 + G);
+        for (int kc = 0; kc < KC && !failed; ++kc) {
+          const int slot_b = ib % SB;
+          if (!mbar_wait(&empty_b[slot_b], ((ib / SB) & 1) ^ 1)) { failed = true; break; }
+          mbar_arrive_expect_tx(&full_b[slot_b], NPAD * 128);
+          tma_load_2d(sb + slot_b * NPAD * 128, &tm_x, kc * kKChunk, 0, &full_b[slot_b]);
+          ++ib;
+          for (int t = t0; t < t1; ++t) {
+            const int slot_a = ia % SA;
+            if (!mbar_wait(&empty_a[slot_a], ((ia / SA) & 1) ^ 1)) { failed = true; break; }
+            const int row0 = v0 + t * kTileM;
+            const int rows = min(kTileM, v1 - row0);
+            uint8_t* dst = sa + slot_a * kStageA;
+            if (rows == kTileM) {
+              mbar_arrive_expect_tx(&full_a[slot_a], kStageA);
+              tma_load_2d_hint(dst, &tm_w_full, kc * kKChunk, row0, &full_a[slot_a], pol_w);
+            } else {
+              const int nbox = (rows + kBoxPart - 1) / kBoxPart;
+              mbar_arrive_expect_tx(&full_a[slot_a], nbox * kBoxPart * 128);
+              for (int j = 0; j < nbox; ++j)
+                tma_load_2d_hint(dst + j * kBoxPart * 128, &tm_w_part, kc * kKChunk,
+                                 row0 + j * kBoxPart, &full_a[slot_a], pol_w);
+            }
+            ++ia;
+          }
+        }
+      }
+      // Drain: every load issued has landed before this CTA can exit.
+      for (int n = max(0, ia - SA); n < ia; ++n)
+        if (!mbar_wait(&full_a[n % SA], (n / SA) & 1)) failed = true;
+      for (int n = max(0, ib - SB); n < ib; ++n)
+        if (!mbar_wait(&full_b[n % SB], (n / SB) & 1)) failed = true;
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t idesc = idesc_bf16_f32(kTileM, NPAD);
+      int ia = 0, ib = 0;
+      for (int g = 0; g < n_groups && !failed; ++g) {
+        const int buf = g & 1;
+        if (!mbar_wait(&acc_empty[buf], ((g >> 1) & 1) ^ 1)) { failed = true; break; }
+        tc_fence_after();
+        const int t0 = g * G, t1 = min(n_tiles, t0 + G);
+        for (int kc = 0; kc < KC && !failed; ++kc) {
+          const int slot_b = ib % SB;
+          if (!mbar_wait(&full_b[slot_b], (ib / SB) & 1)) { failed = true; break; }
+          tc_fence_after();
+          const uint32_t b_base = smem_u32(sb + slot_b * NPAD * 128);
+          for (int t = t0; t < t1; ++t) {
+            const int slot_a = ia % SA;
+            if (!mbar_wait(&full_a[slot_a], (ia / SA) & 1)) { failed = true; break; }
+            tc_fence_after();
+            const uint32_t a_base = smem_u32(sa + slot_a * kStageA);
+            const uint32_t d = tmem + (uint32_t)((buf * G + (t - t0)) * NPAD);
+#pragma unroll
+            for (int k = 0; k < kKChunk / 16; ++k)
+              mma_bf16(d, desc_k_sw128(a_base + k * 32), desc_k_sw128(b_base + k * 32),
+                       idesc, (kc | k) != 0 ? 1u : 0u);
+            mma_commit(&empty_a[slot_a]);
+            ++ia;
+          }
+          mma_commit(&empty_b[slot_b]);
+          ++ib;
+        }
+        mma_commit(&acc_full[buf]);
+      }
+      // Drain: all MMAs this thread issued have completed.
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0)) failed = true;
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    MSI st[NCH];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) st[c] = msi_empty();
+    for (int g = 0; g < n_groups; ++g) {
+      const int buf = g & 1;
+      if (!mbar_wait(&acc_full[buf], (g >> 1) & 1)) { failed = true; break; }
+      tc_fence_after();
+      const int t0 = g * G, t1 = min(n_tiles, t0 + G);
+      for (int t = t0; t < t1; ++t) {
+        const int vocab = v0 + t * kTileM + q * 32 + lane;
+        const bool valid = vocab < v1;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) +
+                                 (uint32_t)((buf * G + (t - t0)) * NPAD + c * 32),
+                             r);
+          tmem_ld_wait();
+          MSI s[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            s[j] = valid ? MSI{__uint_as_float(r[j]), 1.f, vocab} : msi_empty();
+          st[c] = msi_merge(st[c], reduce_scatter32(s, lane));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+    }
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) s_red[q * NPAD + c * 32 + lane] = st[c];
+    named_barrier_epilogue();
+    for (int col = threadIdx.x - 64; col < NPAD; col += 128) {
+      MSI m = s_red[col];
+#pragma unroll
+      for (int j = 1; j < 4; ++j) m = msi_merge(m, s_red[j * NPAD + col]);
+      if (col < a.R) {
+        Partial p;
+        p.m = m.m;
+        p.s = m.s;
+        p.i = m.i;
+        p.pad = 0;
+        a.part[(size_t)blockIdx.x * a.R + col] = p;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tp.tmem_cols);
+  }
+  if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
+  if (!last_cta_arrives(&a.ctrl->lm_ticket, a.n_cta)) return;
+  lm_final_merge(a);
+  if (threadIdx.x == 0) a.ctrl->lm_ticket = 0u;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 tensor map [outer, inner] (inner contiguous), 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+              uint32_t box_inner, uint32_t box_outer, CUtensorMapL2promotion promo) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NCH>
+cudaError_t launch_nch(const CUtensorMap& wf, const CUtensorMap& wp, const CUtensorMap& x,
+                       const LmArgs& a, const TcParams& tp, size_t smem, cudaStream_t s) {
+  auto k = lmhead_tc_kernel<NCH>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<a.n_cta, kThreads, smem, s>>>(wf, wp, x, a, tp);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Tiles per CTA, group size, ring depths and TMEM columns for a call.
+bool lmhead_tc_params(int R, int rows_per_cta, TcParams* tp, size_t* smem);
+
+bool lmhead_tc_params(int R, int rows_per_cta, TcParams* tp, size_t* smem) {
+  int nch = 1;
+  while (nch * 32 < R) nch *= 2;
+  if (nch > 8) return false;
+  tp->npad = nch * 32;
+  const int n_tiles = (rows_per_cta + kTileM - 1) / kTileM;
+  int G = (n_tiles + 2) / 3;
+  const int gmax = 256 / tp->npad;
+  if (G > gmax) G = gmax;
+  if (G < 1) G = 1;
+  tp->group = G;
+  uint32_t cols = 32;
+  while (cols < (uint32_t)(2 * G * tp->npad)) cols *= 2;
+  tp->tmem_cols = cols;
+  tp->stages_b = tp->npad <= 64 ? 4 : 2;
+  const size_t b_bytes = (size_t)tp->stages_b * tp->npad * 128;
+  const size_t budget = 200 * 1024;
+  int sa = (int)((budget - b_bytes) / kStageA);
+  if (sa > 12) sa = 12;
+  tp->stages_a = sa;
+  const size_t bars = 8 * (size_t)(2 * sa + 2 * tp->stages_b + 5) + 16;
+  *smem = 1024 + (size_t)sa * kStageA + b_bytes + bars + 4 * (size_t)tp->npad * sizeof(MSI);
+  return true;
+}
+
+cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s) {
+  TcParams tp;
+  size_t smem = 0;
+  if (!lmhead_tc_params(a.R, a.rows_per_cta, &tp, &smem)) return cudaErrorInvalidValue;
+  CUtensorMap wf, wp, x;
+  if (!make_map(&wf, a.w, a.H, a.V, kKChunk, kTileM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+      !make_map(&wp, a.w, a.H, a.V, kKChunk, kBoxPart, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+      !make_map(&x, a.rows, a.H, a.R, kKChunk, tp.npad, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+    return cudaErrorInvalidValue;
+  switch (tp.npad / 32) {
+    case 1: return launch_nch<1>(wf, wp, x, a, tp, smem, s);
+    case 2: return launch_nch<2>(wf, wp, x, a, tp, smem, s);
+    case 4: return launch_nch<4>(wf, wp, x, a, tp, smem, s);
+    case 8: return launch_nch<8>(wf, wp, x, a, tp, smem, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fdl

@@ -12,8 +12,9 @@ oracle and redraw the input row behind every active row whose
 * predicted token equals the mask id (a commit that leaves a mask),
 
 and, for a unit where the fallback fires, the row behind the best candidate
-when the two best confidences lie within ``CONF_MARGIN``.  We repeat until
-every margin holds and report how many rows were redrawn.
+when the two best confidences differ by less than ``CAND_REL`` of the best
+(relative, because fallback confidences can be ~1/V).  We repeat until every
+margin holds and report how many rows were redrawn.
 """
 from __future__ import annotations
 
@@ -25,6 +26,7 @@ from . import step
 
 GAP = 0.05
 CONF_MARGIN = 5e-3
+CAND_REL = 2e-3
 
 
 def _np(t, dtype=np.float64):
@@ -63,7 +65,7 @@ def _violations(case: synth.Case, res: dict):
                     or abs(res["conf"][b, i] - tau) < CONF_MARGIN
                     or res["tok"][b, i] == c["mask_id"]):
                 bad.add((b, i))
-        if res["cand_gap"][b] < CONF_MARGIN:
+        if res["cand_gap"][b] < CAND_REL:
             conf_b = np.where(act[b], res["conf"][b], -np.inf)
             bad.add((b, int(np.argmax(conf_b))))
     return sorted(bad)

@@ -279,12 +279,13 @@ def denoise_step(c: dict, q, k_pre, v_pre, len_pre, prompt_len, k_blk, v_blk,
     new, committed, n_comm, n_left = threshold_commit(bt, conf, tok, q_off, q_len,
                                                       mask_id, tau)
     # Decision margins: logit gap and |conf - tau| per active row; the
-    # confidence gap between the two best candidates where the fallback fires.
+    # relative confidence gap between the two best candidates where the
+    # fallback fires.
     cand_gap = np.full(B, np.inf)
     for b in range(B):
         cs = sorted(conf[b][active[b]], reverse=True)
         if len(cs) >= 2 and cs[0] < tau:
-            cand_gap[b] = cs[0] - cs[1]
+            cand_gap[b] = (cs[0] - cs[1]) / cs[0]
     return dict(attn=attn, attn_rounded=attn_r, rows=rows, active=active,
                 conf=conf, tok=tok, logit_gap=gap, block_tokens=new,
                 committed=committed, n_committed=n_comm, n_masked_left=n_left,

@@ -188,3 +188,32 @@ def test_sweep_full_size(batch, prefix):
     case, ref, _ = cases.parity_case("sweep", 0, cfg=cfg)
     gpu = gh.run_denoise_step(case)
     gh.compare_step(case, gpu, ref, check_attn=True)
+
+
+# ---------------------------------------------- LM head shapes and tails
+
+@pytest.mark.parametrize("R,V,H", [(1, 5000, 64), (32, 5000, 448), (33, 33000, 128),
+                                   (128, 20000, 256), (256, 7001, 64), (8, 151936, 1536)])
+def test_lmhead_shapes_against_oracle(R, V, H):
+    """Every N padding (32..256), partial vocab tiles (5000 / 148 CTAs = 48
+    rows each), ragged vocab ends and several K depths.  Tokens must match
+    wherever the oracle's top-2 logit gap exceeds 1e-3 (fp32 accumulation
+    error is ~1e-5 at these sizes); confidences within 1e-3 relative."""
+    g = torch.Generator().manual_seed(R * 7 + V + H)
+    rows = torch.randn((R, H), generator=g).to(torch.bfloat16)
+    w = (torch.randn((V, H), generator=g) * (8.0 / H ** 0.5)).to(torch.bfloat16)
+    cfg = fdl.make_cfg(dict(batch=R, n_q_heads=1, n_kv_heads=1, head_dim=32,
+                            block_size=1, q_off=0, q_len=1, cap_prefix=0, hidden=H,
+                            vocab=V, mask_id=V - 1, shift=0, tau=0.9, dtype="bf16"))
+    conf = torch.empty(R, dtype=torch.float32, device="cuda")
+    tok = torch.empty(R, dtype=torch.int32, device="cuda")
+    ws = fdl.workspace(cfg)
+    for _ in range(2):                       # the second call reuses the workspace
+        fdl.lmhead_confidence(cfg, rows.cuda(), w.cuda(), None, conf, tok, ws)
+        torch.cuda.synchronize()
+        t_ref, c_ref, gap = step.lmhead_confidence(rows.double().numpy(), w.float().numpy())
+        t_gpu = tok.cpu().numpy()
+        sure = gap > 1e-3
+        assert np.array_equal(t_gpu[sure], t_ref[sure])
+        np.testing.assert_allclose(conf.cpu().numpy().astype(np.float64), c_ref, rtol=1e-3)
+    assert fdl.get_status(ws) == 0
