@@ -169,14 +169,20 @@ def barrier(world):
         dist.barrier(device_ids=[torch.cuda.current_device()])
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's time: every rank's number, max-reduced."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank decodes its own batch of sequences (weak scaling)."""
+    return seed + 7919 * rank
 
 
 def run_reference(args):
@@ -238,7 +244,7 @@ def main():
 
     world, rank, local = dist_setup()
     peaks = measured_peaks()
-    case = synth.make_case(WORKLOAD, args.seed + rank)
+    case = synth.make_case(WORKLOAD, rank_seed(args.seed, rank))
     c = case.cfg
     cfg = fdl.make_cfg(c)
     B, q_len, H, V = c["batch"], c["q_len"], c["hidden"], c["vocab"]

@@ -1,0 +1,678 @@
+// Block-wise attention on the 5th-generation tensor cores (bf16, d = 128).
+//
+// The active unit's queries attend to [prefix cache | block rows | suffix
+// cache] ("Fast-dLLM v2" section 3.4, Figure 7b and Level 3; technical review
+// eq. (3) and section 3).  One (sequence, KV head, query-row tile) is an
+// item: its rows are the unit's q_len positions x the group of query heads
+// sharing the KV head (GQA packing: 8 x 7 = 56 rows at Qwen2.5-7B shapes),
+// padded to the M = 128 tile.
+//
+// Stream-K split: every CTA (one per SM) reads the per-sequence lengths,
+// cuts the concatenation of all items' 64-key chunks into equal contiguous
+// ranges and takes its own, so the split follows the actual lengths and a CTA
+// produces at most two partial results (its first and last item); items it
+// covers whole are written out directly.  Per chunk:
+//   warp 0   TMA: K and V [64 keys x 128] in four 8 KB boxes (128-byte
+//            swizzle) through a 3-slot ring; Q of each item by a 3D box
+//            (d, head group, positions) into one of two Q buffers;
+//   warp 1   tcgen05.mma: S = Q K^T (M 128, N 64, K 128) into one of two TMEM
+//            S buffers, then, one chunk behind, O += P V (M 128, N 128, K 64,
+//            V read MN-major) into the item's TMEM O buffer;
+//   warps 2-5  softmax, one thread per row: S from TMEM, online max with a
+//            lazy rescale (O in TMEM is rescaled only when the running max
+//            grows by more than 2^8), P = exp2(S - m) as bf16 into shared
+//            memory (swizzled K-major), and the item epilogue.
+// Partial results (unnormalised O, m, l) go to the workspace; the last CTA
+// to finish an item merges them.  No thread waits on another CTA.
+#include <cudaTypedefs.h>
+
+#include "fdl_common.cuh"
+#include "sm100.cuh"
+
+namespace fdl {
+namespace {
+
+using namespace sm100;
+
+constexpr int kCh = 64;                  // keys per chunk
+constexpr int kQRegion = 128 * 128;      // 128 rows x 64 bf16 (16 KB)
+constexpr int kQBuf = 2 * kQRegion;      // d 0-63 and 64-127
+constexpr int kKVRegion = kCh * 128;     // 64 keys x 64 bf16 (8 KB)
+constexpr int kKVSlot = 4 * kKVRegion;   // K lo, K hi, V lo, V hi
+constexpr int kPBuf = 128 * 128;         // 128 rows x 64 keys bf16 (16 KB)
+constexpr int kStages = 3;
+constexpr int kThreads = 192;
+constexpr float kRescale = 8.0f;         // log2-domain growth forcing a rescale
+constexpr unsigned kDevTimeout = 4u;
+constexpr int kMaxSeq = 256;
+
+struct TcArgs {
+  int B, Hq, Hkv, q_len, D, cap_p, cap_s, group, qpt, n_rt, n_cta, dual;
+  float scale_log2;
+  const int32_t* len_pre;
+  const int32_t* len_suf;
+  bf16* out;
+  Control* ctrl;
+  unsigned int* tickets;  // one per item
+  float* part_o;          // [2 * n_cta][128][128]
+  float2* part_ml;        // [2 * n_cta][128]
+};
+
+struct Maps {
+  CUtensorMap q, kp, vp, kb, vb, ks, vs;
+};
+
+struct Smem {
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full[2], p_empty[2];
+  uint64_t pv_done;
+  uint64_t o_full[2], o_empty[2];
+  uint64_t drain;
+  uint32_t tmem;
+  int flag;
+  int cb[kMaxSeq + 1];  // first global chunk of sequence b
+  int nc[kMaxSeq];      // chunks per item of sequence b
+  int lp[kMaxSeq];
+  int ls[kMaxSeq];
+};
+
+// Position in the chunk sequence of one CTA.
+struct Cursor {
+  int b, it, j;  // sequence, item within sequence, chunk within item
+};
+
+__device__ __forceinline__ Cursor locate(const Smem& S, int B, int per_seq, long long g) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {  // last b with cb[b] <= g
+    const int mid = (lo + hi + 1) >> 1;
+    if (S.cb[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  const int rem = (int)(g - S.cb[lo]);
+  Cursor c;
+  c.b = lo;
+  c.it = rem / S.nc[lo];
+  c.j = rem % S.nc[lo];
+  (void)per_seq;
+  return c;
+}
+
+__device__ __forceinline__ void advance(Cursor& c, const Smem& S, int per_seq) {
+  if (++c.j == S.nc[c.b]) {
+    c.j = 0;
+    if (++c.it == per_seq) {
+      c.it = 0;
+      ++c.b;
+    }
+  }
+}
+
+// CTA owning global chunk g: the largest i with floor(T i / n) <= g.
+__device__ __forceinline__ int cta_of(long long g, long long T, int n) {
+  return (int)(((g + 1) * n - 1) / T);
+}
+
+__device__ __forceinline__ long long cta_start(int i, long long T, int n) {
+  return T * i / n;
+}
+
+// With fewer chunks than CTAs some ranges are empty; only non-empty ones
+// between the first and last owner of an item touched it.
+__device__ __forceinline__ bool cta_nonempty(int i, long long T, int n) {
+  return cta_start(i, T, n) < cta_start(i + 1, T, n);
+}
+
+struct ChunkInfo {
+  int seg;     // 0 prefix, 1 block, 2 suffix
+  int key0;    // first key of the chunk within its segment
+  int nvalid;  // valid keys in the chunk
+};
+
+__device__ __forceinline__ ChunkInfo chunk_info(int j, int Lp, int Ls, int D) {
+  const int ncp = (Lp + kCh - 1) / kCh;
+  ChunkInfo ci;
+  if (j < ncp) {
+    ci.seg = 0;
+    ci.key0 = j * kCh;
+    ci.nvalid = min(kCh, Lp - ci.key0);
+  } else if (j == ncp) {
+    ci.seg = 1;
+    ci.key0 = 0;
+    ci.nvalid = D;
+  } else {
+    ci.seg = 2;
+    ci.key0 = (j - ncp - 1) * kCh;
+    ci.nvalid = min(kCh, Ls - ci.key0);
+  }
+  (void)Ls;
+  return ci;
+}
+
+__device__ __forceinline__ void named_barrier_softmax() {
+  asm volatile("bar.sync 2, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_smem = base;                       // 2 x 32 KB
+  uint8_t* kv_smem = q_smem + 2 * kQBuf;        // 3 x 32 KB
+  uint8_t* p_smem = kv_smem + kStages * kKVSlot;  // 2 x 16 KB
+  Smem& S = *reinterpret_cast<Smem*>(p_smem + 2 * kPBuf);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per_seq = a.Hkv * a.n_rt;  // items per sequence
+  const int rows_full = a.qpt * a.group;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&S.kv_full[i], 1);
+      mbar_init(&S.kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.q_full[i], 1);
+      mbar_init(&S.q_empty[i], 1);
+      mbar_init(&S.s_full[i], 1);
+      mbar_init(&S.s_empty[i], 128);
+      mbar_init(&S.p_full[i], 128);
+      mbar_init(&S.p_empty[i], 1);
+      mbar_init(&S.o_full[i], 1);
+      mbar_init(&S.o_empty[i], 128);
+    }
+    mbar_init(&S.pv_done, 1);
+    mbar_init(&S.drain, 1);
+    fence_barrier_init();
+    // Sequence table from the device-resident lengths.
+    long long run = 0;
+    for (int b = 0; b < a.B; ++b) {
+      int Lp = a.len_pre[b];
+      if (Lp < 0 || Lp > a.cap_p) {
+        if (blockIdx.x == 0) atomicOr(&a.ctrl->status, FDL_DEV_BAD_PREFIX_LEN);
+        Lp = 0;
+      }
+      int Ls = 0;
+      if (a.dual) {
+        Ls = a.len_suf[b];
+        if (Ls < 0 || Ls > a.cap_s) {
+          if (blockIdx.x == 0) atomicOr(&a.ctrl->status, FDL_DEV_BAD_SUFFIX_LEN);
+          Ls = 0;
+        }
+      }
+      S.lp[b] = Lp;
+      S.ls[b] = Ls;
+      S.nc[b] = (Lp + kCh - 1) / kCh + 1 + (Ls + kCh - 1) / kCh;
+      S.cb[b] = (int)run;
+      run += (long long)S.nc[b] * per_seq;
+    }
+    S.cb[a.B] = (int)run;
+  }
+  // Padding rows of both Q buffers are never written by TMA: zero them once.
+  for (int t = threadIdx.x; t < 2 * 2 * (128 - rows_full) * 8; t += kThreads) {
+    const int per_region = (128 - rows_full) * 8;
+    const int region = t / per_region, w = t % per_region;
+    const int row = rows_full + w / 8, chunk = w % 8;
+    *reinterpret_cast<uint4*>(q_smem + region * kQRegion + row * 128 + chunk * 16) =
+        make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
+  if (warp == 1) tmem_alloc(&S.tmem, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem;
+
+  const long long T = S.cb[a.B];
+  const int n = a.n_cta;
+  const long long c_begin = cta_start(blockIdx.x, T, n);
+  const long long c_end = cta_start(blockIdx.x + 1, T, n);
+  bool failed = false;
+
+  if (c_begin < c_end && warp == 0) {
+    // -------------------------------------------------------------- TMA
+    if (lane == 0) {
+      int kv_i = 0, q_i = 0, prev_x = -1;
+      Cursor c = locate(S, a.B, per_seq, c_begin);
+      for (long long g = c_begin; g < c_end && !failed; ++g, advance(c, S, per_seq)) {
+        const int x = c.b * per_seq + c.it;
+        const int kvh = c.it / a.n_rt, rt = c.it % a.n_rt;
+        if (x != prev_x) {
+          const int qb = q_i & 1;
+          if (!mbar_wait(&S.q_empty[qb], ((q_i >> 1) & 1) ^ 1)) { failed = true; break; }
+          mbar_arrive_expect_tx(&S.q_full[qb], 2u * 128u * (uint32_t)rows_full);
+          const int z = c.b * a.q_len + rt * a.qpt;
+          tma_load_3d(q_smem + qb * kQBuf, &maps.q, 0, kvh * a.group, z, &S.q_full[qb]);
+          tma_load_3d(q_smem + qb * kQBuf + kQRegion, &maps.q, 64, kvh * a.group, z,
+                      &S.q_full[qb]);
+          ++q_i;
+          prev_x = x;
+        }
+        const int slot = kv_i % kStages;
+        if (!mbar_wait(&S.kv_empty[slot], ((kv_i / kStages) & 1) ^ 1)) { failed = true; break; }
+        const ChunkInfo ci = chunk_info(c.j, S.lp[c.b], S.ls[c.b], a.D);
+        const CUtensorMap* mk;
+        const CUtensorMap* mv;
+        int row;
+        const int bk = c.b * a.Hkv + kvh;
+        if (ci.seg == 0) {
+          mk = &maps.kp; mv = &maps.vp; row = bk * a.cap_p + ci.key0;
+        } else if (ci.seg == 1) {
+          mk = &maps.kb; mv = &maps.vb; row = bk * a.D;
+        } else {
+          mk = &maps.ks; mv = &maps.vs; row = bk * a.cap_s + ci.key0;
+        }
+        uint8_t* dst = kv_smem + slot * kKVSlot;
+        mbar_arrive_expect_tx(&S.kv_full[slot], kKVSlot);
+        tma_load_2d(dst, mk, 0, row, &S.kv_full[slot]);
+        tma_load_2d(dst + kKVRegion, mk, 64, row, &S.kv_full[slot]);
+        tma_load_2d(dst + 2 * kKVRegion, mv, 0, row, &S.kv_full[slot]);
+        tma_load_2d(dst + 3 * kKVRegion, mv, 64, row, &S.kv_full[slot]);
+        ++kv_i;
+      }
+      for (int m = max(0, kv_i - kStages); m < kv_i; ++m)
+        if (!mbar_wait(&S.kv_full[m % kStages], (m / kStages) & 1)) failed = true;
+      for (int m = max(0, q_i - 2); m < q_i; ++m)
+        if (!mbar_wait(&S.q_full[m & 1], (m >> 1) & 1)) failed = true;
+    }
+  } else if (c_begin < c_end && warp == 1) {
+    // -------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16_f32(128, kCh);
+      const uint32_t id_pv = idesc_bf16_f32(128, 128) | (1u << 16);  // V is MN-major
+      int kv_i = 0, q_i = 0, s_i = 0, pv_i = 0, o_i = 0, prev_x = -1;
+      // pending P V of the previous chunk
+      bool pend = false;
+      int pend_slot = 0, pend_first = 0, pend_last = 0;
+      auto issue_pv = [&](int slot, int first, int last) -> bool {
+        const int pb = pv_i & 1;
+        if (!mbar_wait(&S.p_full[pb], (pv_i >> 1) & 1)) return false;
+        const int ob = o_i & 1;
+        if (first && !mbar_wait(&S.o_empty[ob], ((o_i >> 1) & 1) ^ 1)) return false;
+        tc_fence_after();
+        const uint32_t p_base = smem_u32(p_smem + pb * kPBuf);
+        const uint32_t v_base = smem_u32(kv_smem + slot * kKVSlot + 2 * kKVRegion);
+        const uint32_t d_o = tmem + 128u + (uint32_t)ob * 128u;
+#pragma unroll
+        for (int k = 0; k < kCh / 16; ++k)
+          mma_bf16(d_o, desc_k_sw128(p_base + k * 32),
+                   desc_mn_sw128(v_base + k * 2048, kKVRegion, 1024), id_pv,
+                   (first && k == 0) ? 0u : 1u);
+        mma_commit(&S.kv_empty[slot]);
+        mma_commit(&S.p_empty[pb]);
+        mma_commit(&S.pv_done);
+        if (last) {
+          mma_commit(&S.o_full[ob]);
+          ++o_i;
+        }
+        ++pv_i;
+        return true;
+      };
+      Cursor c = locate(S, a.B, per_seq, c_begin);
+      for (long long g = c_begin; g < c_end && !failed; ++g, advance(c, S, per_seq)) {
+        const int x = c.b * per_seq + c.it;
+        const int first = x != prev_x;
+        const int last = (g + 1 == c_end) || (c.j + 1 == S.nc[c.b]);
+        if (first) {
+          if (!mbar_wait(&S.q_full[q_i & 1], (q_i >> 1) & 1)) { failed = true; break; }
+          ++q_i;
+          prev_x = x;
+        }
+        const int qb = (q_i - 1) & 1;
+        const int slot = kv_i % kStages;
+        if (!mbar_wait(&S.kv_full[slot], (kv_i / kStages) & 1)) { failed = true; break; }
+        const int sb = s_i & 1;
+        if (!mbar_wait(&S.s_empty[sb], ((s_i >> 1) & 1) ^ 1)) { failed = true; break; }
+        tc_fence_after();
+        const uint32_t q_base = smem_u32(q_smem + qb * kQBuf);
+        const uint32_t k_base = smem_u32(kv_smem + slot * kKVSlot);
+        const uint32_t d_s = tmem + (uint32_t)sb * kCh;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_bf16(d_s, desc_k_sw128(q_base + (k >> 2) * kQRegion + (k & 3) * 32),
+                   desc_k_sw128(k_base + (k >> 2) * kKVRegion + (k & 3) * 32), id_s,
+                   k ? 1u : 0u);
+        mma_commit(&S.s_full[sb]);
+        if (last) mma_commit(&S.q_empty[qb]);
+        ++s_i;
+        if (pend && !issue_pv(pend_slot, pend_first, pend_last)) { failed = true; break; }
+        pend = true;
+        pend_slot = slot;
+        pend_first = first;
+        pend_last = last;
+        ++kv_i;
+      }
+      if (pend && !failed && !issue_pv(pend_slot, pend_first, pend_last)) failed = true;
+      mma_commit(&S.drain);
+      if (!mbar_wait(&S.drain, 0)) failed = true;
+    }
+  } else if (c_begin < c_end && warp >= 2) {
+    // ------------------------------------------------- softmax + epilogue
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;  // TMEM lane = tile row
+    const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+    float m_used = kEmptyMax, l = 0.f;
+    int s_i = 0, o_i = 0, prev_x = -1;
+    const int first_x = [&] {
+      const Cursor c0 = locate(S, a.B, per_seq, c_begin);
+      return c0.b * per_seq + c0.it;
+    }();
+    Cursor c = locate(S, a.B, per_seq, c_begin);
+    for (long long g = c_begin; g < c_end && !failed; ++g, advance(c, S, per_seq)) {
+      const int x = c.b * per_seq + c.it;
+      const int first = x != prev_x;
+      const int last = (g + 1 == c_end) || (c.j + 1 == S.nc[c.b]);
+      const int kvh = c.it / a.n_rt, rt = c.it % a.n_rt;
+      const int qpt_eff = min(a.qpt, a.q_len - rt * a.qpt);
+      const int rows = qpt_eff * a.group;
+      const bool warp_active = q4 * 32 < rows;
+      if (first) {
+        m_used = kEmptyMax;
+        l = 0.f;
+        prev_x = x;
+      }
+      const ChunkInfo ci = chunk_info(c.j, S.lp[c.b], S.ls[c.b], a.D);
+      const int sb = s_i & 1;
+      if (!mbar_wait(&S.s_full[sb], (s_i >> 1) & 1)) { failed = true; break; }
+      tc_fence_after();
+      uint32_t sr[64];
+      if (warp_active) {
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        tmem_ld_32x32b_x32(tmem + lane_addr + (uint32_t)sb * kCh, lo);
+        tmem_ld_32x32b_x32(tmem + lane_addr + (uint32_t)sb * kCh + 32, hi);
+        tmem_ld_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(&S.s_empty[sb]);
+      const int pb = s_i & 1;
+      if (!mbar_wait(&S.p_empty[pb], ((s_i >> 1) & 1) ^ 1)) { failed = true; break; }
+      if (warp_active) {
+        float xs[64];
+        float cmax = kEmptyMax;
+#pragma unroll
+        for (int jj = 0; jj < 64; ++jj) {
+          xs[jj] = jj < ci.nvalid ? __uint_as_float(sr[jj]) * a.scale_log2 : kEmptyMax;
+          cmax = fmaxf(cmax, xs[jj]);
+        }
+        float alpha = 1.f;
+        if (first) {
+          m_used = cmax;
+        } else if (cmax > m_used + kRescale) {
+          alpha = exp2f(m_used - cmax);
+          m_used = cmax;
+        }
+        // O rescale (warp-collective TMEM access) when any row needs it.
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+          if (!mbar_wait(&S.pv_done, (s_i - 1) & 1)) { failed = true; }
+          tc_fence_after();
+          const uint32_t o_addr = tmem + lane_addr + 128u + (uint32_t)(o_i & 1) * 128u;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t ov[32];
+            tmem_ld_32x32b_x32(o_addr + cc * 32, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) ov[jj] = __float_as_uint(__uint_as_float(ov[jj]) * alpha);
+            tmem_st_32x32b_x32(o_addr + cc * 32, ov);
+          }
+          tmem_st_wait();
+        }
+        l *= alpha;
+        float psum = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int jj = 0; jj < 64; jj += 2) {
+          const float p0 = exp2f(xs[jj] - m_used);
+          const float p1 = exp2f(xs[jj + 1] - m_used);
+          psum += p0 + p1;
+          pk[jj >> 1] = pack_bf16(p0, p1);
+        }
+        l += psum;
+        uint8_t* prow = p_smem + pb * kPBuf + r * 128;
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          *reinterpret_cast<uint4*>(prow + ((t ^ (r & 7)) * 16)) =
+              make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      mbar_arrive(&S.p_full[pb]);
+      ++s_i;
+      if (failed) break;
+      if (!last) continue;
+
+      // ----------------------------------------------------- item epilogue
+      const int ob = o_i & 1;
+      if (!mbar_wait(&S.o_full[ob], (o_i >> 1) & 1)) { failed = true; break; }
+      tc_fence_after();
+      const long long x_start = S.cb[c.b] + (long long)c.it * S.nc[c.b];
+      const long long x_end = x_start + S.nc[c.b];
+      const int cta_lo = cta_of(x_start, T, n), cta_hi = cta_of(x_end - 1, T, n);
+      const int p_pos = r / a.group, jh = r % a.group;
+      const int qi = rt * a.qpt + p_pos;
+      const bool row_ok = r < rows;
+      bf16* orow = a.out + (((size_t)c.b * a.q_len + qi) * a.Hq + kvh * a.group + jh) * 128;
+      const uint32_t o_addr = tmem + lane_addr + 128u + (uint32_t)ob * 128u;
+      if (cta_lo == cta_hi) {
+        const float inv = 1.f / l;
+        if (warp_active) {
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t ov[32];
+            tmem_ld_32x32b_x32(o_addr + cc * 32, ov);
+            tmem_ld_wait();
+            if (row_ok) {
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                uint4 v;
+                v.x = pack_bf16(__uint_as_float(ov[8 * t + 0]) * inv, __uint_as_float(ov[8 * t + 1]) * inv);
+                v.y = pack_bf16(__uint_as_float(ov[8 * t + 2]) * inv, __uint_as_float(ov[8 * t + 3]) * inv);
+                v.z = pack_bf16(__uint_as_float(ov[8 * t + 4]) * inv, __uint_as_float(ov[8 * t + 5]) * inv);
+                v.w = pack_bf16(__uint_as_float(ov[8 * t + 6]) * inv, __uint_as_float(ov[8 * t + 7]) * inv);
+                *reinterpret_cast<uint4*>(orow + cc * 32 + 8 * t) = v;
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&S.o_empty[ob]);
+        ++o_i;
+        continue;
+      }
+      // Partial of this CTA: slot 2*cta for its first item, 2*cta+1 otherwise.
+      const int slot = 2 * blockIdx.x + (x == first_x ? 0 : 1);
+      float* po = a.part_o + ((size_t)slot * 128 + r) * 128;
+      if (warp_active) {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t ov[32];
+          tmem_ld_32x32b_x32(o_addr + cc * 32, ov);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              *reinterpret_cast<uint4*>(po + cc * 32 + 4 * t) =
+                  make_uint4(ov[4 * t], ov[4 * t + 1], ov[4 * t + 2], ov[4 * t + 3]);
+          }
+        }
+        if (row_ok) a.part_ml[(size_t)slot * 128 + r] = make_float2(m_used, l);
+      }
+      tc_fence_before();
+      mbar_arrive(&S.o_empty[ob]);
+      ++o_i;
+      __threadfence();
+      named_barrier_softmax();
+      if (threadIdx.x == 64) {
+        int n_touch = 0;
+        for (int j2 = cta_lo; j2 <= cta_hi; ++j2) n_touch += cta_nonempty(j2, T, n);
+        const unsigned prev = atomicAdd(&a.tickets[x], 1u);
+        S.flag = prev == (unsigned)(n_touch - 1);
+      }
+      named_barrier_softmax();
+      if (!S.flag) continue;
+      __threadfence();
+      if (row_ok) {
+        float M = kEmptyMax;
+        for (int j2 = cta_lo; j2 <= cta_hi; ++j2) {
+          if (!cta_nonempty(j2, T, n)) continue;
+          const int s2 = 2 * j2 + ((j2 == cta_lo && cta_start(j2, T, n) != x_start) ? 1 : 0);
+          M = fmaxf(M, __ldcg(&a.part_ml[(size_t)s2 * 128 + r]).x);
+        }
+        float L = 0.f;
+        float acc[128];
+#pragma unroll
+        for (int t = 0; t < 128; ++t) acc[t] = 0.f;
+        for (int j2 = cta_lo; j2 <= cta_hi; ++j2) {
+          if (!cta_nonempty(j2, T, n)) continue;
+          const int s2 = 2 * j2 + ((j2 == cta_lo && cta_start(j2, T, n) != x_start) ? 1 : 0);
+          const float2 ml = __ldcg(&a.part_ml[(size_t)s2 * 128 + r]);
+          const float w = exp2f(ml.x - M);
+          L += ml.y * w;
+          const float4* src = reinterpret_cast<const float4*>(a.part_o + ((size_t)s2 * 128 + r) * 128);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const float4 v = __ldcg(src + t);
+            acc[4 * t] += v.x * w;
+            acc[4 * t + 1] += v.y * w;
+            acc[4 * t + 2] += v.z * w;
+            acc[4 * t + 3] += v.w * w;
+          }
+        }
+        const float inv = 1.f / L;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          uint4 v;
+          v.x = pack_bf16(acc[8 * t + 0] * inv, acc[8 * t + 1] * inv);
+          v.y = pack_bf16(acc[8 * t + 2] * inv, acc[8 * t + 3] * inv);
+          v.z = pack_bf16(acc[8 * t + 4] * inv, acc[8 * t + 5] * inv);
+          v.w = pack_bf16(acc[8 * t + 6] * inv, acc[8 * t + 7] * inv);
+          *reinterpret_cast<uint4*>(orow + 8 * t) = v;
+        }
+      }
+      if (threadIdx.x == 64) a.tickets[x] = 0u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Rows of 128 bf16 (256 B), box [64 d x 64 rows], 128-byte swizzle.
+bool map_rows(CUtensorMap* m, const void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {64, kCh};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// Q [B*q_len, Hq, 128] as a 3D map; box [64 d, group heads, qpt positions].
+bool map_q(CUtensorMap* m, const void* base, int Hq, int BQ, int group, int qpt) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)Hq, (cuuint64_t)BQ};
+  cuuint64_t strides[2] = {256, (cuuint64_t)Hq * 256};
+  cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)qpt};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// Query positions per 128-row tile for a GQA group; 0 if unsupported.
+int attn_tc_qpt(int q_len, int group) {
+  if (group > 128) return 0;
+  const int qpt = 128 / group;
+  return qpt < q_len ? qpt : q_len;
+}
+
+size_t attn_tc_smem_bytes() {
+  return 1024 + 2 * kQBuf + kStages * kKVSlot + 2 * kPBuf + sizeof(Smem);
+}
+
+cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
+                           unsigned int* tickets, int n_cta, cudaStream_t s) {
+  const int qpt = attn_tc_qpt(a.q_len, a.group);
+  if (a.d != 128 || qpt == 0 || a.B > kMaxSeq) return cudaErrorInvalidValue;
+  Maps maps;
+  const uint64_t bk = (uint64_t)a.B * a.Hkv;
+  bool ok = map_q(&maps.q, a.q, a.Hq, a.B * a.q_len, a.group, qpt) &&
+            map_rows(&maps.kb, a.k_blk, bk * a.D) && map_rows(&maps.vb, a.v_blk, bk * a.D);
+  if (a.cap_p > 0) {
+    ok = ok && map_rows(&maps.kp, a.k_pre, bk * a.cap_p) &&
+         map_rows(&maps.vp, a.v_pre, bk * a.cap_p);
+  } else {
+    maps.kp = maps.kb;
+    maps.vp = maps.vb;
+  }
+  if (a.k_suf != nullptr) {
+    ok = ok && map_rows(&maps.ks, a.k_suf, bk * a.cap_s) &&
+         map_rows(&maps.vs, a.v_suf, bk * a.cap_s);
+  } else {
+    maps.ks = maps.kb;
+    maps.vs = maps.vb;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  TcArgs t;
+  t.B = a.B;
+  t.Hq = a.Hq;
+  t.Hkv = a.Hkv;
+  t.q_len = a.q_len;
+  t.D = a.D;
+  t.cap_p = a.cap_p;
+  t.cap_s = a.cap_s;
+  t.group = a.group;
+  t.qpt = qpt;
+  t.n_rt = (a.q_len + qpt - 1) / qpt;
+  t.n_cta = n_cta;
+  t.dual = a.k_suf != nullptr;
+  t.scale_log2 = a.scale_log2;
+  t.len_pre = a.len_pre;
+  t.len_suf = a.len_suf;
+  t.out = static_cast<bf16*>(a.out);
+  t.ctrl = a.ctrl;
+  t.tickets = tickets;
+  t.part_o = part_o;
+  t.part_ml = part_ml;
+  const size_t smem = attn_tc_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<<<n_cta, kThreads, smem, s>>>(maps, t);
+  return cudaGetLastError();
+}
+
+}  // namespace fdl

@@ -128,7 +128,12 @@ int run_attention(const fdl_step_cfg& c, const Plan& p, bool dual, const void* q
                   cudaStream_t s) {
   AttnArgs a = attn_args(c, p, dual, q, k_pre, v_pre, len_pre, k_blk, v_blk,
                          k_suf, v_suf, len_suf, out, ws);
-  cudaError_t e = launch_attn_simt(a, (fdl_dtype)c.dtype, kAttnRowTile, s);
+  // bf16 with d = 128: tensor-core kernel; otherwise the CUDA-core kernel.
+  cudaError_t e = p.attn_tc
+                      ? launch_attn_tc(a, at<float>(ws, p.off_tc_part_o),
+                                       at<float2>(ws, p.off_tc_part_ml), a.tickets,
+                                       kPlanCTAs, s)
+                      : launch_attn_simt(a, (fdl_dtype)c.dtype, kAttnRowTile, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return FDL_OK;
 }

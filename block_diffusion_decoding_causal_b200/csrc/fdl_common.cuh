@@ -175,6 +175,8 @@ __device__ __forceinline__ void commit_sequence_warp(
 // Host-side launchers (one .cu file each).
 cudaError_t launch_attn_simt(const AttnArgs& a, fdl_dtype dt, int row_tile,
                              cudaStream_t s);
+cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
+                           unsigned int* tickets, int n_cta, cudaStream_t s);
 cudaError_t launch_lmhead_simt(const LmArgs& a, fdl_dtype dt, cudaStream_t s);
 cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s);
 cudaError_t launch_commit(const float* conf, const int32_t* tok,

@@ -25,8 +25,9 @@ struct Plan {
   AttnSplit attn_plain, attn_dual;
   int lm_cta, lm_rows_per_cta;        // CUDA-core LM head (fp32)
   int lm_tc_cta, lm_tc_rows_per_cta;  // tensor-core LM head (bf16): one CTA per SM
+  bool attn_tc;     // tensor-core attention (bf16, d 128)
   size_t off_ctrl, off_tickets, off_part_o, off_part_ml, off_rows, off_lm_part,
-      off_attn, total;
+      off_attn, off_tc_part_o, off_tc_part_ml, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -109,6 +110,15 @@ inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why) {
   off = align256(off + 16 * (size_t)kLmMaxCTAs * R);
   p->off_attn = off;
   off = align256(off + (size_t)p->elem * R * c->n_q_heads * c->head_dim);
+  // Tensor-core attention: at most two partials (first and last item) per CTA.
+  p->attn_tc = c->dtype == FDL_BF16 && c->head_dim == 128 && group <= 128 && c->batch <= 256;
+  p->off_tc_part_o = off;
+  p->off_tc_part_ml = off;
+  if (p->attn_tc) {
+    off = align256(off + sizeof(float) * 2 * (size_t)kPlanCTAs * 128 * 128);
+    p->off_tc_part_ml = off;
+    off = align256(off + 8 * 2 * (size_t)kPlanCTAs * 128);
+  }
   p->total = off;
   return true;
 }

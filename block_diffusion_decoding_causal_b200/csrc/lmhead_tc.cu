@@ -8,8 +8,9 @@
 // Swap-AB: the weight is the M = 128 operand (a tile of 128 vocabulary rows),
 // the <= 256 input rows are N.  Each CTA (one per SM) owns a contiguous
 // vocabulary range of ~V/148 rows and streams it once:
-//   warp 0   TMA producer: W tiles [128 x 64] (128-byte swizzle) through an
-//            A ring, X chunks [N x 64] through a B ring;
+//   warp 0   TMA producer: W tiles [128 x 64*KSUB] (KSUB boxes of 128-byte
+//            swizzled rows, so each weight row is read 512 contiguous bytes at
+//            a time) through an A ring, X chunks [N x 64*KSUB] through a B ring;
 //   warp 1   MMA issuer: tcgen05.mma kind::f16, accumulators in TMEM; tiles
 //            are processed in groups of G, K-outer inside a group so each X
 //            chunk is reused by G tiles; two TMEM buffers let the epilogue
@@ -38,6 +39,7 @@ constexpr unsigned kDevTimeout = 4u;        // status bit: a bounded wait expire
 
 struct TcParams {
   int npad;        // MMA N: 32, 64, 128 or 256
+  int ksub;        // 64-wide K boxes per pipeline stage
   int group;       // tiles per TMEM buffer
   int stages_a;
   int stages_b;
@@ -64,20 +66,22 @@ __device__ __forceinline__ MSI reduce_scatter32(MSI (&s)[32], int lane) {
   return s[0];
 }
 
-template <int NCH>
+template <int NCH, int KSUB>
 __global__ void __launch_bounds__(kThreads, 1)
 lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
                  const __grid_constant__ CUtensorMap tm_w_part,
                  const __grid_constant__ CUtensorMap tm_x, const LmArgs a,
                  const TcParams tp) {
   constexpr int NPAD = NCH * 32;
+  constexpr int SA_BYTES = kStageA * KSUB;        // one A stage: 128 rows x 64*KSUB
+  constexpr int SB_BYTES = NPAD * 128 * KSUB;     // one B stage: NPAD rows x 64*KSUB
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int SA = tp.stages_a, SB = tp.stages_b;
   uint8_t* sa = smem;
-  uint8_t* sb = sa + SA * kStageA;
-  uint64_t* full_a = reinterpret_cast<uint64_t*>(sb + SB * NPAD * 128);
+  uint8_t* sb = sa + SA * SA_BYTES;
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(sb + SB * SB_BYTES);
   uint64_t* empty_a = full_a + SA;
   uint64_t* full_b = empty_a + SA;
   uint64_t* empty_b = full_b + SB;
@@ -94,7 +98,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
   const int n_tiles = (n_rows + kTileM - 1) / kTileM;
   const int G = tp.group;
   const int n_groups = (n_tiles + G - 1) / G;
-  const int KC = a.H / kKChunk;
+  const int KC = a.H / (kKChunk * KSUB);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SA; ++i) {
@@ -132,24 +136,32 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
         for (int kc = 0; kc < KC && !failed; ++kc) {
           const int slot_b = ib % SB;
           if (!mbar_wait(&empty_b[slot_b], ((ib / SB) & 1) ^ 1)) { failed = true; break; }
-          mbar_arrive_expect_tx(&full_b[slot_b], NPAD * 128);
-          tma_load_2d(sb + slot_b * NPAD * 128, &tm_x, kc * kKChunk, 0, &full_b[slot_b]);
+          mbar_arrive_expect_tx(&full_b[slot_b], SB_BYTES);
+#pragma unroll
+          for (int u = 0; u < KSUB; ++u)
+            tma_load_2d(sb + slot_b * SB_BYTES + u * NPAD * 128, &tm_x,
+                        (kc * KSUB + u) * kKChunk, 0, &full_b[slot_b]);
           ++ib;
           for (int t = t0; t < t1; ++t) {
             const int slot_a = ia % SA;
             if (!mbar_wait(&empty_a[slot_a], ((ia / SA) & 1) ^ 1)) { failed = true; break; }
             const int row0 = v0 + t * kTileM;
             const int rows = min(kTileM, v1 - row0);
-            uint8_t* dst = sa + slot_a * kStageA;
+            uint8_t* dst = sa + slot_a * SA_BYTES;
             if (rows == kTileM) {
-              mbar_arrive_expect_tx(&full_a[slot_a], kStageA);
-              tma_load_2d_hint(dst, &tm_w_full, kc * kKChunk, row0, &full_a[slot_a], pol_w);
+              mbar_arrive_expect_tx(&full_a[slot_a], SA_BYTES);
+#pragma unroll
+              for (int u = 0; u < KSUB; ++u)
+                tma_load_2d_hint(dst + u * kStageA, &tm_w_full, (kc * KSUB + u) * kKChunk,
+                                 row0, &full_a[slot_a], pol_w);
             } else {
               const int nbox = (rows + kBoxPart - 1) / kBoxPart;
-              mbar_arrive_expect_tx(&full_a[slot_a], nbox * kBoxPart * 128);
-              for (int j = 0; j < nbox; ++j)
-                tma_load_2d_hint(dst + j * kBoxPart * 128, &tm_w_part, kc * kKChunk,
-                                 row0 + j * kBoxPart, &full_a[slot_a], pol_w);
+              mbar_arrive_expect_tx(&full_a[slot_a], KSUB * nbox * kBoxPart * 128);
+              for (int u = 0; u < KSUB; ++u)
+                for (int j = 0; j < nbox; ++j)
+                  tma_load_2d_hint(dst + u * kStageA + j * kBoxPart * 128, &tm_w_part,
+                                   (kc * KSUB + u) * kKChunk, row0 + j * kBoxPart,
+                                   &full_a[slot_a], pol_w);
             }
             ++ia;
           }
@@ -175,17 +187,20 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
           const int slot_b = ib % SB;
           if (!mbar_wait(&full_b[slot_b], (ib / SB) & 1)) { failed = true; break; }
           tc_fence_after();
-          const uint32_t b_base = smem_u32(sb + slot_b * NPAD * 128);
+          const uint32_t b_base = smem_u32(sb + slot_b * SB_BYTES);
           for (int t = t0; t < t1; ++t) {
             const int slot_a = ia % SA;
             if (!mbar_wait(&full_a[slot_a], (ia / SA) & 1)) { failed = true; break; }
             tc_fence_after();
-            const uint32_t a_base = smem_u32(sa + slot_a * kStageA);
+            const uint32_t a_base = smem_u32(sa + slot_a * SA_BYTES);
             const uint32_t d = tmem + (uint32_t)((buf * G + (t - t0)) * NPAD);
 #pragma unroll
-            for (int k = 0; k < kKChunk / 16; ++k)
-              mma_bf16(d, desc_k_sw128(a_base + k * 32), desc_k_sw128(b_base + k * 32),
-                       idesc, (kc | k) != 0 ? 1u : 0u);
+            for (int u = 0; u < KSUB; ++u)
+#pragma unroll
+              for (int k = 0; k < kKChunk / 16; ++k)
+                mma_bf16(d, desc_k_sw128(a_base + u * kStageA + k * 32),
+                         desc_k_sw128(b_base + u * NPAD * 128 + k * 32), idesc,
+                         (kc | u | k) != 0 ? 1u : 0u);
             mma_commit(&empty_a[slot_a]);
             ++ia;
           }
@@ -286,10 +301,10 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NCH>
+template <int NCH, int KSUB>
 cudaError_t launch_nch(const CUtensorMap& wf, const CUtensorMap& wp, const CUtensorMap& x,
                        const LmArgs& a, const TcParams& tp, size_t smem, cudaStream_t s) {
-  auto k = lmhead_tc_kernel<NCH>;
+  auto k = lmhead_tc_kernel<NCH, KSUB>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
@@ -300,48 +315,70 @@ cudaError_t launch_nch(const CUtensorMap& wf, const CUtensorMap& wp, const CUten
 }  // namespace
 
 // Tiles per CTA, group size, ring depths and TMEM columns for a call.
-bool lmhead_tc_params(int R, int rows_per_cta, TcParams* tp, size_t* smem);
+bool lmhead_tc_params(int R, int H, int rows_per_cta, TcParams* tp, size_t* smem);
 
-bool lmhead_tc_params(int R, int rows_per_cta, TcParams* tp, size_t* smem) {
+bool lmhead_tc_params(int R, int H, int rows_per_cta, TcParams* tp, size_t* smem) {
   int nch = 1;
   while (nch * 32 < R) nch *= 2;
   if (nch > 8) return false;
   tp->npad = nch * 32;
+  // K width per stage: up to 4 boxes (512 contiguous bytes of each weight
+  // row), as long as the B stage stays within 16 KB.
+  const int kchunks = H / kKChunk;
+  int kmax = 16384 / (tp->npad * 128);
+  if (kmax < 1) kmax = 1;
+  tp->ksub = 1;
+  for (int k = 4; k >= 2; k >>= 1)
+    if (k <= kmax && kchunks % k == 0) { tp->ksub = k; break; }
+  // Tiles per TMEM buffer: about half a CTA's range, so each X chunk serves
+  // several weight tiles and the epilogue of one group hides under the next
+  // group's stream (both buffers together stay within TMEM's 512 columns).
   const int n_tiles = (rows_per_cta + kTileM - 1) / kTileM;
-  int G = (n_tiles + 2) / 3;
+  int G = (n_tiles + 1) / 2;
   const int gmax = 256 / tp->npad;
   if (G > gmax) G = gmax;
   if (G < 1) G = 1;
   tp->group = G;
+  if (kchunks % tp->ksub != 0) return false;
+  if (tp->group < 1 || 2 * tp->group * tp->npad > 512) return false;  // TMEM has 512 columns
   uint32_t cols = 32;
-  while (cols < (uint32_t)(2 * G * tp->npad)) cols *= 2;
+  while (cols < (uint32_t)(2 * tp->group * tp->npad)) cols *= 2;
   tp->tmem_cols = cols;
-  tp->stages_b = tp->npad <= 64 ? 4 : 2;
-  const size_t b_bytes = (size_t)tp->stages_b * tp->npad * 128;
+  const size_t a_stage = (size_t)kStageA * tp->ksub;
+  const size_t b_stage = (size_t)tp->npad * 128 * tp->ksub;
+  tp->stages_b = b_stage <= 16384 ? 4 : 2;
+  const size_t b_bytes = (size_t)tp->stages_b * b_stage;
   const size_t budget = 200 * 1024;
-  int sa = (int)((budget - b_bytes) / kStageA);
+  int sa = (int)((budget - b_bytes) / a_stage);
   if (sa > 12) sa = 12;
+  if (sa < 2) return false;
   tp->stages_a = sa;
   const size_t bars = 8 * (size_t)(2 * sa + 2 * tp->stages_b + 5) + 16;
-  *smem = 1024 + (size_t)sa * kStageA + b_bytes + bars + 4 * (size_t)tp->npad * sizeof(MSI);
+  *smem = 1024 + (size_t)sa * a_stage + b_bytes + bars + 4 * (size_t)tp->npad * sizeof(MSI);
   return true;
 }
 
 cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s) {
   TcParams tp;
   size_t smem = 0;
-  if (!lmhead_tc_params(a.R, a.rows_per_cta, &tp, &smem)) return cudaErrorInvalidValue;
+  if (!lmhead_tc_params(a.R, a.H, a.rows_per_cta, &tp, &smem)) return cudaErrorInvalidValue;
   CUtensorMap wf, wp, x;
   if (!make_map(&wf, a.w, a.H, a.V, kKChunk, kTileM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
       !make_map(&wp, a.w, a.H, a.V, kKChunk, kBoxPart, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
       !make_map(&x, a.rows, a.H, a.R, kKChunk, tp.npad, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
     return cudaErrorInvalidValue;
+#define FDL_LM_CASE(NCH)                                                   \
+  case NCH:                                                                \
+    if (tp.ksub == 4) return launch_nch<NCH, 4>(wf, wp, x, a, tp, smem, s); \
+    if (tp.ksub == 2) return launch_nch<NCH, 2>(wf, wp, x, a, tp, smem, s); \
+    return launch_nch<NCH, 1>(wf, wp, x, a, tp, smem, s);
   switch (tp.npad / 32) {
-    case 1: return launch_nch<1>(wf, wp, x, a, tp, smem, s);
-    case 2: return launch_nch<2>(wf, wp, x, a, tp, smem, s);
-    case 4: return launch_nch<4>(wf, wp, x, a, tp, smem, s);
-    case 8: return launch_nch<8>(wf, wp, x, a, tp, smem, s);
+    FDL_LM_CASE(1)
+    FDL_LM_CASE(2)
+    FDL_LM_CASE(4)
+    FDL_LM_CASE(8)
   }
+#undef FDL_LM_CASE
   return cudaErrorInvalidValue;
 }
 

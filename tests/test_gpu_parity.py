@@ -217,3 +217,40 @@ def test_lmhead_shapes_against_oracle(R, V, H):
         assert np.array_equal(t_gpu[sure], t_ref[sure])
         np.testing.assert_allclose(conf.cpu().numpy().astype(np.float64), c_ref, rtol=1e-3)
     assert fdl.get_status(ws) == 0
+
+
+# ------------------------------------------- attention split bookkeeping
+
+EDGE = dict(batch=1, n_q_heads=1, n_kv_heads=1, head_dim=128, block_size=32,
+            q_len=1, q_off=0, prefix=(0, 0), cap_prefix=64, suffix=0, cap_suffix=0,
+            hidden=128, vocab=1000, mask_id=999, shift=0, tau=0.9, w_scale=8.0,
+            dtype="bf16", masked=(1, 1))
+
+
+@pytest.mark.parametrize("over", [
+    dict(),                                                    # one chunk in total
+    dict(n_q_heads=8, q_len=8, prefix=(8192, 8192), cap_prefix=8192),  # 1 item, ~129 CTAs
+    dict(batch=3, n_q_heads=4, n_kv_heads=2, q_len=8, prefix=(1, 5000), cap_prefix=5000),
+    dict(batch=2, n_q_heads=32, n_kv_heads=1, q_len=32, prefix=(100, 700), cap_prefix=700),
+    dict(batch=2, n_q_heads=6, n_kv_heads=3, q_len=3, prefix=(60, 70), cap_prefix=80,
+         suffix=130, cap_suffix=130),                          # DualCache, short
+])
+def test_attention_split_extremes(over):
+    """Stream-K partition edges: fewer chunks than CTAs, one item spread over
+    most CTAs, row tiles of 128 (group 32 x 4 positions), DualCache."""
+    cfg = dict(EDGE, **over)
+    case = synth.make_case("edge", 3, cfg=cfg)
+    c = fdl.make_cfg(case.cfg)
+    d = gh.device_case(case)
+    out = torch.empty_like(d["q"])
+    ws = fdl.workspace(c)
+    for _ in range(2):
+        if case.k_suf is None:
+            fdl.block_attn(c, d["q"], d["k_pre"], d["v_pre"], d["len_pre"], d["k_blk"],
+                           d["v_blk"], out, ws)
+        else:
+            fdl.dualcache_attn(c, d["q"], d["k_pre"], d["v_pre"], d["len_pre"], d["k_blk"],
+                               d["v_blk"], d["k_suf"], d["v_suf"], d["len_suf"], out, ws)
+        ref = cases.run_oracle(case)
+        gh.assert_close_scaled(out.double().cpu().numpy(), ref["attn"], 2e-2, "attn")
+    assert fdl.get_status(ws) == 0
