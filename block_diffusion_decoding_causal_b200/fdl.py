@@ -25,7 +25,7 @@ DEV_BAD_PREFIX_LEN, DEV_BAD_SUFFIX_LEN = 1, 2
 SYMBOLS = ["fdl_version", "fdl_last_error", "fdl_workspace_size",
            "fdl_reset_workspace", "fdl_block_attn", "fdl_dualcache_attn",
            "fdl_lmhead_confidence", "fdl_threshold_commit", "fdl_denoise_step",
-           "fdl_get_status"]
+           "fdl_get_status", "fdl_lmhead_confidence_noalloc"]
 
 
 class StepCfg(ctypes.Structure):
@@ -73,9 +73,11 @@ def lib() -> ctypes.CDLL:
         L.fdl_denoise_step.argtypes = [ctypes.POINTER(StepCfg)] + [_P] * 19 + [
             _P, ctypes.c_size_t, _P]
         L.fdl_get_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
+        L.fdl_lmhead_confidence_noalloc.argtypes = [ctypes.POINTER(StepCfg)] + [_P] * 5 + [_P]
         for name in ["fdl_reset_workspace", "fdl_block_attn", "fdl_dualcache_attn",
                      "fdl_lmhead_confidence", "fdl_threshold_commit",
-                     "fdl_denoise_step", "fdl_get_status"]:
+                     "fdl_denoise_step", "fdl_get_status",
+                     "fdl_lmhead_confidence_noalloc"]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -145,6 +147,15 @@ def lmhead_confidence(cfg, rows, w_lm, row_active, conf, tok, ws, stream=None):
     _check(lib().fdl_lmhead_confidence(ctypes.byref(cfg), ptr(rows), ptr(w_lm),
                                        ptr(row_active), ptr(conf), ptr(tok), ptr(ws),
                                        ws.numel(), stream_ptr(stream)))
+
+
+def lmhead_confidence_noalloc(cfg, rows, w_lm, row_active, conf, tok, stream=None):
+    """fdl_lmhead_confidence with the library's built-in scratch instead of a
+    caller workspace (at most 128 rows; calls on one device must not overlap
+    on the GPU; make the first call on a device before any stream capture)."""
+    _check(lib().fdl_lmhead_confidence_noalloc(ctypes.byref(cfg), ptr(rows), ptr(w_lm),
+                                               ptr(row_active), ptr(conf), ptr(tok),
+                                               stream_ptr(stream)))
 
 
 def threshold_commit(cfg, conf, tok, block_tokens, committed, n_committed,

@@ -131,7 +131,7 @@ int fdl_block_attn(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
 
 /*
  * DualCache attention, v1 (stage a; technical review section 3 and its
- * Algorithm 1, lines 6-7).  As fdl_block_attn with a third key segment,
+ * Algorithm 1).  As fdl_block_attn with a third key segment,
  * the frozen suffix cache k_suf/v_suf [B, Hkv, cap_suffix, d], rows
  * 0:len_suf[b]; every key of prefix, block and suffix is visible (the
  * full-attention dLLMs DualCache accelerates).
@@ -145,7 +145,7 @@ int fdl_dualcache_attn(const fdl_step_cfg* cfg, const void* q,
 
 /*
  * LM head + confidence (stage b, first half; "Fast-dLLM v2" Level 2 and
- * Algorithm 2 steps 1-2 of the technical review).
+ * Algorithm 2 of the technical review, section 4).
  *   For each row i of rows [B*q_len, H] (already token-shifted: row
  *   (b, i) predicts block position q_off + i):
  *     l = w_lm . rows[i]  over the full vocabulary (w_lm [V, H] row-major),
@@ -162,7 +162,7 @@ int fdl_lmhead_confidence(const fdl_step_cfg* cfg, const void* rows,
 
 /*
  * Threshold commit (stage b, second half; technical review Algorithm 2
- * steps 3-5; "Fast-dLLM v2" Level 2 and the sub-block paragraph).
+ * section 4; "Fast-dLLM v2" Level 2 and the sub-block paragraph).
  *   Candidates C_b = unit positions p in [q_off, q_off+q_len) with
  *   block_tokens[b,p] == mask_id.  S_b = {p in C_b : conf[b,p-q_off] >= tau};
  *   if S_b is empty and C_b is not, S_b = {the p in C_b with the largest
@@ -199,6 +199,28 @@ int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
                      int32_t* tok, uint8_t* committed, int32_t* n_committed,
                      int32_t* n_masked_left, void* ws, size_t ws_bytes,
                      void* stream);
+
+/*
+ * LM head + confidence without a workspace (the pages have no counterpart;
+ * this is a deployment convenience).  Same computation, arguments and
+ * outputs as fdl_lmhead_confidence, minus `ws`.
+ * For callers that cannot allocate device memory: a plugin inside another
+ * engine that owns every allocation, a loop where allocation is forbidden
+ * after start-up, or code that cannot reach the host framework's allocator.
+ * The scratch is a fixed array inside libfdl (606,464 bytes, held by every
+ * GPU that loads the library until the process exits), so:
+ *  - batch * q_len must be at most 128 (else FDL_ERR_UNSUPPORTED);
+ *  - the first call on a device looks the array up and zeroes its control
+ *    words, synchronously, with that device current: make that first call
+ *    before any stream capture;
+ *  - every call on a device shares the array and leaves its counters at zero;
+ *    calls whose kernels overlap on the GPU (other streams, other threads)
+ *    race on it and must be serialised by the caller.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+int fdl_lmhead_confidence_noalloc(const fdl_step_cfg* cfg, const void* rows,
+                                  const void* w_lm, const uint8_t* row_active,
+                                  float* conf, int32_t* tok, void* stream);
 
 /* Synchronise `stream`, read the workspace status word into *status (bits
  * FDL_DEV_*) and clear it.  Returns FDL_ERR_DEVICE_STATUS if any bit was
