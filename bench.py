@@ -358,7 +358,7 @@ def main():
 
     lm_bytes = V * H * 2 + B * q_len * H * 2 + B * q_len * 8
     lm_gbs = lm_bytes / t_lm / 1e9
-    traffic = _profiled_traffic("lmhead")
+    traffic = _profiled_traffic("lmhead", "lmhead_tc_qwen7b.md")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -403,15 +403,46 @@ def _launches_per_step(c) -> int:
     return 3 if c["shift"] else 2
 
 
-def _profiled_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if it covers the
-    current kernel build (see profiles/)."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = {
+    "lmhead": ["lmhead_tc.cu", "lm_merge.cuh", "fdl_common.cuh", "sm100.cuh"],
+    "attn": ["attn_tc.cu", "fdl_common.cuh", "sm100.cuh"],
+}
+
+
+def kernel_source_sha(kernel: str) -> str:
+    """SHA-256 over the CUDA sources a kernel is built from."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_diffusion_decoding_causal_b200", "csrc")
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def _profiled_traffic(kernel: str, summary: str, units_here: float = None):
+    """DRAM bytes per launch from a committed ncu summary under profiles/, or
+    None when the summary is missing or the kernel's sources changed since the
+    counters were taken.  A summary captured on a smaller case states its
+    units; the bytes are scaled to this launch's units."""
+    path = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(path):
         return None
+    fields = {}
     with open(path) as f:
-        d = json.load(f)
-    return d.get(kernel)
+        for line in f:
+            if ":" in line and not line.startswith("|"):
+                k, v = line.split(":", 1)
+                fields[k.strip().lstrip("- ")] = v.strip().strip("`")
+    if fields.get("kernel_source_sha256") != kernel_source_sha(kernel):
+        return None
+    try:
+        b = float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+    if units_here is not None and "units_per_launch" in fields:
+        b *= units_here / float(fields["units_per_launch"])
+    return b
 
 
 if __name__ == "__main__":

@@ -38,9 +38,10 @@ constexpr int kCh = 64;                  // keys per chunk
 constexpr int kQRegion = 128 * 128;      // 128 rows x 64 bf16 (16 KB)
 constexpr int kQBuf = 2 * kQRegion;      // d 0-63 and 64-127
 constexpr int kKVRegion = kCh * 128;     // 64 keys x 64 bf16 (8 KB)
-constexpr int kKVSlot = 4 * kKVRegion;   // K lo, K hi, V lo, V hi
+constexpr int kKVSlot = 2 * kKVRegion;   // one of K or V: d 0-63, d 64-127
 constexpr int kPBuf = 128 * 128;         // 128 rows x 64 keys bf16 (16 KB)
-constexpr int kStages = 3;
+constexpr int kKStages = 3;              // K is consumed by S right away
+constexpr int kVStages = 4;              // V waits for the softmax
 constexpr int kThreads = 192;
 constexpr float kRescale = 8.0f;         // log2-domain growth forcing a rescale
 constexpr unsigned kDevTimeout = 4u;
@@ -63,7 +64,8 @@ struct Maps {
 };
 
 struct Smem {
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
@@ -76,6 +78,10 @@ struct Smem {
   int nc[kMaxSeq];      // chunks per item of sequence b
   int lp[kMaxSeq];
   int ls[kMaxSeq];
+  int n_slots;
+  int slots[2 * 160];   // partial slots of the item being merged
+  float row_m[128];     // merged running max per row
+  float row_inv_l[128]; // 1 / merged sum per row
 };
 
 // Position in the chunk sequence of one CTA.
@@ -163,9 +169,10 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_smem = base;                       // 2 x 32 KB
-  uint8_t* kv_smem = q_smem + 2 * kQBuf;        // 3 x 32 KB
-  uint8_t* p_smem = kv_smem + kStages * kKVSlot;  // 2 x 16 KB
+  uint8_t* q_smem = base;                          // 2 x 32 KB
+  uint8_t* k_smem = q_smem + 2 * kQBuf;            // 3 x 16 KB
+  uint8_t* v_smem = k_smem + kKStages * kKVSlot;   // 4 x 16 KB
+  uint8_t* p_smem = v_smem + kVStages * kKVSlot;   // 2 x 16 KB
   Smem& S = *reinterpret_cast<Smem*>(p_smem + 2 * kPBuf);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -173,9 +180,13 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   const int rows_full = a.qpt * a.group;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&S.kv_full[i], 1);
-      mbar_init(&S.kv_empty[i], 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&S.k_full[i], 1);
+      mbar_init(&S.k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&S.v_full[i], 1);
+      mbar_init(&S.v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.q_full[i], 1);
@@ -237,118 +248,147 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
 
   if (c_begin < c_end && warp == 0) {
     // -------------------------------------------------------------- TMA
+    // Order K_0, K_1, V_0, K_2, V_1, ...: K runs one chunk ahead of V.
     if (lane == 0) {
-      int kv_i = 0, q_i = 0, prev_x = -1;
-      Cursor c = locate(S, a.B, per_seq, c_begin);
-      for (long long g = c_begin; g < c_end && !failed; ++g, advance(c, S, per_seq)) {
-        const int x = c.b * per_seq + c.it;
-        const int kvh = c.it / a.n_rt, rt = c.it % a.n_rt;
-        if (x != prev_x) {
-          const int qb = q_i & 1;
-          if (!mbar_wait(&S.q_empty[qb], ((q_i >> 1) & 1) ^ 1)) { failed = true; break; }
-          mbar_arrive_expect_tx(&S.q_full[qb], 2u * 128u * (uint32_t)rows_full);
-          const int z = c.b * a.q_len + rt * a.qpt;
-          tma_load_3d(q_smem + qb * kQBuf, &maps.q, 0, kvh * a.group, z, &S.q_full[qb]);
-          tma_load_3d(q_smem + qb * kQBuf + kQRegion, &maps.q, 64, kvh * a.group, z,
-                      &S.q_full[qb]);
-          ++q_i;
-          prev_x = x;
+      const int n_my = (int)(c_end - c_begin);
+      int q_i = 0, prev_x = -1;
+      Cursor ck = locate(S, a.B, per_seq, c_begin), cv = ck;
+      for (int i = 0; i <= n_my && !failed; ++i) {
+        if (i < n_my) {
+          const int x = ck.b * per_seq + ck.it;
+          const int kvh = ck.it / a.n_rt, rt = ck.it % a.n_rt;
+          if (x != prev_x) {
+            const int qb = q_i & 1;
+            if (!mbar_wait(&S.q_empty[qb], ((q_i >> 1) & 1) ^ 1)) { failed = true; break; }
+            mbar_arrive_expect_tx(&S.q_full[qb], 2u * 128u * (uint32_t)rows_full);
+            const int z = ck.b * a.q_len + rt * a.qpt;
+            tma_load_3d(q_smem + qb * kQBuf, &maps.q, 0, kvh * a.group, z, &S.q_full[qb]);
+            tma_load_3d(q_smem + qb * kQBuf + kQRegion, &maps.q, 64, kvh * a.group, z,
+                        &S.q_full[qb]);
+            ++q_i;
+            prev_x = x;
+          }
+          const int slot = i % kKStages;
+          if (!mbar_wait(&S.k_empty[slot], ((i / kKStages) & 1) ^ 1)) { failed = true; break; }
+          const ChunkInfo ci = chunk_info(ck.j, S.lp[ck.b], S.ls[ck.b], a.D);
+          const int bk = ck.b * a.Hkv + kvh;
+          const CUtensorMap* mk = ci.seg == 0 ? &maps.kp : (ci.seg == 1 ? &maps.kb : &maps.ks);
+          const int row = ci.seg == 0 ? bk * a.cap_p + ci.key0
+                                      : (ci.seg == 1 ? bk * a.D : bk * a.cap_s + ci.key0);
+          uint8_t* dst = k_smem + slot * kKVSlot;
+          mbar_arrive_expect_tx(&S.k_full[slot], kKVSlot);
+          tma_load_2d(dst, mk, 0, row, &S.k_full[slot]);
+          tma_load_2d(dst + kKVRegion, mk, 64, row, &S.k_full[slot]);
+          advance(ck, S, per_seq);
         }
-        const int slot = kv_i % kStages;
-        if (!mbar_wait(&S.kv_empty[slot], ((kv_i / kStages) & 1) ^ 1)) { failed = true; break; }
-        const ChunkInfo ci = chunk_info(c.j, S.lp[c.b], S.ls[c.b], a.D);
-        const CUtensorMap* mk;
-        const CUtensorMap* mv;
-        int row;
-        const int bk = c.b * a.Hkv + kvh;
-        if (ci.seg == 0) {
-          mk = &maps.kp; mv = &maps.vp; row = bk * a.cap_p + ci.key0;
-        } else if (ci.seg == 1) {
-          mk = &maps.kb; mv = &maps.vb; row = bk * a.D;
-        } else {
-          mk = &maps.ks; mv = &maps.vs; row = bk * a.cap_s + ci.key0;
+        if (i >= 1) {
+          const int j = i - 1;
+          const int kvh = cv.it / a.n_rt;
+          const int slot = j % kVStages;
+          if (!mbar_wait(&S.v_empty[slot], ((j / kVStages) & 1) ^ 1)) { failed = true; break; }
+          const ChunkInfo ci = chunk_info(cv.j, S.lp[cv.b], S.ls[cv.b], a.D);
+          const int bk = cv.b * a.Hkv + kvh;
+          const CUtensorMap* mv = ci.seg == 0 ? &maps.vp : (ci.seg == 1 ? &maps.vb : &maps.vs);
+          const int row = ci.seg == 0 ? bk * a.cap_p + ci.key0
+                                      : (ci.seg == 1 ? bk * a.D : bk * a.cap_s + ci.key0);
+          uint8_t* dst = v_smem + slot * kKVSlot;
+          mbar_arrive_expect_tx(&S.v_full[slot], kKVSlot);
+          tma_load_2d(dst, mv, 0, row, &S.v_full[slot]);
+          tma_load_2d(dst + kKVRegion, mv, 64, row, &S.v_full[slot]);
+          advance(cv, S, per_seq);
         }
-        uint8_t* dst = kv_smem + slot * kKVSlot;
-        mbar_arrive_expect_tx(&S.kv_full[slot], kKVSlot);
-        tma_load_2d(dst, mk, 0, row, &S.kv_full[slot]);
-        tma_load_2d(dst + kKVRegion, mk, 64, row, &S.kv_full[slot]);
-        tma_load_2d(dst + 2 * kKVRegion, mv, 0, row, &S.kv_full[slot]);
-        tma_load_2d(dst + 3 * kKVRegion, mv, 64, row, &S.kv_full[slot]);
-        ++kv_i;
       }
-      for (int m = max(0, kv_i - kStages); m < kv_i; ++m)
-        if (!mbar_wait(&S.kv_full[m % kStages], (m / kStages) & 1)) failed = true;
+      // Drain: every load issued has landed before this CTA can exit.
+      for (int m = max(0, n_my - kKStages); m < n_my; ++m)
+        if (!mbar_wait(&S.k_full[m % kKStages], (m / kKStages) & 1)) failed = true;
+      for (int m = max(0, n_my - kVStages); m < n_my; ++m)
+        if (!mbar_wait(&S.v_full[m % kVStages], (m / kVStages) & 1)) failed = true;
       for (int m = max(0, q_i - 2); m < q_i; ++m)
         if (!mbar_wait(&S.q_full[m & 1], (m >> 1) & 1)) failed = true;
     }
   } else if (c_begin < c_end && warp == 1) {
     // -------------------------------------------------------------- MMA
+    // S for chunk i and P V for chunk j < i are issued as soon as each one's
+    // inputs are ready (non-blocking probes), so the slot release that lets
+    // the next loads start never waits on an unrelated load.
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(128, kCh);
       const uint32_t id_pv = idesc_bf16_f32(128, 128) | (1u << 16);  // V is MN-major
-      int kv_i = 0, q_i = 0, s_i = 0, pv_i = 0, o_i = 0, prev_x = -1;
-      // pending P V of the previous chunk
-      bool pend = false;
-      int pend_slot = 0, pend_first = 0, pend_last = 0;
-      auto issue_pv = [&](int slot, int first, int last) -> bool {
-        const int pb = pv_i & 1;
-        if (!mbar_wait(&S.p_full[pb], (pv_i >> 1) & 1)) return false;
-        const int ob = o_i & 1;
-        if (first && !mbar_wait(&S.o_empty[ob], ((o_i >> 1) & 1) ^ 1)) return false;
-        tc_fence_after();
-        const uint32_t p_base = smem_u32(p_smem + pb * kPBuf);
-        const uint32_t v_base = smem_u32(kv_smem + slot * kKVSlot + 2 * kKVRegion);
-        const uint32_t d_o = tmem + 128u + (uint32_t)ob * 128u;
+      const int n_my = (int)(c_end - c_begin);
+      int is = 0, ip = 0, q_s = 0, o_i = 0, prev_xs = -1, prev_xp = -1;
+      Cursor cs = locate(S, a.B, per_seq, c_begin), cp = cs;
+      long long t_last = clock64();
+      while (ip < n_my) {
+        bool progress = false;
+        if (is < n_my) {
+          const int x = cs.b * per_seq + cs.it;
+          const bool first = x != prev_xs;
+          const int slot = is % kKStages, sb = is & 1;
+          bool ready = first ? mbar_test(&S.q_full[q_s & 1], (q_s >> 1) & 1) : true;
+          ready = ready && mbar_test(&S.k_full[slot], (is / kKStages) & 1) &&
+                  mbar_test(&S.s_empty[sb], ((is >> 1) & 1) ^ 1);
+          if (ready) {
+            if (first) {
+              ++q_s;
+              prev_xs = x;
+            }
+            const int qb = (q_s - 1) & 1;
+            const bool last = (is + 1 == n_my) || (cs.j + 1 == S.nc[cs.b]);
+            tc_fence_after();
+            const uint32_t q_base = smem_u32(q_smem + qb * kQBuf);
+            const uint32_t k_base = smem_u32(k_smem + slot * kKVSlot);
+            const uint32_t d_s = tmem + (uint32_t)sb * kCh;
 #pragma unroll
-        for (int k = 0; k < kCh / 16; ++k)
-          mma_bf16(d_o, desc_k_sw128(p_base + k * 32),
-                   desc_mn_sw128(v_base + k * 2048, kKVRegion, 1024), id_pv,
-                   (first && k == 0) ? 0u : 1u);
-        mma_commit(&S.kv_empty[slot]);
-        mma_commit(&S.p_empty[pb]);
-        mma_commit(&S.pv_done);
-        if (last) {
-          mma_commit(&S.o_full[ob]);
-          ++o_i;
+            for (int k = 0; k < 8; ++k)
+              mma_bf16(d_s, desc_k_sw128(q_base + (k >> 2) * kQRegion + (k & 3) * 32),
+                       desc_k_sw128(k_base + (k >> 2) * kKVRegion + (k & 3) * 32), id_s,
+                       k ? 1u : 0u);
+            mma_commit(&S.s_full[sb]);
+            mma_commit(&S.k_empty[slot]);
+            if (last) mma_commit(&S.q_empty[qb]);
+            advance(cs, S, per_seq);
+            ++is;
+            progress = true;
+          }
         }
-        ++pv_i;
-        return true;
-      };
-      Cursor c = locate(S, a.B, per_seq, c_begin);
-      for (long long g = c_begin; g < c_end && !failed; ++g, advance(c, S, per_seq)) {
-        const int x = c.b * per_seq + c.it;
-        const int first = x != prev_x;
-        const int last = (g + 1 == c_end) || (c.j + 1 == S.nc[c.b]);
-        if (first) {
-          if (!mbar_wait(&S.q_full[q_i & 1], (q_i >> 1) & 1)) { failed = true; break; }
-          ++q_i;
-          prev_x = x;
-        }
-        const int qb = (q_i - 1) & 1;
-        const int slot = kv_i % kStages;
-        if (!mbar_wait(&S.kv_full[slot], (kv_i / kStages) & 1)) { failed = true; break; }
-        const int sb = s_i & 1;
-        if (!mbar_wait(&S.s_empty[sb], ((s_i >> 1) & 1) ^ 1)) { failed = true; break; }
-        tc_fence_after();
-        const uint32_t q_base = smem_u32(q_smem + qb * kQBuf);
-        const uint32_t k_base = smem_u32(kv_smem + slot * kKVSlot);
-        const uint32_t d_s = tmem + (uint32_t)sb * kCh;
+        if (ip < is) {
+          const int x = cp.b * per_seq + cp.it;
+          const bool first = x != prev_xp;
+          const int pb = ip & 1, vslot = ip % kVStages, ob = o_i & 1;
+          bool ready = mbar_test(&S.p_full[pb], (ip >> 1) & 1) &&
+                       mbar_test(&S.v_full[vslot], (ip / kVStages) & 1);
+          if (first) ready = ready && mbar_test(&S.o_empty[ob], ((o_i >> 1) & 1) ^ 1);
+          if (ready) {
+            if (first) prev_xp = x;
+            const bool last = (ip + 1 == n_my) || (cp.j + 1 == S.nc[cp.b]);
+            tc_fence_after();
+            const uint32_t p_base = smem_u32(p_smem + pb * kPBuf);
+            const uint32_t v_base = smem_u32(v_smem + vslot * kKVSlot);
+            const uint32_t d_o = tmem + 128u + (uint32_t)ob * 128u;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          mma_bf16(d_s, desc_k_sw128(q_base + (k >> 2) * kQRegion + (k & 3) * 32),
-                   desc_k_sw128(k_base + (k >> 2) * kKVRegion + (k & 3) * 32), id_s,
-                   k ? 1u : 0u);
-        mma_commit(&S.s_full[sb]);
-        if (last) mma_commit(&S.q_empty[qb]);
-        ++s_i;
-        if (pend && !issue_pv(pend_slot, pend_first, pend_last)) { failed = true; break; }
-        pend = true;
-        pend_slot = slot;
-        pend_first = first;
-        pend_last = last;
-        ++kv_i;
+            for (int k = 0; k < kCh / 16; ++k)
+              mma_bf16(d_o, desc_k_sw128(p_base + k * 32),
+                       desc_mn_sw128(v_base + k * 2048, kKVRegion, 1024), id_pv,
+                       (first && k == 0) ? 0u : 1u);
+            mma_commit(&S.v_empty[vslot]);
+            mma_commit(&S.p_empty[pb]);
+            mma_commit(&S.pv_done);
+            if (last) {
+              mma_commit(&S.o_full[ob]);
+              ++o_i;
+            }
+            advance(cp, S, per_seq);
+            ++ip;
+            progress = true;
+          }
+        }
+        if (progress) {
+          t_last = clock64();
+        } else if (clock64() - t_last > kWaitCycles) {
+          failed = true;
+          break;
+        }
       }
-      if (pend && !failed && !issue_pv(pend_slot, pend_first, pend_last)) failed = true;
       mma_commit(&S.drain);
       if (!mbar_wait(&S.drain, 0)) failed = true;
     }
@@ -518,44 +558,68 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
       named_barrier_softmax();
       if (!S.flag) continue;
       __threadfence();
-      if (row_ok) {
+      // Merge the item's partials: the slot list, then per-row (max, sum),
+      // then all 128 threads over (row, 16-column group) work units.
+      if (threadIdx.x == 64) {
+        int np = 0;
+        for (int j2 = cta_lo; j2 <= cta_hi; ++j2)
+          if (cta_nonempty(j2, T, n))
+            S.slots[np++] =
+                2 * j2 + ((j2 == cta_lo && cta_start(j2, T, n) != x_start) ? 1 : 0);
+        S.n_slots = np;
+      }
+      named_barrier_softmax();
+      const int np = S.n_slots;
+      if (r < rows) {
         float M = kEmptyMax;
-        for (int j2 = cta_lo; j2 <= cta_hi; ++j2) {
-          if (!cta_nonempty(j2, T, n)) continue;
-          const int s2 = 2 * j2 + ((j2 == cta_lo && cta_start(j2, T, n) != x_start) ? 1 : 0);
-          M = fmaxf(M, __ldcg(&a.part_ml[(size_t)s2 * 128 + r]).x);
-        }
+        for (int p = 0; p < np; ++p)
+          M = fmaxf(M, __ldcg(&a.part_ml[(size_t)S.slots[p] * 128 + r]).x);
         float L = 0.f;
-        float acc[128];
+        for (int p = 0; p < np; ++p) {
+          const float2 ml = __ldcg(&a.part_ml[(size_t)S.slots[p] * 128 + r]);
+          L += ml.y * exp2f(ml.x - M);
+        }
+        S.row_m[r] = M;
+        S.row_inv_l[r] = 1.f / L;
+      }
+      named_barrier_softmax();
+      for (int w = threadIdx.x - 64; w < rows * 8; w += 128) {
+        const int rr = w % rows, cg = w / rows;
+        const float M = S.row_m[rr], inv = S.row_inv_l[rr];
+        float acc[16];
 #pragma unroll
-        for (int t = 0; t < 128; ++t) acc[t] = 0.f;
-        for (int j2 = cta_lo; j2 <= cta_hi; ++j2) {
-          if (!cta_nonempty(j2, T, n)) continue;
-          const int s2 = 2 * j2 + ((j2 == cta_lo && cta_start(j2, T, n) != x_start) ? 1 : 0);
-          const float2 ml = __ldcg(&a.part_ml[(size_t)s2 * 128 + r]);
-          const float w = exp2f(ml.x - M);
-          L += ml.y * w;
-          const float4* src = reinterpret_cast<const float4*>(a.part_o + ((size_t)s2 * 128 + r) * 128);
+        for (int t = 0; t < 16; ++t) acc[t] = 0.f;
+#pragma unroll 4
+        for (int p = 0; p < np; ++p) {
+          const int sl = S.slots[p];
+          const float wgt = exp2f(__ldcg(&a.part_ml[(size_t)sl * 128 + rr]).x - M);
+          const float4* src =
+              reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + rr) * 128 + cg * 16);
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
+          for (int t = 0; t < 4; ++t) {
             const float4 v = __ldcg(src + t);
-            acc[4 * t] += v.x * w;
-            acc[4 * t + 1] += v.y * w;
-            acc[4 * t + 2] += v.z * w;
-            acc[4 * t + 3] += v.w * w;
+            acc[4 * t] += v.x * wgt;
+            acc[4 * t + 1] += v.y * wgt;
+            acc[4 * t + 2] += v.z * wgt;
+            acc[4 * t + 3] += v.w * wgt;
           }
         }
-        const float inv = 1.f / L;
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          uint4 v;
-          v.x = pack_bf16(acc[8 * t + 0] * inv, acc[8 * t + 1] * inv);
-          v.y = pack_bf16(acc[8 * t + 2] * inv, acc[8 * t + 3] * inv);
-          v.z = pack_bf16(acc[8 * t + 4] * inv, acc[8 * t + 5] * inv);
-          v.w = pack_bf16(acc[8 * t + 6] * inv, acc[8 * t + 7] * inv);
-          *reinterpret_cast<uint4*>(orow + 8 * t) = v;
-        }
+        const int pq = rr / a.group, jq = rr % a.group;
+        bf16* dst = a.out + (((size_t)c.b * a.q_len + rt * a.qpt + pq) * a.Hq + kvh * a.group + jq) * 128 +
+                    cg * 16;
+        uint4 v0, v1;
+        v0.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+        v0.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+        v0.z = pack_bf16(acc[4] * inv, acc[5] * inv);
+        v0.w = pack_bf16(acc[6] * inv, acc[7] * inv);
+        v1.x = pack_bf16(acc[8] * inv, acc[9] * inv);
+        v1.y = pack_bf16(acc[10] * inv, acc[11] * inv);
+        v1.z = pack_bf16(acc[12] * inv, acc[13] * inv);
+        v1.w = pack_bf16(acc[14] * inv, acc[15] * inv);
+        reinterpret_cast<uint4*>(dst)[0] = v0;
+        reinterpret_cast<uint4*>(dst)[1] = v1;
       }
+      named_barrier_softmax();
       if (threadIdx.x == 64) a.tickets[x] = 0u;
     }
   }
@@ -620,7 +684,7 @@ int attn_tc_qpt(int q_len, int group) {
 }
 
 size_t attn_tc_smem_bytes() {
-  return 1024 + 2 * kQBuf + kStages * kKVSlot + 2 * kPBuf + sizeof(Smem);
+  return 1024 + 2 * kQBuf + (kKStages + kVStages) * kKVSlot + 2 * kPBuf + sizeof(Smem);
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,

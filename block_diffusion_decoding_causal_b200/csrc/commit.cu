@@ -4,7 +4,7 @@
 namespace fdl {
 namespace {
 
-// One warp per sequence (technical review Algorithm 2 steps 3-5).
+// One warp per sequence (technical review, section 4, Algorithm 2).
 __global__ void commit_kernel(const float* conf, const int32_t* tok,
                               int32_t* block_tokens, uint8_t* committed,
                               int32_t* n_committed, int32_t* n_masked_left,

@@ -123,7 +123,7 @@ struct LmArgs {
 
 // --------------------------------------------------------------- commit
 
-// One warp commits sequence b (technical review Algorithm 2 steps 3-5).
+// One warp commits sequence b (technical review, section 4, Algorithm 2).
 // conf_of(i) / tok_of(i) give the unit row i's confidence and token.
 template <typename ConfF, typename TokF>
 __device__ __forceinline__ void commit_sequence_warp(

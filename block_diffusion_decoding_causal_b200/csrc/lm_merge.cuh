@@ -21,7 +21,7 @@ __device__ __forceinline__ bool last_cta_arrives(unsigned int* ticket,
 }
 
 // Merge the n_cta partials of each row into (conf, tok); then, when the call
-// is the fused step, commit (technical review Algorithm 2 steps 3-5).
+// is the fused step, commit (technical review, section 4, Algorithm 2).
 // conf = 1 / sum_v exp(l_v - l_max) is the max softmax probability; the
 // token is the argmax with the lowest vocabulary index on a tie.
 __device__ __forceinline__ void lm_final_merge(const LmArgs& a) {

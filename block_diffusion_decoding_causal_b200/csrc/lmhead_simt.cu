@@ -2,7 +2,7 @@
 //
 // For each row: logits over the full vocabulary, reduced on the fly to the
 // running (max, sum exp, argmax) triple, so logits never reach global
-// memory ("Fast-dLLM v2" Level 2; technical review Algorithm 2 steps 1-2).
+// memory ("Fast-dLLM v2" Level 2; technical review, section 4, Algorithm 2).
 // Each CTA owns a contiguous vocabulary range; a warp computes one vocab row
 // against 32 input rows per pass (lane-strided 16-byte loads, warp
 // all-reduce), lane r keeps row r's running triple.  The last CTA merges the

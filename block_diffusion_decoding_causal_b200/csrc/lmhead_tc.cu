@@ -3,7 +3,7 @@
 // logits[v, r] = W[v, :] . X[r, :] over the full vocabulary, reduced on the
 // chip to each row's running (max logit, sum exp(l - max), argmax)
 // ("Fast-dLLM v2" Level 2: the greedy token and its probability; technical
-// review Algorithm 2 steps 1-2).  Logits never reach global memory.
+// review, section 4, Algorithm 2).  Logits never reach global memory.
 //
 // Swap-AB: the weight is the M = 128 operand (a tile of 128 vocabulary rows),
 // the <= 256 input rows are N.  Each CTA (one per SM) owns a contiguous

@@ -174,7 +174,7 @@ def shifted_rows(src, h_prev, shift: int) -> np.ndarray:
 
 def lmhead_confidence(rows, w, chunk: int = 8192):
     """Greedy prediction and its confidence for each row (v2 digest, Level 2;
-    technical review Algorithm 2 steps 1-2).
+    technical review, section 4, Algorithm 2).
 
     logits l = W h over the full vocabulary; token = argmax l (lowest index
     on a tie, numpy's argmax); confidence = the probability softmax(l) gives
