@@ -398,9 +398,9 @@ def _gpu_id(torch) -> str:
 
 
 def _launches_per_step(c) -> int:
-    """Kernels one fdl_denoise_step launches: attention, (token-shift gather),
-    fused LM head + commit."""
-    return 3 if c["shift"] else 2
+    """Kernels one fdl_denoise_step launches at these shapes: attention and
+    its partial merge, the token-shift gather, the fused LM head + commit."""
+    return 4 if c["shift"] else 3
 
 
 KERNEL_SOURCES = {

@@ -22,8 +22,9 @@
 //            lazy rescale (O in TMEM is rescaled only when the running max
 //            grows by more than 2^8), P = exp2(S - m) as bf16 into shared
 //            memory (swizzled K-major), and the item epilogue.
-// Partial results (unnormalised O, m, l) go to the workspace; the last CTA
-// to finish an item merges them.  No thread waits on another CTA.
+// Partial results (unnormalised O, m, l) go to the workspace; a small merge
+// kernel, launched as a programmatic dependent of this grid, combines the
+// partials of every item that was split.  No thread waits on another CTA.
 #include <cudaTypedefs.h>
 
 #include "fdl_common.cuh"
@@ -38,10 +39,9 @@ constexpr int kCh = 64;                  // keys per chunk
 constexpr int kQRegion = 128 * 128;      // 128 rows x 64 bf16 (16 KB)
 constexpr int kQBuf = 2 * kQRegion;      // d 0-63 and 64-127
 constexpr int kKVRegion = kCh * 128;     // 64 keys x 64 bf16 (8 KB)
-constexpr int kKVSlot = 2 * kKVRegion;   // one of K or V: d 0-63, d 64-127
+constexpr int kKVSlot = 4 * kKVRegion;   // K lo, K hi, V lo, V hi: one 32 KB stage
 constexpr int kPBuf = 128 * 128;         // 128 rows x 64 keys bf16 (16 KB)
-constexpr int kKStages = 3;              // K is consumed by S right away
-constexpr int kVStages = 4;              // V waits for the softmax
+constexpr int kStages = 3;
 constexpr int kThreads = 192;
 constexpr float kRescale = 8.0f;         // log2-domain growth forcing a rescale
 constexpr unsigned kDevTimeout = 4u;
@@ -64,8 +64,7 @@ struct Maps {
 };
 
 struct Smem {
-  uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
@@ -78,10 +77,6 @@ struct Smem {
   int nc[kMaxSeq];      // chunks per item of sequence b
   int lp[kMaxSeq];
   int ls[kMaxSeq];
-  int n_slots;
-  int slots[2 * 160];   // partial slots of the item being merged
-  float row_m[128];     // merged running max per row
-  float row_inv_l[128]; // 1 / merged sum per row
 };
 
 // Position in the chunk sequence of one CTA.
@@ -170,9 +165,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_smem = base;                          // 2 x 32 KB
-  uint8_t* k_smem = q_smem + 2 * kQBuf;            // 3 x 16 KB
-  uint8_t* v_smem = k_smem + kKStages * kKVSlot;   // 4 x 16 KB
-  uint8_t* p_smem = v_smem + kVStages * kKVSlot;   // 2 x 16 KB
+  uint8_t* kv_smem = q_smem + 2 * kQBuf;           // 3 x 32 KB
+  uint8_t* p_smem = kv_smem + kStages * kKVSlot;   // 2 x 16 KB
   Smem& S = *reinterpret_cast<Smem*>(p_smem + 2 * kPBuf);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -180,13 +174,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   const int rows_full = a.qpt * a.group;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kKStages; ++i) {
-      mbar_init(&S.k_full[i], 1);
-      mbar_init(&S.k_empty[i], 1);
-    }
-    for (int i = 0; i < kVStages; ++i) {
-      mbar_init(&S.v_full[i], 1);
-      mbar_init(&S.v_empty[i], 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&S.kv_full[i], 1);
+      mbar_init(&S.kv_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.q_full[i], 1);
@@ -240,6 +230,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   tc_fence_after();
   const uint32_t tmem = S.tmem;
 
+  // The merge kernel that follows may be scheduled now; it waits for this
+  // grid to finish before it reads anything.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long T = S.cb[a.B];
   const int n = a.n_cta;
   const long long c_begin = cta_start(blockIdx.x, T, n);
@@ -248,61 +241,44 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
 
   if (c_begin < c_end && warp == 0) {
     // -------------------------------------------------------------- TMA
-    // Order K_0, K_1, V_0, K_2, V_1, ...: K runs one chunk ahead of V.
+    // One 32 KB stage per chunk (K and V, four boxes, one barrier): the TMA
+    // engine streams far faster with few large stages than many small ones.
     if (lane == 0) {
       const int n_my = (int)(c_end - c_begin);
       int q_i = 0, prev_x = -1;
-      Cursor ck = locate(S, a.B, per_seq, c_begin), cv = ck;
-      for (int i = 0; i <= n_my && !failed; ++i) {
-        if (i < n_my) {
-          const int x = ck.b * per_seq + ck.it;
-          const int kvh = ck.it / a.n_rt, rt = ck.it % a.n_rt;
-          if (x != prev_x) {
-            const int qb = q_i & 1;
-            if (!mbar_wait(&S.q_empty[qb], ((q_i >> 1) & 1) ^ 1)) { failed = true; break; }
-            mbar_arrive_expect_tx(&S.q_full[qb], 2u * 128u * (uint32_t)rows_full);
-            const int z = ck.b * a.q_len + rt * a.qpt;
-            tma_load_3d(q_smem + qb * kQBuf, &maps.q, 0, kvh * a.group, z, &S.q_full[qb]);
-            tma_load_3d(q_smem + qb * kQBuf + kQRegion, &maps.q, 64, kvh * a.group, z,
-                        &S.q_full[qb]);
-            ++q_i;
-            prev_x = x;
-          }
-          const int slot = i % kKStages;
-          if (!mbar_wait(&S.k_empty[slot], ((i / kKStages) & 1) ^ 1)) { failed = true; break; }
-          const ChunkInfo ci = chunk_info(ck.j, S.lp[ck.b], S.ls[ck.b], a.D);
-          const int bk = ck.b * a.Hkv + kvh;
-          const CUtensorMap* mk = ci.seg == 0 ? &maps.kp : (ci.seg == 1 ? &maps.kb : &maps.ks);
-          const int row = ci.seg == 0 ? bk * a.cap_p + ci.key0
-                                      : (ci.seg == 1 ? bk * a.D : bk * a.cap_s + ci.key0);
-          uint8_t* dst = k_smem + slot * kKVSlot;
-          mbar_arrive_expect_tx(&S.k_full[slot], kKVSlot);
-          tma_load_2d(dst, mk, 0, row, &S.k_full[slot]);
-          tma_load_2d(dst + kKVRegion, mk, 64, row, &S.k_full[slot]);
-          advance(ck, S, per_seq);
+      Cursor c = locate(S, a.B, per_seq, c_begin);
+      for (int i = 0; i < n_my && !failed; ++i, advance(c, S, per_seq)) {
+        const int x = c.b * per_seq + c.it;
+        const int kvh = c.it / a.n_rt, rt = c.it % a.n_rt;
+        if (x != prev_x) {
+          const int qb = q_i & 1;
+          if (!mbar_wait(&S.q_empty[qb], ((q_i >> 1) & 1) ^ 1)) { failed = true; break; }
+          mbar_arrive_expect_tx(&S.q_full[qb], 2u * 128u * (uint32_t)rows_full);
+          const int z = c.b * a.q_len + rt * a.qpt;
+          tma_load_3d(q_smem + qb * kQBuf, &maps.q, 0, kvh * a.group, z, &S.q_full[qb]);
+          tma_load_3d(q_smem + qb * kQBuf + kQRegion, &maps.q, 64, kvh * a.group, z,
+                      &S.q_full[qb]);
+          ++q_i;
+          prev_x = x;
         }
-        if (i >= 1) {
-          const int j = i - 1;
-          const int kvh = cv.it / a.n_rt;
-          const int slot = j % kVStages;
-          if (!mbar_wait(&S.v_empty[slot], ((j / kVStages) & 1) ^ 1)) { failed = true; break; }
-          const ChunkInfo ci = chunk_info(cv.j, S.lp[cv.b], S.ls[cv.b], a.D);
-          const int bk = cv.b * a.Hkv + kvh;
-          const CUtensorMap* mv = ci.seg == 0 ? &maps.vp : (ci.seg == 1 ? &maps.vb : &maps.vs);
-          const int row = ci.seg == 0 ? bk * a.cap_p + ci.key0
-                                      : (ci.seg == 1 ? bk * a.D : bk * a.cap_s + ci.key0);
-          uint8_t* dst = v_smem + slot * kKVSlot;
-          mbar_arrive_expect_tx(&S.v_full[slot], kKVSlot);
-          tma_load_2d(dst, mv, 0, row, &S.v_full[slot]);
-          tma_load_2d(dst + kKVRegion, mv, 64, row, &S.v_full[slot]);
-          advance(cv, S, per_seq);
-        }
+        const int slot = i % kStages;
+        if (!mbar_wait(&S.kv_empty[slot], ((i / kStages) & 1) ^ 1)) { failed = true; break; }
+        const ChunkInfo ci = chunk_info(c.j, S.lp[c.b], S.ls[c.b], a.D);
+        const int bk = c.b * a.Hkv + kvh;
+        const CUtensorMap* mk = ci.seg == 0 ? &maps.kp : (ci.seg == 1 ? &maps.kb : &maps.ks);
+        const CUtensorMap* mv = ci.seg == 0 ? &maps.vp : (ci.seg == 1 ? &maps.vb : &maps.vs);
+        const int row = ci.seg == 0 ? bk * a.cap_p + ci.key0
+                                    : (ci.seg == 1 ? bk * a.D : bk * a.cap_s + ci.key0);
+        uint8_t* dst = kv_smem + slot * kKVSlot;
+        mbar_arrive_expect_tx(&S.kv_full[slot], kKVSlot);
+        tma_load_2d(dst, mk, 0, row, &S.kv_full[slot]);
+        tma_load_2d(dst + kKVRegion, mk, 64, row, &S.kv_full[slot]);
+        tma_load_2d(dst + 2 * kKVRegion, mv, 0, row, &S.kv_full[slot]);
+        tma_load_2d(dst + 3 * kKVRegion, mv, 64, row, &S.kv_full[slot]);
       }
       // Drain: every load issued has landed before this CTA can exit.
-      for (int m = max(0, n_my - kKStages); m < n_my; ++m)
-        if (!mbar_wait(&S.k_full[m % kKStages], (m / kKStages) & 1)) failed = true;
-      for (int m = max(0, n_my - kVStages); m < n_my; ++m)
-        if (!mbar_wait(&S.v_full[m % kVStages], (m / kVStages) & 1)) failed = true;
+      for (int m = max(0, n_my - kStages); m < n_my; ++m)
+        if (!mbar_wait(&S.kv_full[m % kStages], (m / kStages) & 1)) failed = true;
       for (int m = max(0, q_i - 2); m < q_i; ++m)
         if (!mbar_wait(&S.q_full[m & 1], (m >> 1) & 1)) failed = true;
     }
@@ -323,9 +299,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         if (is < n_my) {
           const int x = cs.b * per_seq + cs.it;
           const bool first = x != prev_xs;
-          const int slot = is % kKStages, sb = is & 1;
+          const int slot = is % kStages, sb = is & 1;
           bool ready = first ? mbar_test(&S.q_full[q_s & 1], (q_s >> 1) & 1) : true;
-          ready = ready && mbar_test(&S.k_full[slot], (is / kKStages) & 1) &&
+          ready = ready && mbar_test(&S.kv_full[slot], (is / kStages) & 1) &&
                   mbar_test(&S.s_empty[sb], ((is >> 1) & 1) ^ 1);
           if (ready) {
             if (first) {
@@ -336,7 +312,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
             const bool last = (is + 1 == n_my) || (cs.j + 1 == S.nc[cs.b]);
             tc_fence_after();
             const uint32_t q_base = smem_u32(q_smem + qb * kQBuf);
-            const uint32_t k_base = smem_u32(k_smem + slot * kKVSlot);
+            const uint32_t k_base = smem_u32(kv_smem + slot * kKVSlot);
             const uint32_t d_s = tmem + (uint32_t)sb * kCh;
 #pragma unroll
             for (int k = 0; k < 8; ++k)
@@ -344,7 +320,6 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
                        desc_k_sw128(k_base + (k >> 2) * kKVRegion + (k & 3) * 32), id_s,
                        k ? 1u : 0u);
             mma_commit(&S.s_full[sb]);
-            mma_commit(&S.k_empty[slot]);
             if (last) mma_commit(&S.q_empty[qb]);
             advance(cs, S, per_seq);
             ++is;
@@ -354,23 +329,22 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         if (ip < is) {
           const int x = cp.b * per_seq + cp.it;
           const bool first = x != prev_xp;
-          const int pb = ip & 1, vslot = ip % kVStages, ob = o_i & 1;
-          bool ready = mbar_test(&S.p_full[pb], (ip >> 1) & 1) &&
-                       mbar_test(&S.v_full[vslot], (ip / kVStages) & 1);
+          const int pb = ip & 1, vslot = ip % kStages, ob = o_i & 1;
+          bool ready = mbar_test(&S.p_full[pb], (ip >> 1) & 1);
           if (first) ready = ready && mbar_test(&S.o_empty[ob], ((o_i >> 1) & 1) ^ 1);
           if (ready) {
             if (first) prev_xp = x;
             const bool last = (ip + 1 == n_my) || (cp.j + 1 == S.nc[cp.b]);
             tc_fence_after();
             const uint32_t p_base = smem_u32(p_smem + pb * kPBuf);
-            const uint32_t v_base = smem_u32(v_smem + vslot * kKVSlot);
+            const uint32_t v_base = smem_u32(kv_smem + vslot * kKVSlot + 2 * kKVRegion);
             const uint32_t d_o = tmem + 128u + (uint32_t)ob * 128u;
 #pragma unroll
             for (int k = 0; k < kCh / 16; ++k)
               mma_bf16(d_o, desc_k_sw128(p_base + k * 32),
                        desc_mn_sw128(v_base + k * 2048, kKVRegion, 1024), id_pv,
                        (first && k == 0) ? 0u : 1u);
-            mma_commit(&S.v_empty[vslot]);
+            mma_commit(&S.kv_empty[vslot]);
             mma_commit(&S.p_empty[pb]);
             mma_commit(&S.pv_done);
             if (last) {
@@ -526,7 +500,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         ++o_i;
         continue;
       }
-      // Partial of this CTA: slot 2*cta for its first item, 2*cta+1 otherwise.
+      // Partial of this CTA: slot 2*cta for its first item, 2*cta+1 otherwise;
+      // the merge kernel that follows combines the item's partials.
       const int slot = 2 * blockIdx.x + (x == first_x ? 0 : 1);
       float* po = a.part_o + ((size_t)slot * 128 + r) * 128;
       if (warp_active) {
@@ -547,80 +522,6 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
       tc_fence_before();
       mbar_arrive(&S.o_empty[ob]);
       ++o_i;
-      __threadfence();
-      named_barrier_softmax();
-      if (threadIdx.x == 64) {
-        int n_touch = 0;
-        for (int j2 = cta_lo; j2 <= cta_hi; ++j2) n_touch += cta_nonempty(j2, T, n);
-        const unsigned prev = atomicAdd(&a.tickets[x], 1u);
-        S.flag = prev == (unsigned)(n_touch - 1);
-      }
-      named_barrier_softmax();
-      if (!S.flag) continue;
-      __threadfence();
-      // Merge the item's partials: the slot list, then per-row (max, sum),
-      // then all 128 threads over (row, 16-column group) work units.
-      if (threadIdx.x == 64) {
-        int np = 0;
-        for (int j2 = cta_lo; j2 <= cta_hi; ++j2)
-          if (cta_nonempty(j2, T, n))
-            S.slots[np++] =
-                2 * j2 + ((j2 == cta_lo && cta_start(j2, T, n) != x_start) ? 1 : 0);
-        S.n_slots = np;
-      }
-      named_barrier_softmax();
-      const int np = S.n_slots;
-      if (r < rows) {
-        float M = kEmptyMax;
-        for (int p = 0; p < np; ++p)
-          M = fmaxf(M, __ldcg(&a.part_ml[(size_t)S.slots[p] * 128 + r]).x);
-        float L = 0.f;
-        for (int p = 0; p < np; ++p) {
-          const float2 ml = __ldcg(&a.part_ml[(size_t)S.slots[p] * 128 + r]);
-          L += ml.y * exp2f(ml.x - M);
-        }
-        S.row_m[r] = M;
-        S.row_inv_l[r] = 1.f / L;
-      }
-      named_barrier_softmax();
-      for (int w = threadIdx.x - 64; w < rows * 8; w += 128) {
-        const int rr = w % rows, cg = w / rows;
-        const float M = S.row_m[rr], inv = S.row_inv_l[rr];
-        float acc[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) acc[t] = 0.f;
-#pragma unroll 4
-        for (int p = 0; p < np; ++p) {
-          const int sl = S.slots[p];
-          const float wgt = exp2f(__ldcg(&a.part_ml[(size_t)sl * 128 + rr]).x - M);
-          const float4* src =
-              reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + rr) * 128 + cg * 16);
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float4 v = __ldcg(src + t);
-            acc[4 * t] += v.x * wgt;
-            acc[4 * t + 1] += v.y * wgt;
-            acc[4 * t + 2] += v.z * wgt;
-            acc[4 * t + 3] += v.w * wgt;
-          }
-        }
-        const int pq = rr / a.group, jq = rr % a.group;
-        bf16* dst = a.out + (((size_t)c.b * a.q_len + rt * a.qpt + pq) * a.Hq + kvh * a.group + jq) * 128 +
-                    cg * 16;
-        uint4 v0, v1;
-        v0.x = pack_bf16(acc[0] * inv, acc[1] * inv);
-        v0.y = pack_bf16(acc[2] * inv, acc[3] * inv);
-        v0.z = pack_bf16(acc[4] * inv, acc[5] * inv);
-        v0.w = pack_bf16(acc[6] * inv, acc[7] * inv);
-        v1.x = pack_bf16(acc[8] * inv, acc[9] * inv);
-        v1.y = pack_bf16(acc[10] * inv, acc[11] * inv);
-        v1.z = pack_bf16(acc[12] * inv, acc[13] * inv);
-        v1.w = pack_bf16(acc[14] * inv, acc[15] * inv);
-        reinterpret_cast<uint4*>(dst)[0] = v0;
-        reinterpret_cast<uint4*>(dst)[1] = v1;
-      }
-      named_barrier_softmax();
-      if (threadIdx.x == 64) a.tickets[x] = 0u;
     }
   }
 
@@ -631,6 +532,107 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
     tmem_dealloc(tmem, 512);
   }
   if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
+}
+
+// Merge of the partials of every item the split spread over several CTAs.
+// One warp per tile row; its 32 lanes are 8 column groups (16 columns each)
+// x 4 partial groups, so the item's partials are read in parallel and
+// combined with the usual (max, sum) rescaling, then reduced across the 4
+// partial groups by shuffles.  Runs after the attention grid completes
+// (programmatic dependent launch: it may be scheduled early and waits).
+constexpr int kMergeRows = 8;
+
+__global__ void __launch_bounds__(32 * kMergeRows)
+attn_merge_kernel(const TcArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per_seq = a.Hkv * a.n_rt;
+  const int x = blockIdx.x;
+  const int b = x / per_seq, it = x % per_seq;
+  const int kvh = it / a.n_rt, rt = it % a.n_rt;
+  const int qpt_eff = min(a.qpt, a.q_len - rt * a.qpt);
+  const int rows = qpt_eff * a.group;
+  const int r = blockIdx.y * kMergeRows + warp;
+  if (r >= rows) return;
+  // Recompute the split exactly as the attention kernel did.
+  long long T = 0, cb = 0;
+  int ncb = 0;
+  for (int s2 = 0; s2 < a.B; ++s2) {
+    int Lp = a.len_pre[s2];
+    if (Lp < 0 || Lp > a.cap_p) Lp = 0;
+    int Ls = 0;
+    if (a.dual) {
+      Ls = a.len_suf[s2];
+      if (Ls < 0 || Ls > a.cap_s) Ls = 0;
+    }
+    const int nc = (Lp + kCh - 1) / kCh + 1 + (Ls + kCh - 1) / kCh;
+    if (s2 == b) {
+      cb = T;
+      ncb = nc;
+    }
+    T += (long long)nc * per_seq;
+  }
+  const int n = a.n_cta;
+  const long long x_start = cb + (long long)it * ncb, x_end = x_start + ncb;
+  const int cta_lo = cta_of(x_start, T, n), cta_hi = cta_of(x_end - 1, T, n);
+  if (cta_lo == cta_hi) return;  // written directly by its only CTA
+  const int cg = lane & 7, pg = lane >> 3;
+  float M = kEmptyMax, L = 0.f, acc[16];
+#pragma unroll
+  for (int t = 0; t < 16; ++t) acc[t] = 0.f;
+  for (int j = cta_lo + pg; j <= cta_hi; j += 4) {
+    if (!cta_nonempty(j, T, n)) continue;
+    const int sl = 2 * j + ((j == cta_lo && cta_start(j, T, n) != x_start) ? 1 : 0);
+    const float2 ml = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
+    const float4* src =
+        reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128 + cg * 16);
+    float4 v[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) v[t] = __ldcg(src + t);
+    const float m_new = fmaxf(M, ml.x);
+    const float f_old = exp2f(M - m_new), w = exp2f(ml.x - m_new);
+    L = L * f_old + ml.y * w;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      acc[4 * t] = acc[4 * t] * f_old + v[t].x * w;
+      acc[4 * t + 1] = acc[4 * t + 1] * f_old + v[t].y * w;
+      acc[4 * t + 2] = acc[4 * t + 2] * f_old + v[t].z * w;
+      acc[4 * t + 3] = acc[4 * t + 3] * f_old + v[t].w * w;
+    }
+    M = m_new;
+  }
+  // Combine the 4 partial groups (lanes cg, cg+8, cg+16, cg+24).
+  float Mall = M;
+  Mall = fmaxf(Mall, __shfl_xor_sync(0xffffffffu, Mall, 8));
+  Mall = fmaxf(Mall, __shfl_xor_sync(0xffffffffu, Mall, 16));
+  const float f = exp2f(M - Mall);
+  L *= f;
+  L += __shfl_xor_sync(0xffffffffu, L, 8);
+  L += __shfl_xor_sync(0xffffffffu, L, 16);
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    float v = acc[t] * f;
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 16);
+    acc[t] = v;
+  }
+  if (pg == 0) {
+    const float inv = 1.f / L;
+    const int pq = r / a.group, jq = r % a.group;
+    bf16* dst = a.out + (((size_t)b * a.q_len + rt * a.qpt + pq) * a.Hq + kvh * a.group + jq) * 128 +
+                cg * 16;
+    uint4 v0, v1;
+    v0.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+    v0.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+    v0.z = pack_bf16(acc[4] * inv, acc[5] * inv);
+    v0.w = pack_bf16(acc[6] * inv, acc[7] * inv);
+    v1.x = pack_bf16(acc[8] * inv, acc[9] * inv);
+    v1.y = pack_bf16(acc[10] * inv, acc[11] * inv);
+    v1.z = pack_bf16(acc[12] * inv, acc[13] * inv);
+    v1.w = pack_bf16(acc[14] * inv, acc[15] * inv);
+    reinterpret_cast<uint4*>(dst)[0] = v0;
+    reinterpret_cast<uint4*>(dst)[1] = v1;
+  }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -684,7 +686,7 @@ int attn_tc_qpt(int q_len, int group) {
 }
 
 size_t attn_tc_smem_bytes() {
-  return 1024 + 2 * kQBuf + (kKStages + kVStages) * kKVSlot + 2 * kPBuf + sizeof(Smem);
+  return 1024 + 2 * kQBuf + kStages * kKVSlot + 2 * kPBuf + sizeof(Smem);
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
@@ -736,6 +738,20 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   attn_tc_kernel<<<n_cta, kThreads, smem, s>>>(maps, t);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(a.B * a.Hkv * t.n_rt, (qpt * a.group + kMergeRows - 1) / kMergeRows, 1);
+  lc.blockDim = dim3(32 * kMergeRows, 1, 1);
+  lc.dynamicSmemBytes = 0;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  e = cudaLaunchKernelEx(&lc, attn_merge_kernel, t);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
