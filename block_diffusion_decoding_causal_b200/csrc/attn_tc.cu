@@ -191,29 +191,44 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
     mbar_init(&S.pv_done, 1);
     mbar_init(&S.drain, 1);
     fence_barrier_init();
-    // Sequence table from the device-resident lengths.
-    long long run = 0;
-    for (int b = 0; b < a.B; ++b) {
-      int Lp = a.len_pre[b];
-      if (Lp < 0 || Lp > a.cap_p) {
-        if (blockIdx.x == 0) atomicOr(&a.ctrl->status, FDL_DEV_BAD_PREFIX_LEN);
-        Lp = 0;
-      }
-      int Ls = 0;
-      if (a.dual) {
-        Ls = a.len_suf[b];
-        if (Ls < 0 || Ls > a.cap_s) {
-          if (blockIdx.x == 0) atomicOr(&a.ctrl->status, FDL_DEV_BAD_SUFFIX_LEN);
-          Ls = 0;
+  }
+  // Sequence table from the device-resident lengths: warp 0 reads 32
+  // lengths at a time and prefix-sums the chunk counts with shuffles.
+  if (warp == 0) {
+    int run = 0;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+      const int b = b0 + lane;
+      int Lp = 0, Ls = 0, nc = 0;
+      if (b < a.B) {
+        Lp = a.len_pre[b];
+        if (Lp < 0 || Lp > a.cap_p) {
+          if (blockIdx.x == 0) atomicOr(&a.ctrl->status, FDL_DEV_BAD_PREFIX_LEN);
+          Lp = 0;
         }
+        if (a.dual) {
+          Ls = a.len_suf[b];
+          if (Ls < 0 || Ls > a.cap_s) {
+            if (blockIdx.x == 0) atomicOr(&a.ctrl->status, FDL_DEV_BAD_SUFFIX_LEN);
+            Ls = 0;
+          }
+        }
+        nc = (Lp + kCh - 1) / kCh + 1 + (Ls + kCh - 1) / kCh;
       }
-      S.lp[b] = Lp;
-      S.ls[b] = Ls;
-      S.nc[b] = (Lp + kCh - 1) / kCh + 1 + (Ls + kCh - 1) / kCh;
-      S.cb[b] = (int)run;
-      run += (long long)S.nc[b] * per_seq;
+      int incl = nc * per_seq;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (b < a.B) {
+        S.lp[b] = Lp;
+        S.ls[b] = Ls;
+        S.nc[b] = nc;
+        S.cb[b] = run + incl - nc * per_seq;
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    S.cb[a.B] = (int)run;
+    if (lane == 0) S.cb[a.B] = run;
   }
   // Padding rows of both Q buffers are never written by TMA: zero them once.
   for (int t = threadIdx.x; t < 2 * 2 * (128 - rows_full) * 8; t += kThreads) {
@@ -230,9 +245,6 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   tc_fence_after();
   const uint32_t tmem = S.tmem;
 
-  // The merge kernel that follows may be scheduled now; it waits for this
-  // grid to finish before it reads anything.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long T = S.cb[a.B];
   const int n = a.n_cta;
   const long long c_begin = cta_start(blockIdx.x, T, n);
@@ -532,68 +544,82 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
     tmem_dealloc(tmem, 512);
   }
   if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
+  // This CTA is done: the merge kernel may be scheduled once every CTA got
+  // here (it still waits for the whole grid before reading anything).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Merge of the partials of every item the split spread over several CTAs.
-// One warp per tile row; its 32 lanes are 8 column groups (16 columns each)
-// x 4 partial groups, so the item's partials are read in parallel and
-// combined with the usual (max, sum) rescaling, then reduced across the 4
-// partial groups by shuffles.  Runs after the attention grid completes
-// (programmatic dependent launch: it may be scheduled early and waits).
-constexpr int kMergeRows = 8;
-
-__global__ void __launch_bounds__(32 * kMergeRows)
+// A warp per (item, tile row); its lanes are PG partial groups x (32 / PG)
+// column groups, so the partials are read in parallel (PG ~ the expected
+// number of partials per item) and combined with the usual (max, sum)
+// rescaling, then reduced across the partial groups by shuffles.  A CTA
+// holds 8 rows of one item.  Launched as a programmatic dependent of the
+// attention grid: scheduled as its CTAs retire, it waits for the whole grid
+// before reading anything.
+template <int PG>
+__global__ void __launch_bounds__(256)
 attn_merge_kernel(const TcArgs a) {
+  constexpr int CGL = 32 / PG;      // column groups per warp
+  constexpr int COLS = 128 / CGL;   // columns per lane
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_seq = a.Hkv * a.n_rt;
-  const int x = blockIdx.x;
+  const int x = blockIdx.x, r = blockIdx.y * 8 + warp;
   const int b = x / per_seq, it = x % per_seq;
   const int kvh = it / a.n_rt, rt = it % a.n_rt;
   const int qpt_eff = min(a.qpt, a.q_len - rt * a.qpt);
-  const int rows = qpt_eff * a.group;
-  const int r = blockIdx.y * kMergeRows + warp;
-  if (r >= rows) return;
-  // Recompute the split exactly as the attention kernel did.
+  if (r >= qpt_eff * a.group) return;
+  // The split, recomputed exactly as the attention kernel did.
   long long T = 0, cb = 0;
   int ncb = 0;
-  for (int s2 = 0; s2 < a.B; ++s2) {
-    int Lp = a.len_pre[s2];
-    if (Lp < 0 || Lp > a.cap_p) Lp = 0;
-    int Ls = 0;
-    if (a.dual) {
-      Ls = a.len_suf[s2];
-      if (Ls < 0 || Ls > a.cap_s) Ls = 0;
+  for (int b0 = 0; b0 < a.B; b0 += 32) {
+    const int s2 = b0 + lane;
+    int nc = 0;
+    if (s2 < a.B) {
+      int Lp = a.len_pre[s2];
+      if (Lp < 0 || Lp > a.cap_p) Lp = 0;
+      int Ls = 0;
+      if (a.dual) {
+        Ls = a.len_suf[s2];
+        if (Ls < 0 || Ls > a.cap_s) Ls = 0;
+      }
+      nc = (Lp + kCh - 1) / kCh + 1 + (Ls + kCh - 1) / kCh;
     }
-    const int nc = (Lp + kCh - 1) / kCh + 1 + (Ls + kCh - 1) / kCh;
-    if (s2 == b) {
-      cb = T;
-      ncb = nc;
+    int incl = nc * per_seq;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
     }
-    T += (long long)nc * per_seq;
+    if (b >= b0 && b < b0 + 32) {
+      cb = T + __shfl_sync(0xffffffffu, incl - nc * per_seq, b - b0);
+      ncb = __shfl_sync(0xffffffffu, nc, b - b0);
+    }
+    T += __shfl_sync(0xffffffffu, incl, 31);
   }
   const int n = a.n_cta;
   const long long x_start = cb + (long long)it * ncb, x_end = x_start + ncb;
   const int cta_lo = cta_of(x_start, T, n), cta_hi = cta_of(x_end - 1, T, n);
   if (cta_lo == cta_hi) return;  // written directly by its only CTA
-  const int cg = lane & 7, pg = lane >> 3;
-  float M = kEmptyMax, L = 0.f, acc[16];
+  const int cg = lane % CGL, pg = lane / CGL;
+  float M = kEmptyMax, L = 0.f, acc[COLS];
 #pragma unroll
-  for (int t = 0; t < 16; ++t) acc[t] = 0.f;
-  for (int j = cta_lo + pg; j <= cta_hi; j += 4) {
+  for (int t = 0; t < COLS; ++t) acc[t] = 0.f;
+  for (int j = cta_lo + pg; j <= cta_hi; j += PG) {
     if (!cta_nonempty(j, T, n)) continue;
     const int sl = 2 * j + ((j == cta_lo && cta_start(j, T, n) != x_start) ? 1 : 0);
     const float2 ml = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
     const float4* src =
-        reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128 + cg * 16);
-    float4 v[4];
+        reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128 + cg * COLS);
+    float4 v[COLS / 4];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) v[t] = __ldcg(src + t);
+    for (int t = 0; t < COLS / 4; ++t) v[t] = __ldcg(src + t);
     const float m_new = fmaxf(M, ml.x);
     const float f_old = exp2f(M - m_new), w = exp2f(ml.x - m_new);
     L = L * f_old + ml.y * w;
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
+    for (int t = 0; t < COLS / 4; ++t) {
       acc[4 * t] = acc[4 * t] * f_old + v[t].x * w;
       acc[4 * t + 1] = acc[4 * t + 1] * f_old + v[t].y * w;
       acc[4 * t + 2] = acc[4 * t + 2] * f_old + v[t].z * w;
@@ -601,37 +627,35 @@ attn_merge_kernel(const TcArgs a) {
     }
     M = m_new;
   }
-  // Combine the 4 partial groups (lanes cg, cg+8, cg+16, cg+24).
+  // Combine the partial groups: lanes with the same cg, strides CGL.
   float Mall = M;
-  Mall = fmaxf(Mall, __shfl_xor_sync(0xffffffffu, Mall, 8));
-  Mall = fmaxf(Mall, __shfl_xor_sync(0xffffffffu, Mall, 16));
+#pragma unroll
+  for (int o = CGL; o < 32; o <<= 1) Mall = fmaxf(Mall, __shfl_xor_sync(0xffffffffu, Mall, o));
   const float f = exp2f(M - Mall);
   L *= f;
-  L += __shfl_xor_sync(0xffffffffu, L, 8);
-  L += __shfl_xor_sync(0xffffffffu, L, 16);
 #pragma unroll
-  for (int t = 0; t < 16; ++t) {
+  for (int o = CGL; o < 32; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+#pragma unroll
+  for (int t = 0; t < COLS; ++t) {
     float v = acc[t] * f;
-    v += __shfl_xor_sync(0xffffffffu, v, 8);
-    v += __shfl_xor_sync(0xffffffffu, v, 16);
+#pragma unroll
+    for (int o = CGL; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     acc[t] = v;
   }
   if (pg == 0) {
     const float inv = 1.f / L;
     const int pq = r / a.group, jq = r % a.group;
     bf16* dst = a.out + (((size_t)b * a.q_len + rt * a.qpt + pq) * a.Hq + kvh * a.group + jq) * 128 +
-                cg * 16;
-    uint4 v0, v1;
-    v0.x = pack_bf16(acc[0] * inv, acc[1] * inv);
-    v0.y = pack_bf16(acc[2] * inv, acc[3] * inv);
-    v0.z = pack_bf16(acc[4] * inv, acc[5] * inv);
-    v0.w = pack_bf16(acc[6] * inv, acc[7] * inv);
-    v1.x = pack_bf16(acc[8] * inv, acc[9] * inv);
-    v1.y = pack_bf16(acc[10] * inv, acc[11] * inv);
-    v1.z = pack_bf16(acc[12] * inv, acc[13] * inv);
-    v1.w = pack_bf16(acc[14] * inv, acc[15] * inv);
-    reinterpret_cast<uint4*>(dst)[0] = v0;
-    reinterpret_cast<uint4*>(dst)[1] = v1;
+                cg * COLS;
+#pragma unroll
+    for (int t = 0; t < COLS / 8; ++t) {
+      uint4 v;
+      v.x = pack_bf16(acc[8 * t + 0] * inv, acc[8 * t + 1] * inv);
+      v.y = pack_bf16(acc[8 * t + 2] * inv, acc[8 * t + 3] * inv);
+      v.z = pack_bf16(acc[8 * t + 4] * inv, acc[8 * t + 5] * inv);
+      v.w = pack_bf16(acc[8 * t + 6] * inv, acc[8 * t + 7] * inv);
+      reinterpret_cast<uint4*>(dst)[t] = v;
+    }
   }
 }
 
@@ -741,8 +765,9 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(a.B * a.Hkv * t.n_rt, (qpt * a.group + kMergeRows - 1) / kMergeRows, 1);
-  lc.blockDim = dim3(32 * kMergeRows, 1, 1);
+  const int n_items = a.B * a.Hkv * t.n_rt;
+  lc.gridDim = dim3(n_items, (qpt * a.group + 7) / 8, 1);
+  lc.blockDim = dim3(256, 1, 1);
   lc.dynamicSmemBytes = 0;
   lc.stream = s;
   cudaLaunchAttribute attr[1];
@@ -750,7 +775,12 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  e = cudaLaunchKernelEx(&lc, attn_merge_kernel, t);
+  // Partials per split item are about n_cta / n_items + 1 (the split is
+  // even); the lanes spread over that many partial groups.
+  const int est = n_cta / n_items + 1;
+  e = est <= 4 ? cudaLaunchKernelEx(&lc, attn_merge_kernel<4>, t)
+               : (est <= 8 ? cudaLaunchKernelEx(&lc, attn_merge_kernel<8>, t)
+                           : cudaLaunchKernelEx(&lc, attn_merge_kernel<16>, t));
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
