@@ -40,8 +40,11 @@ constexpr int kQRegion = 128 * 128;      // 128 rows x 64 bf16 (16 KB)
 constexpr int kQBuf = 2 * kQRegion;      // d 0-63 and 64-127
 constexpr int kKVRegion = kCh * 128;     // 64 keys x 64 bf16 (8 KB)
 constexpr int kKVSlot = 4 * kKVRegion;   // K lo, K hi, V lo, V hi: one 32 KB stage
-constexpr int kPBuf = 128 * 128;         // 128 rows x 64 keys bf16 (16 KB)
-constexpr int kStages = 3;
+constexpr int kStages = 2;              // K/V stages (two CTAs share an SM)
+constexpr int kQBufs = 1;                // Q is reloaded per item
+constexpr int kSB = 2;                   // S buffers in TMEM; P overwrites its S
+constexpr uint32_t kTmemCols = 256;      // S 2 x 64 columns, O 128 columns
+constexpr uint32_t kOCol = kSB * 64;     // first column of O
 constexpr int kThreads = 192;
 constexpr float kRescale = 8.0f;         // log2-domain growth forcing a rescale
 constexpr unsigned kDevTimeout = 4u;
@@ -66,9 +69,8 @@ struct Maps {
 struct Smem {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_empty[2];
-  uint64_t pv_done;
+  uint64_t s_full[kSB], s_empty[kSB];   // S ready / S and its P free again
+  uint64_t p_full[kSB];                 // P written into TMEM
   uint64_t o_full[2], o_empty[2];
   uint64_t drain;
   uint32_t tmem;
@@ -159,15 +161,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_smem = base;                          // 2 x 32 KB
-  uint8_t* kv_smem = q_smem + 2 * kQBuf;           // 3 x 32 KB
-  uint8_t* p_smem = kv_smem + kStages * kKVSlot;   // 2 x 16 KB
-  Smem& S = *reinterpret_cast<Smem*>(p_smem + 2 * kPBuf);
+  uint8_t* q_smem = base;                          // kQBufs x 32 KB
+  uint8_t* kv_smem = q_smem + kQBufs * kQBuf;      // kStages x 32 KB
+  Smem& S = *reinterpret_cast<Smem*>(kv_smem + kStages * kKVSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_seq = a.Hkv * a.n_rt;  // items per sequence
@@ -181,14 +182,14 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.q_full[i], 1);
       mbar_init(&S.q_empty[i], 1);
-      mbar_init(&S.s_full[i], 1);
-      mbar_init(&S.s_empty[i], 128);
-      mbar_init(&S.p_full[i], 128);
-      mbar_init(&S.p_empty[i], 1);
       mbar_init(&S.o_full[i], 1);
       mbar_init(&S.o_empty[i], 128);
     }
-    mbar_init(&S.pv_done, 1);
+    for (int i = 0; i < kSB; ++i) {
+      mbar_init(&S.s_full[i], 1);
+      mbar_init(&S.s_empty[i], 1);
+      mbar_init(&S.p_full[i], 128);
+    }
     mbar_init(&S.drain, 1);
     fence_barrier_init();
   }
@@ -231,7 +232,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
     if (lane == 0) S.cb[a.B] = run;
   }
   // Padding rows of both Q buffers are never written by TMA: zero them once.
-  for (int t = threadIdx.x; t < 2 * 2 * (128 - rows_full) * 8; t += kThreads) {
+  for (int t = threadIdx.x; t < kQBufs * 2 * (128 - rows_full) * 8; t += kThreads) {
     const int per_region = (128 - rows_full) * 8;
     const int region = t / per_region, w = t % per_region;
     const int row = rows_full + w / 8, chunk = w % 8;
@@ -239,7 +240,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async_smem();
-  if (warp == 1) tmem_alloc(&S.tmem, 512);
+  if (warp == 1) tmem_alloc(&S.tmem, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -262,17 +263,6 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
       for (int i = 0; i < n_my && !failed; ++i, advance(c, S, per_seq)) {
         const int x = c.b * per_seq + c.it;
         const int kvh = c.it / a.n_rt, rt = c.it % a.n_rt;
-        if (x != prev_x) {
-          const int qb = q_i & 1;
-          if (!mbar_wait(&S.q_empty[qb], ((q_i >> 1) & 1) ^ 1)) { failed = true; break; }
-          mbar_arrive_expect_tx(&S.q_full[qb], 2u * 128u * (uint32_t)rows_full);
-          const int z = c.b * a.q_len + rt * a.qpt;
-          tma_load_3d(q_smem + qb * kQBuf, &maps.q, 0, kvh * a.group, z, &S.q_full[qb]);
-          tma_load_3d(q_smem + qb * kQBuf + kQRegion, &maps.q, 64, kvh * a.group, z,
-                      &S.q_full[qb]);
-          ++q_i;
-          prev_x = x;
-        }
         const int slot = i % kStages;
         if (!mbar_wait(&S.kv_empty[slot], ((i / kStages) & 1) ^ 1)) { failed = true; break; }
         const ChunkInfo ci = chunk_info(c.j, S.lp[c.b], S.ls[c.b], a.D);
@@ -287,12 +277,25 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         tma_load_2d(dst + kKVRegion, mk, 64, row, &S.kv_full[slot]);
         tma_load_2d(dst + 2 * kKVRegion, mv, 0, row, &S.kv_full[slot]);
         tma_load_2d(dst + 3 * kKVRegion, mv, 64, row, &S.kv_full[slot]);
+        // A new item's Q goes after its first K/V, so that load overlaps the
+        // wait for the previous item's last S to release the Q buffer.
+        if (x != prev_x) {
+          const int qb = q_i % kQBufs;
+          if (!mbar_wait(&S.q_empty[qb], ((q_i / kQBufs) & 1) ^ 1)) { failed = true; break; }
+          mbar_arrive_expect_tx(&S.q_full[qb], 2u * 128u * (uint32_t)rows_full);
+          const int z = c.b * a.q_len + rt * a.qpt;
+          tma_load_3d(q_smem + qb * kQBuf, &maps.q, 0, kvh * a.group, z, &S.q_full[qb]);
+          tma_load_3d(q_smem + qb * kQBuf + kQRegion, &maps.q, 64, kvh * a.group, z,
+                      &S.q_full[qb]);
+          ++q_i;
+          prev_x = x;
+        }
       }
       // Drain: every load issued has landed before this CTA can exit.
       for (int m = max(0, n_my - kStages); m < n_my; ++m)
         if (!mbar_wait(&S.kv_full[m % kStages], (m / kStages) & 1)) failed = true;
-      for (int m = max(0, q_i - 2); m < q_i; ++m)
-        if (!mbar_wait(&S.q_full[m & 1], (m >> 1) & 1)) failed = true;
+      for (int m = max(0, q_i - kQBufs); m < q_i; ++m)
+        if (!mbar_wait(&S.q_full[m % kQBufs], (m / kQBufs) & 1)) failed = true;
     }
   } else if (c_begin < c_end && warp == 1) {
     // -------------------------------------------------------------- MMA
@@ -311,16 +314,16 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         if (is < n_my) {
           const int x = cs.b * per_seq + cs.it;
           const bool first = x != prev_xs;
-          const int slot = is % kStages, sb = is & 1;
-          bool ready = first ? mbar_test(&S.q_full[q_s & 1], (q_s >> 1) & 1) : true;
+          const int slot = is % kStages, sb = is % kSB;
+          bool ready = first ? mbar_test(&S.q_full[q_s % kQBufs], (q_s / kQBufs) & 1) : true;
           ready = ready && mbar_test(&S.kv_full[slot], (is / kStages) & 1) &&
-                  mbar_test(&S.s_empty[sb], ((is >> 1) & 1) ^ 1);
+                  mbar_test(&S.s_empty[sb], ((is / kSB) & 1) ^ 1);
           if (ready) {
             if (first) {
               ++q_s;
               prev_xs = x;
             }
-            const int qb = (q_s - 1) & 1;
+            const int qb = (q_s - 1) % kQBufs;
             const bool last = (is + 1 == n_my) || (cs.j + 1 == S.nc[cs.b]);
             tc_fence_after();
             const uint32_t q_base = smem_u32(q_smem + qb * kQBuf);
@@ -341,26 +344,24 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         if (ip < is) {
           const int x = cp.b * per_seq + cp.it;
           const bool first = x != prev_xp;
-          const int pb = ip & 1, vslot = ip % kStages, ob = o_i & 1;
-          bool ready = mbar_test(&S.p_full[pb], (ip >> 1) & 1);
-          if (first) ready = ready && mbar_test(&S.o_empty[ob], ((o_i >> 1) & 1) ^ 1);
+          const int pb = ip % kSB, vslot = ip % kStages;
+          bool ready = mbar_test(&S.p_full[pb], (ip / kSB) & 1);
+          if (first) ready = ready && mbar_test(&S.o_empty[0], (o_i & 1) ^ 1);
           if (ready) {
             if (first) prev_xp = x;
             const bool last = (ip + 1 == n_my) || (cp.j + 1 == S.nc[cp.b]);
             tc_fence_after();
-            const uint32_t p_base = smem_u32(p_smem + pb * kPBuf);
             const uint32_t v_base = smem_u32(kv_smem + vslot * kKVSlot + 2 * kKVRegion);
-            const uint32_t d_o = tmem + 128u + (uint32_t)ob * 128u;
+            const uint32_t p_tmem = tmem + (uint32_t)pb * kCh;  // P over its S columns
+            const uint32_t d_o = tmem + kOCol;
 #pragma unroll
-            for (int k = 0; k < kCh / 16; ++k)
-              mma_bf16(d_o, desc_k_sw128(p_base + k * 32),
-                       desc_mn_sw128(v_base + k * 2048, kKVRegion, 1024), id_pv,
-                       (first && k == 0) ? 0u : 1u);
+            for (int k = 0; k < kCh / 16; ++k)  // 16 keys = 8 packed columns of P
+              mma_bf16_ts(d_o, p_tmem + k * 8, desc_mn_sw128(v_base + k * 2048, kKVRegion, 1024),
+                          id_pv, (first && k == 0) ? 0u : 1u);
             mma_commit(&S.kv_empty[vslot]);
-            mma_commit(&S.p_empty[pb]);
-            mma_commit(&S.pv_done);
+            mma_commit(&S.s_empty[pb]);
             if (last) {
-              mma_commit(&S.o_full[ob]);
+              mma_commit(&S.o_full[0]);
               ++o_i;
             }
             advance(cp, S, per_seq);
@@ -370,9 +371,14 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         }
         if (progress) {
           t_last = clock64();
-        } else if (clock64() - t_last > kWaitCycles) {
-          failed = true;
-          break;
+        } else {
+          if (clock64() - t_last > kWaitCycles) {
+            failed = true;
+            break;
+          }
+          // Nothing ready: yield the issue slots this sub-partition shares
+          // with a softmax warp.
+          __nanosleep(64);
         }
       }
       mma_commit(&S.drain);
@@ -404,8 +410,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         prev_x = x;
       }
       const ChunkInfo ci = chunk_info(c.j, S.lp[c.b], S.ls[c.b], a.D);
-      const int sb = s_i & 1;
-      if (!mbar_wait(&S.s_full[sb], (s_i >> 1) & 1)) { failed = true; break; }
+      const int sb = s_i % kSB;
+      if (!mbar_wait(&S.s_full[sb], (s_i / kSB) & 1)) { failed = true; break; }
       tc_fence_after();
       uint32_t sr[64];
       if (warp_active) {
@@ -415,10 +421,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         tmem_ld_32x32b_x32(tmem + lane_addr + (uint32_t)sb * kCh + 32, hi);
         tmem_ld_wait();
       }
-      tc_fence_before();
-      mbar_arrive(&S.s_empty[sb]);
-      const int pb = s_i & 1;
-      if (!mbar_wait(&S.p_empty[pb], ((s_i >> 1) & 1) ^ 1)) { failed = true; break; }
+      const int pb = sb;
       if (warp_active) {
         float xs[64];
         float cmax = kEmptyMax;
@@ -436,9 +439,14 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         }
         // O rescale (warp-collective TMEM access) when any row needs it.
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          if (!mbar_wait(&S.pv_done, (s_i - 1) & 1)) { failed = true; }
+          // P V of the previous chunk must be done before O is touched; its
+          // S buffer's release says so (P V of chunk c - 1 - kSB is known
+          // complete because S of chunk c was issued, so the parity cannot
+          // be stale).
+          const int pq = (s_i - 1) % kSB;
+          if (!mbar_wait(&S.s_empty[pq], ((s_i - 1) / kSB) & 1)) { failed = true; }
           tc_fence_after();
-          const uint32_t o_addr = tmem + lane_addr + 128u + (uint32_t)(o_i & 1) * 128u;
+          const uint32_t o_addr = tmem + lane_addr + kOCol;
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             uint32_t ov[32];
@@ -461,12 +469,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
           pk[jj >> 1] = pack_bf16(p0, p1);
         }
         l += psum;
-        uint8_t* prow = p_smem + pb * kPBuf + r * 128;
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          *reinterpret_cast<uint4*>(prow + ((t ^ (r & 7)) * 16)) =
-              make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
-        fence_proxy_async_smem();
+        // P (bf16 pairs) over the first 32 columns of this chunk's S.
+        tmem_st_32x32b_x32(tmem + lane_addr + (uint32_t)pb * kCh, pk);
+        tmem_st_wait();
       }
       tc_fence_before();
       mbar_arrive(&S.p_full[pb]);
@@ -475,8 +480,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
       if (!last) continue;
 
       // ----------------------------------------------------- item epilogue
-      const int ob = o_i & 1;
-      if (!mbar_wait(&S.o_full[ob], (o_i >> 1) & 1)) { failed = true; break; }
+      if (!mbar_wait(&S.o_full[0], o_i & 1)) { failed = true; break; }
       tc_fence_after();
       const long long x_start = S.cb[c.b] + (long long)c.it * S.nc[c.b];
       const long long x_end = x_start + S.nc[c.b];
@@ -485,7 +489,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
       const int qi = rt * a.qpt + p_pos;
       const bool row_ok = r < rows;
       bf16* orow = a.out + (((size_t)c.b * a.q_len + qi) * a.Hq + kvh * a.group + jh) * 128;
-      const uint32_t o_addr = tmem + lane_addr + 128u + (uint32_t)ob * 128u;
+      const uint32_t o_addr = tmem + lane_addr + kOCol;
       if (cta_lo == cta_hi) {
         const float inv = 1.f / l;
         if (warp_active) {
@@ -508,7 +512,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
           }
         }
         tc_fence_before();
-        mbar_arrive(&S.o_empty[ob]);
+        mbar_arrive(&S.o_empty[0]);
         ++o_i;
         continue;
       }
@@ -532,7 +536,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         if (row_ok) a.part_ml[(size_t)slot * 128 + r] = make_float2(m_used, l);
       }
       tc_fence_before();
-      mbar_arrive(&S.o_empty[ob]);
+      mbar_arrive(&S.o_empty[0]);
       ++o_i;
     }
   }
@@ -541,7 +545,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kTmemCols);
   }
   if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
   // This CTA is done: the merge kernel may be scheduled once every CTA got
@@ -710,7 +714,7 @@ int attn_tc_qpt(int q_len, int group) {
 }
 
 size_t attn_tc_smem_bytes() {
-  return 1024 + 2 * kQBuf + kStages * kKVSlot + 2 * kPBuf + sizeof(Smem);
+  return 1024 + kQBufs * kQBuf + kStages * kKVSlot + sizeof(Smem);
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,

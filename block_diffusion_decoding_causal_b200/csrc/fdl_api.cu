@@ -132,7 +132,7 @@ int run_attention(const fdl_step_cfg& c, const Plan& p, bool dual, const void* q
   cudaError_t e = p.attn_tc
                       ? launch_attn_tc(a, at<float>(ws, p.off_tc_part_o),
                                        at<float2>(ws, p.off_tc_part_ml), a.tickets,
-                                       kPlanCTAs, s)
+                                       kAttnTcCTAs, s)
                       : launch_attn_simt(a, (fdl_dtype)c.dtype, kAttnRowTile, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return FDL_OK;

@@ -12,6 +12,7 @@ namespace fdl {
 constexpr int kAttnRowTile = 16;   // query rows per attention CTA
 constexpr int kPlanCTAs = 148;     // grid sizing unit: one B200's SM count
 constexpr int kLmMaxCTAs = 4 * kPlanCTAs;
+constexpr int kAttnTcCTAs = 2 * kPlanCTAs;  // tensor-core attention: two CTAs per SM
 
 struct AttnSplit {
   int split_keys;  // keys per split, multiple of 64
@@ -115,9 +116,9 @@ inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why) {
   p->off_tc_part_o = off;
   p->off_tc_part_ml = off;
   if (p->attn_tc) {
-    off = align256(off + sizeof(float) * 2 * (size_t)kPlanCTAs * 128 * 128);
+    off = align256(off + sizeof(float) * 2 * (size_t)kAttnTcCTAs * 128 * 128);
     p->off_tc_part_ml = off;
-    off = align256(off + 8 * 2 * (size_t)kPlanCTAs * 128);
+    off = align256(off + 8 * 2 * (size_t)kAttnTcCTAs * 128);
   }
   p->total = off;
   return true;

@@ -265,3 +265,21 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 
 }  // namespace sm100
 }  // namespace fdl
+
+namespace fdl {
+namespace sm100 {
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16.  A (M = 128) sits in
+// TMEM with row m in lane m and K packed two 16-bit values per column.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+}  // namespace sm100
+}  // namespace fdl
