@@ -314,6 +314,8 @@ def main():
     for i in range(3):
         attn(i)
     t_attn = max_over_ranks(timed(attn, args.steps), world) / args.steps
+    pc = prefixcache_leg(torch, fdl, stream, timed, world, args.steps, peaks)
+    lm_big = large_batch_lm_leg(torch, fdl, synth, stream, timed, world, args.steps, peaks)
 
     # End to end through the public API: per step, pinned host inputs copied
     # in, the step, and its results copied out and read on the host.
@@ -358,6 +360,12 @@ def main():
 
     lm_bytes = V * H * 2 + B * q_len * H * 2 + B * q_len * 8
     lm_gbs = lm_bytes / t_lm / 1e9
+    # Algorithmic bytes of the attention (K and V of every visible key, Q in,
+    # O out) and of the whole step (attention + LM head + the token shift).
+    d, Hq, Hkv, D = c["head_dim"], c["n_q_heads"], c["n_kv_heads"], c["block_size"]
+    keys = int(case.len_pre.sum()) + B * D
+    attn_bytes = keys * Hkv * 2 * d * 2 + 2 * B * q_len * Hq * d * 2
+    step_bytes = attn_bytes + lm_bytes + (B * q_len * H * 2 * 2 if c["shift"] else 0)
     traffic = _profiled_traffic("lmhead", "lmhead_tc_qwen7b.md")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -372,7 +380,12 @@ def main():
                      "peak_source": f"{peaks['source']} hbm_gbs (burst copy)",
                      "traffic": traffic, "bytes_per_launch": lm_bytes,
                      "us_per_launch": t_lm * 1e6},
-        "attention": {"us_per_launch": t_attn * 1e6},
+        "attention": {"us_per_launch": t_attn * 1e6, "bytes_per_launch": attn_bytes,
+                      "achieved_gbs": attn_bytes / t_attn / 1e9},
+        "step_roofline": {"bytes": step_bytes, "achieved_gbs": step_bytes / (t_step / args.steps) / 1e9,
+                          "frac": step_bytes / (t_step / args.steps) / 1e9 / peaks["hbm_gbs"]},
+        "prefixcache": pc,
+        "lmhead_large_batch": lm_big,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e / args.steps * 1e3},
         "gpu_launches": _launches_per_step(c) * args.steps,
@@ -388,6 +401,72 @@ def main():
     return 0
 
 
+PREFIXCACHE = dict(batch=1, n_q_heads=32, n_kv_heads=32, head_dim=128, prefix=768, rows=768)
+
+
+def prefixcache_leg(torch, fdl, stream, timed, world, steps, peaks) -> dict:
+    """PrefixCache attention at LLaDA-8B shapes: prompt 512 + 8 finished
+    blocks cached (768 rows), answer length 1024 at block 9, so the active
+    block and the masked suffix are 32 + 736 = 768 recomputed rows.  Eight
+    input sets rotate (about 300 MB, more than L2)."""
+    c = PREFIXCACHE
+    B, Hq, Hkv, d, Lp, n = (c[k] for k in ("batch", "n_q_heads", "n_kv_heads", "head_dim",
+                                           "prefix", "rows"))
+    cfg = fdl.make_cfg(dict(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, block_size=n,
+                            q_off=0, q_len=n, cap_prefix=Lp, hidden=128, vocab=1000,
+                            mask_id=999, shift=0, tau=0.9, dtype="bf16"))
+    g = torch.Generator(device="cuda").manual_seed(7)
+    rn = lambda *sh: torch.randn(sh, generator=g, device="cuda").to(torch.bfloat16)
+    with torch.cuda.stream(stream):
+        sets = [dict(q=rn(B, n, Hq, d), kp=rn(B, Hkv, Lp, d), vp=rn(B, Hkv, Lp, d),
+                     kn=rn(B, Hkv, n, d), vn=rn(B, Hkv, n, d)) for _ in range(8)]
+        lens = torch.full((B,), Lp, dtype=torch.int32, device="cuda")
+        out = torch.empty((B, n, Hq, d), dtype=torch.bfloat16, device="cuda")
+        ws = fdl.workspace(cfg)
+    stream.synchronize()
+
+    def run(i):
+        x = sets[i % 8]
+        fdl.prefixcache_attn(cfg, x["q"], x["kp"], x["vp"], lens, x["kn"], x["vn"], out, ws,
+                             stream)
+    for i in range(3):
+        run(i)
+    t = max_over_ranks(timed(run, steps), world) / steps
+    flops = 4.0 * B * Hq * n * (Lp + n) * d
+    bytes_ = B * Hkv * (Lp + n) * d * 2 * 2 + 2 * B * n * Hq * d * 2
+    bound = "tensor" if flops / (peaks["bf16_tflops"] * 1e12) > bytes_ / (peaks["hbm_gbs"] * 1e9) \
+        else "hbm"
+    return {"workload": "LLaDA-8B shapes, 32/32 heads, d 128, 768 cached + 768 recomputed rows",
+            "us_per_launch": t * 1e6, "flops": flops, "bytes": bytes_, "bound": bound,
+            "tflops": flops / t / 1e12, "frac_tensor": flops / t / 1e12 / peaks["bf16_tflops"],
+            "gbs": bytes_ / t / 1e9, "frac_hbm": bytes_ / t / 1e9 / peaks["hbm_gbs"]}
+
+
+def large_batch_lm_leg(torch, fdl, synth, stream, timed, world, steps, peaks) -> dict:
+    """The LM head past the ridge: Qwen2.5-7B vocabulary, 64 sequences x 8
+    positions = 512 rows, two passes of 256 rows over the weight."""
+    c = dict(synth.CONFIGS["qwen7b"], batch=64, q_off=0)
+    cfg = fdl.make_cfg(c)
+    R, H, V = c["batch"] * c["q_len"], c["hidden"], c["vocab"]
+    g = torch.Generator(device="cuda").manual_seed(11)
+    with torch.cuda.stream(stream):
+        w = (torch.randn((V, H), generator=g, device="cuda") * (8.0 / H ** 0.5)).to(torch.bfloat16)
+        rows = torch.randn((R, H), generator=g, device="cuda").to(torch.bfloat16)
+        conf = torch.empty(R, dtype=torch.float32, device="cuda")
+        tok = torch.empty(R, dtype=torch.int32, device="cuda")
+        ws = fdl.workspace(cfg)
+    stream.synchronize()
+    run = lambda i: fdl.lmhead_confidence(cfg, rows, w, None, conf, tok, ws, stream)
+    for i in range(3):
+        run(i)
+    t = max_over_ranks(timed(run, steps), world) / steps
+    flops = 2.0 * V * H * R
+    del w
+    return {"workload": "Qwen2.5-7B vocabulary, 512 rows (64 x 8), 2 passes",
+            "us_per_launch": t * 1e6, "flops": flops, "bound": "tensor",
+            "tflops": flops / t / 1e12, "frac_tensor": flops / t / 1e12 / peaks["bf16_tflops"]}
+
+
 def _gpu_id(torch) -> str:
     """nvidia-smi identifier (UUID) of the current CUDA device."""
     try:
@@ -398,9 +477,14 @@ def _gpu_id(torch) -> str:
 
 
 def _launches_per_step(c) -> int:
-    """Kernels one fdl_denoise_step launches at these shapes: attention and
-    its partial merge, the token-shift gather, the fused LM head + commit."""
-    return 4 if c["shift"] else 3
+    """Kernels one fdl_denoise_step launches at these shapes.  bf16, head
+    dim 128, hidden rows given and at most 64 LM-head rows: the token-shift
+    gather (if shifting), the fused LM head + commit, and the attention beside
+    it; otherwise attention, its partial merge, the gather (if shifting) and
+    the LM head."""
+    beside = (c["dtype"] == "bf16" and c["head_dim"] == 128
+              and c["batch"] * c["q_len"] <= 64)
+    return (2 if beside else 3) + (1 if c["shift"] else 0)
 
 
 KERNEL_SOURCES = {

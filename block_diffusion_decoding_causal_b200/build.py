@@ -74,8 +74,11 @@ def build(force: bool = False, verbose: bool = False) -> str:
     with concurrent.futures.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose), _sources()))
     tmp = LIB + ".tmp"
+    vmap = os.path.join(BUILD, "fdl.map")
+    with open(vmap, "w") as f:
+        f.write("{ global: fdl_*; local: *; };\n")  # export only the C ABI
     cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs + [
-        "-lrt", "-ldl", "-lpthread"]
+        "-lrt", "-ldl", "-lpthread", "-Xlinker", "--version-script=" + vmap]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}{r.stderr}")

@@ -7,24 +7,28 @@
 // sharing the KV head (GQA packing: 8 x 7 = 56 rows at Qwen2.5-7B shapes),
 // padded to the M = 128 tile.
 //
-// Stream-K split: every CTA (one per SM) reads the per-sequence lengths,
-// cuts the concatenation of all items' 64-key chunks into equal contiguous
-// ranges and takes its own, so the split follows the actual lengths and a CTA
-// produces at most two partial results (its first and last item); items it
-// covers whole are written out directly.  Per chunk:
-//   warp 0   TMA: K and V [64 keys x 128] in four 8 KB boxes (128-byte
-//            swizzle) through a 3-slot ring; Q of each item by a 3D box
-//            (d, head group, positions) into one of two Q buffers;
+// Stream-K split: every CTA reads the per-sequence lengths, cuts the
+// concatenation of all items' 64-key chunks into equal contiguous ranges and
+// takes its own, so the split follows the actual lengths and a CTA produces
+// at most two partial results (its first and last item); items it covers
+// whole are written out directly.  Per chunk:
+//   warp 0   TMA: K and V [64 keys x 128] as one 32 KB stage (four 8 KB boxes,
+//            128-byte swizzle, one barrier) through a STAGES-deep ring; Q of
+//            each item by a 3D box (d, head group, positions);
 //   warp 1   tcgen05.mma: S = Q K^T (M 128, N 64, K 128) into one of two TMEM
-//            S buffers, then, one chunk behind, O += P V (M 128, N 128, K 64,
-//            V read MN-major) into the item's TMEM O buffer;
+//            S buffers, then, one chunk behind, O += P V (M 128, N 128, K 64)
+//            with P read from TMEM and V MN-major from shared memory, into
+//            the item's TMEM O buffer;
 //   warps 2-5  softmax, one thread per row: S from TMEM, online max with a
 //            lazy rescale (O in TMEM is rescaled only when the running max
-//            grows by more than 2^8), P = exp2(S - m) as bf16 into shared
-//            memory (swizzled K-major), and the item epilogue.
-// Partial results (unnormalised O, m, l) go to the workspace; a small merge
-// kernel, launched as a programmatic dependent of this grid, combines the
-// partials of every item that was split.  No thread waits on another CTA.
+//            grows by more than 2^8), P = exp2(S - m) as bf16 written back
+//            over its S columns, and the item epilogue.
+// Partial results (unnormalised O, m, l) go to the workspace.  Alone on the
+// GPU (two CTAs per SM, two stages each) a small merge kernel, launched as a
+// programmatic dependent of this grid, combines them.  Beside the LM head
+// (one CTA per SM, one stage, leaving the SM's other room to that kernel)
+// the thread that writes a row's last partial merges the row itself.
+// No thread waits on another CTA.
 #include <cudaTypedefs.h>
 
 #include "fdl_common.cuh"
@@ -40,14 +44,20 @@ constexpr int kQRegion = 128 * 128;      // 128 rows x 64 bf16 (16 KB)
 constexpr int kQBuf = 2 * kQRegion;      // d 0-63 and 64-127
 constexpr int kKVRegion = kCh * 128;     // 64 keys x 64 bf16 (8 KB)
 constexpr int kKVSlot = 4 * kKVRegion;   // K lo, K hi, V lo, V hi: one 32 KB stage
-constexpr int kStages = 2;              // K/V stages (two CTAs share an SM)
+// K/V stages of the attention alone on the GPU (two CTAs per SM at 2) and
+// beside the LM head (1).
+#ifndef FDL_ATTN_ALONE_STAGES
+#define FDL_ATTN_ALONE_STAGES 2
+#endif
+constexpr int kAloneStages = FDL_ATTN_ALONE_STAGES;
+constexpr int kMaxStages = kAloneStages > 1 ? kAloneStages : 1;
 constexpr int kQBufs = 1;                // Q is reloaded per item
 constexpr int kSB = 2;                   // S buffers in TMEM; P overwrites its S
 constexpr uint32_t kTmemCols = 256;      // S 2 x 64 columns, O 128 columns
 constexpr uint32_t kOCol = kSB * 64;     // first column of O
 constexpr int kThreads = 192;
 constexpr float kRescale = 8.0f;         // log2-domain growth forcing a rescale
-constexpr unsigned kDevTimeout = 4u;
+constexpr unsigned kDevTimeout = FDL_DEV_TIMEOUT;
 constexpr int kMaxSeq = 256;
 
 struct TcArgs {
@@ -57,9 +67,10 @@ struct TcArgs {
   const int32_t* len_suf;
   bf16* out;
   Control* ctrl;
-  unsigned int* tickets;  // one per item
+  unsigned int* tickets;  // [items][128]: arrivals per (item, tile row)
   float* part_o;          // [2 * n_cta][128][128]
   float2* part_ml;        // [2 * n_cta][128]
+  int inline_merge;       // the last CTA to finish a row of an item merges it
 };
 
 struct Maps {
@@ -67,7 +78,7 @@ struct Maps {
 };
 
 struct Smem {
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t kv_full[kMaxStages], kv_empty[kMaxStages];
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[kSB], s_empty[kSB];   // S ready / S and its P free again
   uint64_t p_full[kSB];                 // P written into TMEM
@@ -132,50 +143,116 @@ struct ChunkInfo {
   int nvalid;  // valid keys in the chunk
 };
 
+// Chunks of one item: the prefix, the block rows (one chunk up to 64 rows;
+// more when the recomputed rows of PrefixCache take the block's place) and
+// the suffix, each cut into 64-key chunks.
+__device__ __forceinline__ int item_chunks(int Lp, int Ls, int D) {
+  return (Lp + kCh - 1) / kCh + (D + kCh - 1) / kCh + (Ls + kCh - 1) / kCh;
+}
+
 __device__ __forceinline__ ChunkInfo chunk_info(int j, int Lp, int Ls, int D) {
   const int ncp = (Lp + kCh - 1) / kCh;
+  const int ncb = (D + kCh - 1) / kCh;
   ChunkInfo ci;
   if (j < ncp) {
     ci.seg = 0;
     ci.key0 = j * kCh;
     ci.nvalid = min(kCh, Lp - ci.key0);
-  } else if (j == ncp) {
+  } else if (j < ncp + ncb) {
     ci.seg = 1;
-    ci.key0 = 0;
-    ci.nvalid = D;
+    ci.key0 = (j - ncp) * kCh;
+    ci.nvalid = min(kCh, D - ci.key0);
   } else {
     ci.seg = 2;
-    ci.key0 = (j - ncp - 1) * kCh;
+    ci.key0 = (j - ncp - ncb) * kCh;
     ci.nvalid = min(kCh, Ls - ci.key0);
   }
-  (void)Ls;
   return ci;
 }
 
-__device__ __forceinline__ void named_barrier_softmax() {
-  asm volatile("bar.sync 2, 128;" ::: "memory");
-}
+
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// Partial slot of CTA j for the item whose chunks start at x_start: slot
+// 2j holds a CTA's first item, 2j + 1 its last (when it is a different one).
+__device__ __forceinline__ int partial_slot(int j, int cta_lo, long long x_start, long long T,
+                                            int n) {
+  return 2 * j + ((j == cta_lo && cta_start(j, T, n) != x_start) ? 1 : 0);
+}
+
+// Merge of one row of one item inside the attention kernel, by the thread
+// of the CTA that wrote the row's last partial (used when the grid runs
+// beside the LM head, where a separate merge launch would wait for that
+// kernel).  The partials (O, m, l) of the CTAs cta_lo..cta_hi are combined
+// with the usual max/sum rescaling, 32 columns at a time.
+__device__ __noinline__ void merge_row_inline(const TcArgs& a, int r, int cta_lo, int cta_hi,
+                                              long long x_start, long long T, int n,
+                                              bf16* orow) {
+  float M = kEmptyMax;
+  for (int j = cta_lo; j <= cta_hi; ++j) {
+    if (!cta_nonempty(j, T, n)) continue;
+    M = fmaxf(M, __ldcg(&a.part_ml[(size_t)partial_slot(j, cta_lo, x_start, T, n) * 128 + r]).x);
+  }
+  float L = 0.f;
+  for (int j = cta_lo; j <= cta_hi; ++j) {
+    if (!cta_nonempty(j, T, n)) continue;
+    const float2 ml = __ldcg(&a.part_ml[(size_t)partial_slot(j, cta_lo, x_start, T, n) * 128 + r]);
+    L += ml.y * exp2f(ml.x - M);
+  }
+  const float inv = 1.f / L;
+  for (int cc = 0; cc < 4; ++cc) {
+    float acc[32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t) acc[t] = 0.f;
+    for (int j = cta_lo; j <= cta_hi; ++j) {
+      if (!cta_nonempty(j, T, n)) continue;
+      const int sl = partial_slot(j, cta_lo, x_start, T, n);
+      const float w = exp2f(__ldcg(&a.part_ml[(size_t)sl * 128 + r]).x - M);
+      const float4* src =
+          reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128 + cc * 32);
+      float4 v[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) v[t] = __ldcg(src + t);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        acc[4 * t] += v[t].x * w;
+        acc[4 * t + 1] += v[t].y * w;
+        acc[4 * t + 2] += v[t].z * w;
+        acc[4 * t + 3] += v[t].w * w;
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      uint4 o;
+      o.x = pack_bf16(acc[8 * t + 0] * inv, acc[8 * t + 1] * inv);
+      o.y = pack_bf16(acc[8 * t + 2] * inv, acc[8 * t + 3] * inv);
+      o.z = pack_bf16(acc[8 * t + 4] * inv, acc[8 * t + 5] * inv);
+      o.w = pack_bf16(acc[8 * t + 6] * inv, acc[8 * t + 7] * inv);
+      *reinterpret_cast<uint4*>(orow + cc * 32 + 8 * t) = o;
+    }
+  }
+}
+
+template <int STAGES>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_smem = base;                          // kQBufs x 32 KB
-  uint8_t* kv_smem = q_smem + kQBufs * kQBuf;      // kStages x 32 KB
-  Smem& S = *reinterpret_cast<Smem*>(kv_smem + kStages * kKVSlot);
+  uint8_t* kv_smem = q_smem + kQBufs * kQBuf;      // STAGES x 32 KB
+  Smem& S = *reinterpret_cast<Smem*>(kv_smem + STAGES * kKVSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_seq = a.Hkv * a.n_rt;  // items per sequence
   const int rows_full = a.qpt * a.group;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < STAGES; ++i) {
       mbar_init(&S.kv_full[i], 1);
       mbar_init(&S.kv_empty[i], 1);
     }
@@ -213,7 +290,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
             Ls = 0;
           }
         }
-        nc = (Lp + kCh - 1) / kCh + 1 + (Ls + kCh - 1) / kCh;
+        nc = item_chunks(Lp, Ls, a.D);
       }
       int incl = nc * per_seq;
 #pragma unroll
@@ -263,14 +340,14 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
       for (int i = 0; i < n_my && !failed; ++i, advance(c, S, per_seq)) {
         const int x = c.b * per_seq + c.it;
         const int kvh = c.it / a.n_rt, rt = c.it % a.n_rt;
-        const int slot = i % kStages;
-        if (!mbar_wait(&S.kv_empty[slot], ((i / kStages) & 1) ^ 1)) { failed = true; break; }
+        const int slot = i % STAGES;
+        if (!mbar_wait(&S.kv_empty[slot], ((i / STAGES) & 1) ^ 1)) { failed = true; break; }
         const ChunkInfo ci = chunk_info(c.j, S.lp[c.b], S.ls[c.b], a.D);
         const int bk = c.b * a.Hkv + kvh;
         const CUtensorMap* mk = ci.seg == 0 ? &maps.kp : (ci.seg == 1 ? &maps.kb : &maps.ks);
         const CUtensorMap* mv = ci.seg == 0 ? &maps.vp : (ci.seg == 1 ? &maps.vb : &maps.vs);
         const int row = ci.seg == 0 ? bk * a.cap_p + ci.key0
-                                    : (ci.seg == 1 ? bk * a.D : bk * a.cap_s + ci.key0);
+                                    : (ci.seg == 1 ? bk * a.D + ci.key0 : bk * a.cap_s + ci.key0);
         uint8_t* dst = kv_smem + slot * kKVSlot;
         mbar_arrive_expect_tx(&S.kv_full[slot], kKVSlot);
         tma_load_2d(dst, mk, 0, row, &S.kv_full[slot]);
@@ -292,8 +369,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         }
       }
       // Drain: every load issued has landed before this CTA can exit.
-      for (int m = max(0, n_my - kStages); m < n_my; ++m)
-        if (!mbar_wait(&S.kv_full[m % kStages], (m / kStages) & 1)) failed = true;
+      for (int m = max(0, n_my - STAGES); m < n_my; ++m)
+        if (!mbar_wait(&S.kv_full[m % STAGES], (m / STAGES) & 1)) failed = true;
       for (int m = max(0, q_i - kQBufs); m < q_i; ++m)
         if (!mbar_wait(&S.q_full[m % kQBufs], (m / kQBufs) & 1)) failed = true;
     }
@@ -314,9 +391,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         if (is < n_my) {
           const int x = cs.b * per_seq + cs.it;
           const bool first = x != prev_xs;
-          const int slot = is % kStages, sb = is % kSB;
+          const int slot = is % STAGES, sb = is % kSB;
           bool ready = first ? mbar_test(&S.q_full[q_s % kQBufs], (q_s / kQBufs) & 1) : true;
-          ready = ready && mbar_test(&S.kv_full[slot], (is / kStages) & 1) &&
+          ready = ready && mbar_test(&S.kv_full[slot], (is / STAGES) & 1) &&
                   mbar_test(&S.s_empty[sb], ((is / kSB) & 1) ^ 1);
           if (ready) {
             if (first) {
@@ -344,7 +421,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         if (ip < is) {
           const int x = cp.b * per_seq + cp.it;
           const bool first = x != prev_xp;
-          const int pb = ip % kSB, vslot = ip % kStages;
+          const int pb = ip % kSB, vslot = ip % STAGES;
           bool ready = mbar_test(&S.p_full[pb], (ip / kSB) & 1);
           if (first) ready = ready && mbar_test(&S.o_empty[0], (o_i & 1) ^ 1);
           if (ready) {
@@ -538,6 +615,19 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
       tc_fence_before();
       mbar_arrive(&S.o_empty[0]);
       ++o_i;
+      if (a.inline_merge && row_ok) {
+        // "Last to arrive" per (item, row): publish this partial, count it;
+        // the thread that completes the count merges the row and rearms it.
+        __threadfence();
+        int parts = 0;
+        for (int j = cta_lo; j <= cta_hi; ++j) parts += cta_nonempty(j, T, n) ? 1 : 0;
+        unsigned int* tk = a.tickets + (size_t)x * 128 + r;
+        if (atomicAdd(tk, 1u) == (unsigned int)(parts - 1)) {
+          *tk = 0u;
+          __threadfence();
+          merge_row_inline(a, r, cta_lo, cta_hi, x_start, T, n, orow);
+        }
+      }
     }
   }
 
@@ -551,6 +641,10 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   // This CTA is done: the merge kernel may be scheduled once every CTA got
   // here (it still waits for the whole grid before reading anything).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // When launched beside the step's LM head, finish only after it did, so
+  // that this grid's completion (which the merge waits for) covers both.
+  // Without a programmatic predecessor this returns at once.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Merge of the partials of every item the split spread over several CTAs.
@@ -588,7 +682,7 @@ attn_merge_kernel(const TcArgs a) {
         Ls = a.len_suf[s2];
         if (Ls < 0 || Ls > a.cap_s) Ls = 0;
       }
-      nc = (Lp + kCh - 1) / kCh + 1 + (Ls + kCh - 1) / kCh;
+      nc = item_chunks(Lp, Ls, a.D);
     }
     int incl = nc * per_seq;
 #pragma unroll
@@ -612,7 +706,7 @@ attn_merge_kernel(const TcArgs a) {
   for (int t = 0; t < COLS; ++t) acc[t] = 0.f;
   for (int j = cta_lo + pg; j <= cta_hi; j += PG) {
     if (!cta_nonempty(j, T, n)) continue;
-    const int sl = 2 * j + ((j == cta_lo && cta_start(j, T, n) != x_start) ? 1 : 0);
+    const int sl = partial_slot(j, cta_lo, x_start, T, n);
     const float2 ml = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
     const float4* src =
         reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128 + cg * COLS);
@@ -713,12 +807,13 @@ int attn_tc_qpt(int q_len, int group) {
   return qpt < q_len ? qpt : q_len;
 }
 
-size_t attn_tc_smem_bytes() {
-  return 1024 + kQBufs * kQBuf + kStages * kKVSlot + sizeof(Smem);
+size_t attn_tc_smem_bytes(int stages) {
+  return 1024 + kQBufs * kQBuf + stages * kKVSlot + sizeof(Smem);
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
-                           unsigned int* tickets, int n_cta, cudaStream_t s) {
+                           unsigned int* tickets, int n_cta, cudaStream_t s,
+                           bool beside_prior) {
   const int qpt = attn_tc_qpt(a.q_len, a.group);
   if (a.d != 128 || qpt == 0 || a.B > kMaxSeq) return cudaErrorInvalidValue;
   Maps maps;
@@ -761,22 +856,39 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   t.tickets = tickets;
   t.part_o = part_o;
   t.part_ml = part_ml;
-  const size_t smem = attn_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  t.inline_merge = beside_prior ? 1 : 0;
+  // Beside the LM head: one K/V stage, so the SM's remaining shared memory
+  // goes to that kernel's weight ring.
+  const int stages = beside_prior ? 1 : kAloneStages;
+  const size_t smem = attn_tc_smem_bytes(stages);
+  auto kern = beside_prior ? attn_tc_kernel<1> : attn_tc_kernel<kAloneStages>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<<<n_cta, kThreads, smem, s>>>(maps, t);
-  e = cudaGetLastError();
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  {
+    cudaLaunchConfig_t mc = {};
+    mc.gridDim = dim3(n_cta, 1, 1);
+    mc.blockDim = dim3(kThreads, 1, 1);
+    mc.dynamicSmemBytes = smem;
+    mc.stream = s;
+    mc.attrs = attr;
+    mc.numAttrs = beside_prior ? 1 : 0;
+    e = cudaLaunchKernelEx(&mc, kern, maps, t);
+    if (e != cudaSuccess) return e;
+  }
+  if (beside_prior) return cudaSuccess;  // merged inside the kernel
   cudaLaunchConfig_t lc = {};
   const int n_items = a.B * a.Hkv * t.n_rt;
   lc.gridDim = dim3(n_items, (qpt * a.group + 7) / 8, 1);
   lc.blockDim = dim3(256, 1, 1);
   lc.dynamicSmemBytes = 0;
   lc.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
   // Partials per split item are about n_cta / n_items + 1 (the split is

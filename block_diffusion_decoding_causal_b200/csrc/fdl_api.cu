@@ -121,18 +121,34 @@ LmArgs lm_args(const fdl_step_cfg& c, const Plan& p, const void* rows,
   return a;
 }
 
+// CTAs for the attention beside the LM head: the largest possible chunk
+// count (lengths at capacity) over about 32 chunks per CTA, between 1 and one
+// per SM.
+int attn_ctas_beside(const fdl_step_cfg& c, bool dual) {
+  const long group = c.n_q_heads / c.n_kv_heads;
+  const long qpt = 128 / group < c.q_len ? 128 / group : c.q_len;
+  const long items = (long)c.batch * c.n_kv_heads * ((c.q_len + qpt - 1) / qpt);
+  const long per_item = (c.cap_prefix + 63) / 64 + 1 + (dual ? (c.cap_suffix + 63) / 64 : 0);
+  const long want = (items * per_item + 31) / 32;
+  return (int)(want < 1 ? 1 : (want > kPlanCTAs ? kPlanCTAs : want));
+}
+
 int run_attention(const fdl_step_cfg& c, const Plan& p, bool dual, const void* q,
                   const void* k_pre, const void* v_pre, const int32_t* len_pre,
                   const void* k_blk, const void* v_blk, const void* k_suf,
                   const void* v_suf, const int32_t* len_suf, void* out, void* ws,
-                  cudaStream_t s) {
+                  cudaStream_t s, bool beside_lmhead = false) {
   AttnArgs a = attn_args(c, p, dual, q, k_pre, v_pre, len_pre, k_blk, v_blk,
                          k_suf, v_suf, len_suf, out, ws);
-  // bf16 with d = 128: tensor-core kernel; otherwise the CUDA-core kernel.
+  // bf16 with d = 128: tensor-core kernel (two CTAs per SM; beside the LM
+  // head, at most one per SM and only as many as keep about 32 chunks each,
+  // so that few partials need merging); otherwise the CUDA-core kernel.
   cudaError_t e = p.attn_tc
                       ? launch_attn_tc(a, at<float>(ws, p.off_tc_part_o),
-                                       at<float2>(ws, p.off_tc_part_ml), a.tickets,
-                                       kAttnTcCTAs, s)
+                                       at<float2>(ws, p.off_tc_part_ml),
+                                       at<unsigned int>(ws, p.off_tc_tickets),
+                                       beside_lmhead ? attn_ctas_beside(c, dual) : kAttnTcCTAs,
+                                       s, beside_lmhead)
                       : launch_attn_simt(a, (fdl_dtype)c.dtype, kAttnRowTile, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return FDL_OK;
@@ -146,10 +162,41 @@ int check_lmhead_supported(const fdl_step_cfg& c) {
   return FDL_OK;
 }
 
-int run_lmhead(const LmArgs& a, const fdl_step_cfg& c, cudaStream_t s) {
-  cudaError_t e = c.dtype == FDL_BF16 ? launch_lmhead_tc(a, s)
+int run_lmhead(const LmArgs& a, const fdl_step_cfg& c, cudaStream_t s, bool shared = false,
+               bool after_gather = false) {
+  cudaError_t e = c.dtype == FDL_BF16 ? launch_lmhead_tc(a, s, shared, after_gather)
                                       : launch_lmhead_simt(a, (fdl_dtype)c.dtype, s);
   if (e != cudaSuccess) return cuda_fail(e, "lm-head launch");
+  return FDL_OK;
+}
+
+// More rows than one pass holds (batch * q_len > 256): one pass per group of
+// whole sequences, each a full read of the weight.  At 256 rows a pass sits
+// at the ridge (as many FLOPs per weight byte as the tensor cores have per
+// HBM byte), so beyond it the passes cost what the arithmetic does.
+int run_lmhead_passes(const LmArgs& a, const fdl_step_cfg& c, const Plan& p, cudaStream_t s,
+                      bool shared = false, bool after_gather = false) {
+  if (a.R <= p.lm_pass_rows) return run_lmhead(a, c, s, shared, after_gather);
+  const size_t row_bytes = (size_t)c.hidden * p.elem;
+  for (int r0 = 0; r0 < a.R; r0 += p.lm_pass_rows) {
+    LmArgs pa = a;
+    const int b0 = r0 / c.q_len;
+    pa.R = a.R - r0 < p.lm_pass_rows ? a.R - r0 : p.lm_pass_rows;
+    pa.B = pa.R / c.q_len;
+    pa.rows = static_cast<const uint8_t*>(a.rows) + (size_t)r0 * row_bytes;
+    if (a.row_active != nullptr) pa.row_active = a.row_active + r0;
+    pa.conf = a.conf + r0;
+    pa.tok = a.tok + r0;
+    if (a.block_tokens_in != nullptr) pa.block_tokens_in = a.block_tokens_in + (size_t)b0 * c.block_size;
+    if (a.commit) {
+      pa.block_tokens = a.block_tokens + (size_t)b0 * c.block_size;
+      pa.committed = a.committed + (size_t)b0 * c.block_size;
+      pa.n_committed = a.n_committed + b0;
+      pa.n_masked_left = a.n_masked_left + b0;
+    }
+    const int rc = run_lmhead(pa, c, s, shared, after_gather && r0 == 0);
+    if (rc != FDL_OK) return rc;
+  }
   return FDL_OK;
 }
 
@@ -172,7 +219,7 @@ const char* fdl_last_error(void) { return g_err.c_str(); }
 size_t fdl_workspace_size(const fdl_step_cfg* cfg) {
   Plan p;
   std::string why;
-  if (!make_plan(cfg, &p, &why)) {
+  if (!make_plan(cfg, &p, &why, false)) {
     fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
     return 0;
   }
@@ -194,7 +241,7 @@ static int attn_common(const fdl_step_cfg* cfg, bool dual, const void* q,
                        void* ws, size_t ws_bytes, void* stream) {
   Plan p;
   std::string why;
-  if (!make_plan(cfg, &p, &why)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
+  if (!make_plan(cfg, &p, &why, false)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
   FDL_CHECK_PTR(q);
   FDL_CHECK_PTR(k_blk);
   FDL_CHECK_PTR(v_blk);
@@ -235,6 +282,20 @@ int fdl_dualcache_attn(const fdl_step_cfg* cfg, const void* q, const void* k_pre
                      v_suf, len_suf, out, ws, ws_bytes, stream);
 }
 
+int fdl_prefixcache_attn(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
+                         const void* v_pre, const int32_t* len_pre, const void* k_fresh,
+                         const void* v_fresh, void* out, void* ws, size_t ws_bytes,
+                         void* stream) {
+  if (cfg != nullptr && (cfg->q_off != 0 || cfg->q_len != cfg->block_size))
+    return fail(FDL_ERR_INVALID_ARG,
+                "PrefixCache queries are all recomputed rows: need q_off = 0 and "
+                "q_len = block_size (got %d, %d, %d)", cfg->q_off, cfg->q_len, cfg->block_size);
+  // The recomputed rows take the block's place: every key of
+  // [prefix | recomputed rows] is visible to every query.
+  return attn_common(cfg, false, q, k_pre, v_pre, len_pre, k_fresh, v_fresh, nullptr, nullptr,
+                     nullptr, out, ws, ws_bytes, stream);
+}
+
 int fdl_lmhead_confidence(const fdl_step_cfg* cfg, const void* rows,
                           const void* w_lm, const uint8_t* row_active,
                           float* conf, int32_t* tok, void* ws, size_t ws_bytes,
@@ -251,7 +312,7 @@ int fdl_lmhead_confidence(const fdl_step_cfg* cfg, const void* rows,
   rc = check_ws(p, ws, ws_bytes);
   if (rc != FDL_OK) return rc;
   LmArgs a = lm_args(*cfg, p, rows, w_lm, row_active, conf, tok, ws);
-  rc = run_lmhead(a, *cfg, (cudaStream_t)stream);
+  rc = run_lmhead_passes(a, *cfg, p, (cudaStream_t)stream);
   return rc != FDL_OK ? rc : ok();
 }
 
@@ -273,6 +334,71 @@ int fdl_threshold_commit(const fdl_step_cfg* cfg, const float* conf,
                                 cfg->q_off, cfg->q_len, cfg->mask_id, cfg->tau,
                                 (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "commit launch");
+  return ok();
+}
+
+int fdl_select_commit(const fdl_step_cfg* cfg, int policy, float param, const float* conf,
+                      const int32_t* tok, int32_t* block_tokens, uint8_t* committed,
+                      int32_t* n_committed, int32_t* n_masked_left, void* stream) {
+  Plan p;
+  std::string why;
+  if (!make_plan(cfg, &p, &why)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
+  if (policy != FDL_SELECT_THRESHOLD && policy != FDL_SELECT_FACTOR &&
+      policy != FDL_SELECT_BUDGET)
+    return fail(FDL_ERR_INVALID_ARG, "unknown selection policy %d", policy);
+  if (!std::isfinite(param)) return fail(FDL_ERR_INVALID_ARG, "param must be finite");
+  FDL_CHECK_PTR(conf);
+  FDL_CHECK_PTR(tok);
+  FDL_CHECK_PTR(block_tokens);
+  FDL_CHECK_PTR(committed);
+  FDL_CHECK_PTR(n_committed);
+  FDL_CHECK_PTR(n_masked_left);
+  cudaError_t e =
+      policy == FDL_SELECT_THRESHOLD
+          ? launch_commit(conf, tok, block_tokens, committed, n_committed, n_masked_left,
+                          cfg->batch, cfg->block_size, cfg->q_off, cfg->q_len, cfg->mask_id,
+                          param, (cudaStream_t)stream)
+          : launch_select_commit(policy, param, conf, tok, block_tokens, committed, n_committed,
+                                 n_masked_left, cfg->batch, cfg->block_size, cfg->q_off,
+                                 cfg->q_len, cfg->mask_id, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "select-commit launch");
+  return ok();
+}
+
+int fdl_unit_status(const fdl_step_cfg* cfg, const int32_t* n_masked_left,
+                    int32_t* any_masked, int32_t* step_count,
+                    unsigned long long while_handle, void* stream) {
+  Plan p;
+  std::string why;
+  if (!make_plan(cfg, &p, &why)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
+  if (n_masked_left == nullptr) return fail(FDL_ERR_INVALID_ARG, "n_masked_left is NULL");
+  if (while_handle != 0ull && step_count == nullptr)
+    return fail(FDL_ERR_INVALID_ARG, "a WHILE handle needs step_count (the loop bound)");
+  cudaError_t e = launch_unit_status(n_masked_left, cfg->batch, any_masked, step_count,
+                                     while_handle, cfg->q_len, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "unit-status launch");
+  return ok();
+}
+
+int fdl_append_block(const fdl_step_cfg* cfg, const void* k_blk, const void* v_blk, void* k_pre,
+                     void* v_pre, int32_t* len_pre, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  std::string why;
+  if (!make_plan(cfg, &p, &why, false)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
+  FDL_CHECK_PTR(k_blk);
+  FDL_CHECK_PTR(v_blk);
+  FDL_CHECK_PTR(k_pre);
+  FDL_CHECK_PTR(v_pre);
+  FDL_CHECK_PTR(len_pre);
+  if (cfg->cap_prefix < cfg->block_size)
+    return fail(FDL_ERR_INVALID_ARG, "cap_prefix is smaller than one block");
+  int rc = check_ws(p, ws, ws_bytes);
+  if (rc != FDL_OK) return rc;
+  cudaError_t e = launch_append_block(k_blk, v_blk, k_pre, v_pre, len_pre,
+                                      &at<Control>(ws, p.off_ctrl)->status, cfg->batch,
+                                      cfg->n_kv_heads, cfg->block_size, cfg->cap_prefix,
+                                      cfg->head_dim * p.elem, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "append-block launch");
   return ok();
 }
 
@@ -324,29 +450,59 @@ int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
   rc = check_ws(p, ws, ws_bytes);
   if (rc != FDL_OK) return rc;
   cudaStream_t s = (cudaStream_t)stream;
-
   void* out = attn_out != nullptr ? attn_out : at<void>(ws, p.off_attn);
+
+  auto lm_rows = [&](const void* src, const void** rows) -> int {
+    *rows = src;
+    if (c.shift) {
+      void* g = at<void>(ws, p.off_rows);
+      cudaError_t e = launch_gather_rows(src, h_prev, g, c.batch, c.q_len, c.hidden,
+                                         1, p.elem, s);
+      if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+      *rows = g;
+    }
+    return FDL_OK;
+  };
+  auto lm_fused = [&](const void* rows) {
+    LmArgs a = lm_args(c, p, rows, w_lm, nullptr, conf, tok, ws);
+    a.block_tokens_in = block_tokens;
+    a.commit = 1;
+    a.block_tokens = block_tokens;
+    a.committed = committed;
+    a.n_committed = n_committed;
+    a.n_masked_left = n_masked_left;
+    return a;
+  };
+
+  if (hidden != nullptr && p.attn_tc && c.dtype == FDL_BF16) {
+    // The LM-head rows are an input, so attention and the LM head are
+    // independent: the LM head goes first in its shared-SM form and the
+    // attention grid starts beside it, one CTA per SM, both streaming HBM.
+    const void* rows = nullptr;
+    rc = lm_rows(hidden, &rows);
+    if (rc != FDL_OK) return rc;
+    LmArgs a = lm_fused(rows);
+    if (lmhead_tc_shared_ok(a)) {
+      rc = run_lmhead(a, c, s, true, c.shift != 0);
+      if (rc != FDL_OK) return rc;
+      rc = run_attention(c, p, dual, q, k_pre, v_pre, len_pre, k_blk, v_blk, k_suf, v_suf,
+                         len_suf, out, ws, s, true);
+      return rc != FDL_OK ? rc : ok();
+    }
+    rc = run_attention(c, p, dual, q, k_pre, v_pre, len_pre, k_blk, v_blk, k_suf, v_suf,
+                       len_suf, out, ws, s);
+    if (rc != FDL_OK) return rc;
+    rc = run_lmhead_passes(a, c, p, s);
+    return rc != FDL_OK ? rc : ok();
+  }
+
   rc = run_attention(c, p, dual, q, k_pre, v_pre, len_pre, k_blk, v_blk, k_suf,
                      v_suf, len_suf, out, ws, s);
   if (rc != FDL_OK) return rc;
-
-  const void* src = hidden != nullptr ? hidden : out;
-  const void* rows = src;
-  if (c.shift) {
-    void* g = at<void>(ws, p.off_rows);
-    cudaError_t e = launch_gather_rows(src, h_prev, g, c.batch, c.q_len, c.hidden,
-                                       1, p.elem, s);
-    if (e != cudaSuccess) return cuda_fail(e, "gather launch");
-    rows = g;
-  }
-  LmArgs a = lm_args(c, p, rows, w_lm, nullptr, conf, tok, ws);
-  a.block_tokens_in = block_tokens;
-  a.commit = 1;
-  a.block_tokens = block_tokens;
-  a.committed = committed;
-  a.n_committed = n_committed;
-  a.n_masked_left = n_masked_left;
-  rc = run_lmhead(a, c, s);
+  const void* rows = nullptr;
+  rc = lm_rows(hidden != nullptr ? hidden : out, &rows);
+  if (rc != FDL_OK) return rc;
+  rc = run_lmhead_passes(lm_fused(rows), c, p, s, false, c.shift != 0);
   return rc != FDL_OK ? rc : ok();
 }
 

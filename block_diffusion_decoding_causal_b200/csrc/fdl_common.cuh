@@ -172,18 +172,125 @@ __device__ __forceinline__ void commit_sequence_warp(
   }
 }
 
+// Write the selection `sel` (bit i = unit position q_off + i) of sequence b:
+// tokens, the committed bitmap over the whole block, and the two counts.
+template <typename TokF>
+__device__ __forceinline__ void apply_selection_warp(
+    int b, int lane, int D, int q_off, int q_len, int mask_id, unsigned sel,
+    TokF tok_of, int32_t* block_tokens, uint8_t* committed, int32_t* n_committed,
+    int32_t* n_masked_left) {
+  int32_t* bt = block_tokens + (size_t)b * D;
+  const bool in_unit = lane < q_len;
+  const int p = q_off + lane;
+  int now = in_unit ? bt[p] : 0;
+  __syncwarp();
+  if (in_unit && ((sel >> lane) & 1u)) {
+    now = tok_of(lane);
+    bt[p] = now;
+  }
+  const unsigned left = __ballot_sync(0xffffffffu, in_unit && now == mask_id);
+  for (int j = lane; j < D; j += 32) {
+    const int jl = j - q_off;
+    const bool s = jl >= 0 && jl < 32 && ((sel >> jl) & 1u);
+    committed[(size_t)b * D + j] = s ? 1 : 0;
+  }
+  if (lane == 0) {
+    n_committed[b] = __popc(sel);
+    n_masked_left[b] = __popc(left);
+  }
+}
+
+// Factor rule (technical review, section 6, eq. 13 and Algorithm 3) and
+// heterogeneous-budget rule (section 5.1, eq. 9) for sequence b.  The unit's
+// still-masked positions are sorted by decreasing confidence (lower
+// position first on ties) with a 32-lane bitonic network; lane n-1 then
+// holds the n-th best.  The largest admissible n is taken (the first
+// position alone if none is admissible).
+constexpr int kSelectFactor = 1;
+constexpr int kSelectBudget = 2;
+
+template <typename ConfF>
+__device__ __forceinline__ unsigned ranked_selection_warp(int b, int lane, int D, int q_off,
+                                                          int q_len, int mask_id, int policy,
+                                                          float param, const int32_t* block_tokens,
+                                                          ConfF conf_of) {
+  const bool in_unit = lane < q_len;
+  const bool cand = in_unit && block_tokens[(size_t)b * D + q_off + lane] == mask_id;
+  float c = cand ? conf_of(lane) : -__int_as_float(0x7f800000);
+  int idx = lane;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const float c2 = __shfl_xor_sync(0xffffffffu, c, j);
+      const int i2 = __shfl_xor_sync(0xffffffffu, idx, j);
+      const bool self_first = c > c2 || (c == c2 && idx < i2);
+      const bool up = (lane & k) == 0, lower = (lane & j) == 0;
+      const bool keep = (lower == up) ? self_first : !self_first;
+      if (!keep) {
+        c = c2;
+        idx = i2;
+      }
+    }
+  }
+  const unsigned n_cand = __popc(__ballot_sync(0xffffffffu, cand));
+  const bool valid = (unsigned)lane < n_cand;
+  const int n = lane + 1;
+  const float eps = 1.0f - c;
+  bool adm;
+  if (policy == kSelectFactor) {
+    adm = valid && (float)(n + 1) * eps < param;
+  } else {
+    float incl = valid ? eps : 0.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    adm = valid && incl + eps < 1.0f;
+  }
+  const unsigned am = __ballot_sync(0xffffffffu, adm);
+  int n_sel = am ? 32 - __clz(am) : 0;
+  if (n_sel == 0 && n_cand > 0) n_sel = 1;
+  unsigned contrib = (lane < n_sel) ? (1u << idx) : 0u;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) contrib |= __shfl_xor_sync(0xffffffffu, contrib, o);
+  return contrib;
+}
+
 // Host-side launchers (one .cu file each).
 cudaError_t launch_attn_simt(const AttnArgs& a, fdl_dtype dt, int row_tile,
                              cudaStream_t s);
+// beside_prior: launched as a programmatic dependent of the kernel before it
+// (the step's LM head), so its CTAs start beside that kernel's; it reads
+// nothing that kernel writes and, before it completes, waits for it.
 cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
-                           unsigned int* tickets, int n_cta, cudaStream_t s);
+                           unsigned int* tickets, int n_cta, cudaStream_t s,
+                           bool beside_prior = false);
 cudaError_t launch_lmhead_simt(const LmArgs& a, fdl_dtype dt, cudaStream_t s);
-cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s);
+// shared: leave room on every SM for one attention CTA (see lmhead_tc.cu).
+// after_producer: a programmatic dependent of the kernel before it (the
+// token-shift gather that writes its rows), which it waits for only before
+// its first read of the rows.
+cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, bool shared = false,
+                             bool after_producer = false);
+bool lmhead_tc_shared_ok(const LmArgs& a);
 cudaError_t launch_commit(const float* conf, const int32_t* tok,
                           int32_t* block_tokens, uint8_t* committed,
                           int32_t* n_committed, int32_t* n_masked_left, int B,
                           int D, int q_off, int q_len, int mask_id, float tau,
                           cudaStream_t s);
+cudaError_t launch_select_commit(int policy, float param, const float* conf,
+                                 const int32_t* tok, int32_t* block_tokens,
+                                 uint8_t* committed, int32_t* n_committed,
+                                 int32_t* n_masked_left, int B, int D, int q_off,
+                                 int q_len, int mask_id, cudaStream_t s);
+cudaError_t launch_unit_status(const int32_t* n_masked_left, int B, int32_t* any_out,
+                               int32_t* steps, unsigned long long handle, int limit,
+                               cudaStream_t s);
+cudaError_t launch_append_block(const void* k_blk, const void* v_blk, void* k_pre, void* v_pre,
+                                int32_t* len_pre, unsigned int* status, int B, int Hkv, int D,
+                                int cap, int row_bytes, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* src, const void* h_prev, void* rows,
                                int B, int q_len, int H, int shift, int elem,
                                cudaStream_t s);

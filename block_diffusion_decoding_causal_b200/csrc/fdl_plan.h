@@ -12,7 +12,14 @@ namespace fdl {
 constexpr int kAttnRowTile = 16;   // query rows per attention CTA
 constexpr int kPlanCTAs = 148;     // grid sizing unit: one B200's SM count
 constexpr int kLmMaxCTAs = 4 * kPlanCTAs;
-constexpr int kAttnTcCTAs = 2 * kPlanCTAs;  // tensor-core attention: two CTAs per SM
+#ifndef FDL_ATTN_ALONE_CTAS_PER_SM
+#define FDL_ATTN_ALONE_CTAS_PER_SM 2
+#endif
+// tensor-core attention alone on the GPU: two CTAs per SM
+constexpr int kAttnTcCTAs = FDL_ATTN_ALONE_CTAS_PER_SM * kPlanCTAs;
+constexpr int kLmPassRows = 256;   // LM-head rows per pass over the weight
+constexpr long kMaxStepRows = 4096;  // batch * q_len of one step
+constexpr int kMaxAttnRows = 4096;   // block_size / q_len of the attention entry points
 
 struct AttnSplit {
   int split_keys;  // keys per split, multiple of 64
@@ -20,13 +27,16 @@ struct AttnSplit {
 };
 
 struct Plan {
+  bool step_ok;    // within the fused step's limits (LM head, commit sized)
   int R;           // LM-head rows = batch * q_len
+  int lm_pass_rows;  // rows per LM-head pass: whole sequences, at most 256
   int elem;        // bytes per floating element
   int n_row_tiles;
   AttnSplit attn_plain, attn_dual;
   int lm_cta, lm_rows_per_cta;        // CUDA-core LM head (fp32)
   int lm_tc_cta, lm_tc_rows_per_cta;  // tensor-core LM head (bf16): one CTA per SM
   bool attn_tc;     // tensor-core attention (bf16, d 128)
+  size_t off_tc_tickets;  // tensor-core attention: one ticket per (item, tile row)
   size_t off_ctrl, off_tickets, off_part_o, off_part_ml, off_rows, off_lm_part,
       off_attn, off_tc_part_o, off_tc_part_ml, total;
 };
@@ -48,7 +58,11 @@ inline AttnSplit plan_split(long keys_cap, long items) {
   return s;
 }
 
-inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why) {
+// step: the limits of the fused step, LM head and commit entry points
+// (block <= 64, unit <= 32 positions, batch * q_len <= 4096); otherwise the
+// wider limits of the attention entry points (block and query rows up to
+// 4096, beyond 64 / 32 on the tensor-core kernel only).
+inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why, bool step = true) {
   if (c == nullptr) { *why = "cfg is NULL"; return false; }
   if (c->dtype != FDL_F32 && c->dtype != FDL_BF16) { *why = "dtype must be FDL_F32 or FDL_BF16"; return false; }
   if (c->batch < 1) { *why = "batch must be >= 1"; return false; }
@@ -58,8 +72,22 @@ inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why) {
   if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) {
     *why = "head_dim must be 32, 64 or 128"; return false;
   }
-  if (c->block_size < 1 || c->block_size > 64) { *why = "block_size must be in [1, 64]"; return false; }
-  if (c->q_len < 1 || c->q_len > 32) { *why = "q_len must be in [1, 32]"; return false; }
+  const bool step_shape = c->block_size >= 1 && c->block_size <= 64 && c->q_len >= 1 &&
+                          c->q_len <= 32;
+  if (step) {
+    if (c->block_size < 1 || c->block_size > 64) { *why = "block_size must be in [1, 64]"; return false; }
+    if (c->q_len < 1 || c->q_len > 32) { *why = "q_len must be in [1, 32]"; return false; }
+  } else {
+    if (c->block_size < 1 || c->block_size > kMaxAttnRows) {
+      *why = "block_size must be in [1, 4096]"; return false;
+    }
+    if (c->q_len < 1 || c->q_len > kMaxAttnRows) { *why = "q_len must be in [1, 4096]"; return false; }
+    if (!step_shape && !(c->dtype == FDL_BF16 && c->head_dim == 128 && c->batch <= 256 &&
+                         c->n_q_heads / c->n_kv_heads <= 128)) {
+      *why = "block_size > 64 or q_len > 32 needs bf16, head_dim 128, batch <= 256";
+      return false;
+    }
+  }
   if (c->q_off < 0 || c->q_off + c->q_len > c->block_size) {
     *why = "the unit [q_off, q_off+q_len) must lie inside the block"; return false;
   }
@@ -70,9 +98,12 @@ inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why) {
   if (c->shift != 0 && c->shift != 1) { *why = "shift must be 0 or 1"; return false; }
   if (!std::isfinite(c->tau)) { *why = "tau must be finite"; return false; }
   const long R = (long)c->batch * c->q_len;
-  if (R > 256) { *why = "batch * q_len must be <= 256"; return false; }
+  p->step_ok = step_shape && R <= kMaxStepRows;
+  if (step && !p->step_ok) { *why = "batch * q_len must be <= 4096"; return false; }
 
-  p->R = (int)R;
+  p->R = p->step_ok ? (int)R : 0;
+  p->lm_pass_rows = p->step_ok ? (R <= kLmPassRows ? (int)R : kLmPassRows / c->q_len * c->q_len)
+                               : 0;
   p->elem = c->dtype == FDL_BF16 ? 2 : 4;
   const int group = c->n_q_heads / c->n_kv_heads;
   const int rows = c->q_len * group;
@@ -99,26 +130,36 @@ inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why) {
   size_t off = 0;
   p->off_ctrl = off;
   off = align256(off + 256);
+  // CUDA-core attention (fp32, head_dim 32 / 64): step shapes only.
+  const size_t simt_items = step_shape ? (size_t)items : 0;
   p->off_tickets = off;
-  off = align256(off + sizeof(unsigned int) * (size_t)items);
+  off = align256(off + sizeof(unsigned int) * simt_items);
   p->off_part_o = off;
-  off = align256(off + sizeof(float) * (size_t)items * max_split * kAttnRowTile * c->head_dim);
+  off = align256(off + sizeof(float) * simt_items * max_split * kAttnRowTile * c->head_dim);
   p->off_part_ml = off;
-  off = align256(off + 8 * (size_t)items * max_split * kAttnRowTile);
+  off = align256(off + 8 * simt_items * max_split * kAttnRowTile);
+  // LM-head rows, per-CTA partials (one pass) and the attention output of
+  // the fused step: sized only for configurations the step accepts.
   p->off_rows = off;
-  off = align256(off + (size_t)p->elem * R * c->hidden);
+  off = align256(off + (size_t)p->elem * p->R * c->hidden);
   p->off_lm_part = off;
-  off = align256(off + 16 * (size_t)kLmMaxCTAs * R);
+  off = align256(off + 16 * (size_t)kLmMaxCTAs * p->lm_pass_rows);
   p->off_attn = off;
-  off = align256(off + (size_t)p->elem * R * c->n_q_heads * c->head_dim);
+  off = align256(off + (size_t)p->elem * p->R * c->n_q_heads * c->head_dim);
   // Tensor-core attention: at most two partials (first and last item) per CTA.
   p->attn_tc = c->dtype == FDL_BF16 && c->head_dim == 128 && group <= 128 && c->batch <= 256;
   p->off_tc_part_o = off;
   p->off_tc_part_ml = off;
+  p->off_tc_tickets = off;
   if (p->attn_tc) {
     off = align256(off + sizeof(float) * 2 * (size_t)kAttnTcCTAs * 128 * 128);
     p->off_tc_part_ml = off;
     off = align256(off + 8 * 2 * (size_t)kAttnTcCTAs * 128);
+    // 128-row tiles: the GQA group x as many positions as fit.
+    const int qpt = 128 / group < c->q_len ? 128 / group : c->q_len;
+    const long tc_items = (long)c->batch * c->n_kv_heads * ((c->q_len + qpt - 1) / qpt);
+    p->off_tc_tickets = off;
+    off = align256(off + sizeof(unsigned int) * 128 * (size_t)tc_items);
   }
   p->total = off;
   return true;

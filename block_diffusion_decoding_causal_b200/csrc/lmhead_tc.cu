@@ -35,7 +35,7 @@ constexpr int kKChunk = 64;                 // bf16 per 128-byte row
 constexpr int kStageA = kTileM * kKChunk * 2;  // 16 KB
 constexpr int kBoxPart = 16;                // rows per box of a partial tile
 constexpr int kThreads = 192;
-constexpr unsigned kDevTimeout = 4u;        // status bit: a bounded wait expired
+constexpr unsigned kDevTimeout = FDL_DEV_TIMEOUT;
 
 struct TcParams {
   int npad;        // MMA N: 32, 64, 128 or 256
@@ -91,6 +91,10 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   MSI* s_red = reinterpret_cast<MSI*>(tmem_holder + 4);  // [4][NPAD]
 
+  // A kernel queued behind this one with programmatic serialisation (the
+  // attention of the same step, which reads nothing this kernel writes) may
+  // start on the SM room this CTA leaves.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int v0 = blockIdx.x * a.rows_per_cta;
   const int v1 = min(a.V, v0 + a.rows_per_cta);
@@ -131,17 +135,33 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
       tma_prefetch_desc(&tm_x);
       const uint64_t pol_w = policy_evict_first();
       int ia = 0, ib = 0;
+      bool x_ready = false;  // the kernel before this one (the gather) finished
+      auto load_x = [&](int kc) {
+        if (!x_ready) {
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          x_ready = true;
+        }
+        const int slot_b = ib % SB;
+        if (!mbar_wait(&empty_b[slot_b], ((ib / SB) & 1) ^ 1)) { failed = true; return; }
+        mbar_arrive_expect_tx(&full_b[slot_b], SB_BYTES);
+#pragma unroll
+        for (int u = 0; u < KSUB; ++u)
+          tma_load_2d(sb + slot_b * SB_BYTES + u * NPAD * 128, &tm_x,
+                      (kc * KSUB + u) * kKChunk, 0, &full_b[slot_b]);
+        ++ib;
+      };
       for (int g = 0; g < n_groups && !failed; ++g) {
         const int t0 = g * G, t1 = min(n_tiles, t0 + G);
         for (int kc = 0; kc < KC && !failed; ++kc) {
-          const int slot_b = ib % SB;
-          if (!mbar_wait(&empty_b[slot_b], ((ib / SB) & 1) ^ 1)) { failed = true; break; }
-          mbar_arrive_expect_tx(&full_b[slot_b], SB_BYTES);
-#pragma unroll
-          for (int u = 0; u < KSUB; ++u)
-            tma_load_2d(sb + slot_b * SB_BYTES + u * NPAD * 128, &tm_x,
-                        (kc * KSUB + u) * kKChunk, 0, &full_b[slot_b]);
-          ++ib;
+          // The rows may come from the kernel launched just before this one
+          // (the token-shift gather, programmatic launch): the first chunk's
+          // weight tiles stream before waiting for it when they all fit in
+          // the empty ring; later chunks load the rows first.
+          const bool x_after = !x_ready && (t1 - t0) <= SA;
+          if (!x_after) {
+            load_x(kc);
+            if (failed) break;
+          }
           for (int t = t0; t < t1; ++t) {
             const int slot_a = ia % SA;
             if (!mbar_wait(&empty_a[slot_a], ((ia / SA) & 1) ^ 1)) { failed = true; break; }
@@ -165,6 +185,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
             }
             ++ia;
           }
+          if (x_after && !failed) load_x(kc);
         }
       }
       // Drain: every load issued has landed before this CTA can exit.
@@ -303,65 +324,120 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
 
 template <int NCH, int KSUB>
 cudaError_t launch_nch(const CUtensorMap& wf, const CUtensorMap& wp, const CUtensorMap& x,
-                       const LmArgs& a, const TcParams& tp, size_t smem, cudaStream_t s) {
+                       const LmArgs& a, const TcParams& tp, size_t smem, cudaStream_t s,
+                       bool after_producer) {
   auto k = lmhead_tc_kernel<NCH, KSUB>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<a.n_cta, kThreads, smem, s>>>(wf, wp, x, a, tp);
-  return cudaGetLastError();
+  // The whole unified L1/shared array as shared memory, so an SM running one
+  // of these CTAs still has room for an attention CTA of the same step.
+  e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(a.n_cta, 1, 1);
+  lc.blockDim = dim3(kThreads, 1, 1);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = after_producer ? 1 : 0;
+  return cudaLaunchKernelEx(&lc, k, wf, wp, x, a, tp);
 }
 
 }  // namespace
 
 // Tiles per CTA, group size, ring depths and TMEM columns for a call.
-bool lmhead_tc_params(int R, int H, int rows_per_cta, TcParams* tp, size_t* smem);
+//
+// Shared mode: the CTA leaves room on its SM for one attention CTA of the
+// same step in its one-stage form (71 KB shared memory, 256 TMEM columns,
+// 192 threads of 168 registers), so the two kernels stream HBM side by side.
+// Its shared memory stays between 114 and 152 KB: two LM-head CTAs never fit
+// on one SM, one LM-head CTA and one attention CTA always do; TMEM stays
+// within 256 columns and registers within 168 per thread (R <= 64).
+bool lmhead_tc_params(int R, int H, int rows_per_cta, bool shared, TcParams* tp,
+                      size_t* smem);
 
-bool lmhead_tc_params(int R, int H, int rows_per_cta, TcParams* tp, size_t* smem) {
+// Shared-mode ring: K width per stage (boxes of 64), X stages, and the bytes
+// of both rings together.
+#ifndef FDL_LM_SHARED_KSUB
+#define FDL_LM_SHARED_KSUB 2
+#endif
+#ifndef FDL_LM_SHARED_STAGES_B
+#define FDL_LM_SHARED_STAGES_B 2
+#endif
+#ifndef FDL_LM_SHARED_RING_KB
+#define FDL_LM_SHARED_RING_KB 144
+#endif
+
+bool lmhead_tc_params(int R, int H, int rows_per_cta, bool shared, TcParams* tp,
+                      size_t* smem) {
   int nch = 1;
   while (nch * 32 < R) nch *= 2;
-  if (nch > 8) return false;
+  if (nch > (shared ? 2 : 8)) return false;
   tp->npad = nch * 32;
   // K width per stage: up to 4 boxes (512 contiguous bytes of each weight
-  // row), as long as the B stage stays within 16 KB.
+  // row), as long as the B stage stays within 16 KB; 2 boxes when shared.
   const int kchunks = H / kKChunk;
   int kmax = 16384 / (tp->npad * 128);
+  if (shared && kmax > FDL_LM_SHARED_KSUB) kmax = FDL_LM_SHARED_KSUB;
   if (kmax < 1) kmax = 1;
   tp->ksub = 1;
   for (int k = 4; k >= 2; k >>= 1)
     if (k <= kmax && kchunks % k == 0) { tp->ksub = k; break; }
   // Tiles per TMEM buffer: about half a CTA's range, so each X chunk serves
   // several weight tiles and the epilogue of one group hides under the next
-  // group's stream (both buffers together stay within TMEM's 512 columns).
+  // group's stream (both buffers together stay within TMEM's 512 columns, or
+  // 256 when shared, in groups of equal size).
   const int n_tiles = (rows_per_cta + kTileM - 1) / kTileM;
   int G = (n_tiles + 1) / 2;
-  const int gmax = 256 / tp->npad;
-  if (G > gmax) G = gmax;
+  const int gmax = (shared ? 128 : 256) / tp->npad;
+  if (G > gmax) {
+    const int n_groups = (n_tiles + gmax - 1) / gmax;
+    G = (n_tiles + n_groups - 1) / n_groups;
+  }
   if (G < 1) G = 1;
   tp->group = G;
   if (kchunks % tp->ksub != 0) return false;
-  if (tp->group < 1 || 2 * tp->group * tp->npad > 512) return false;  // TMEM has 512 columns
+  const int col_limit = shared ? 256 : 512;
+  if (tp->group < 1 || 2 * tp->group * tp->npad > col_limit) return false;
   uint32_t cols = 32;
   while (cols < (uint32_t)(2 * tp->group * tp->npad)) cols *= 2;
   tp->tmem_cols = cols;
   const size_t a_stage = (size_t)kStageA * tp->ksub;
   const size_t b_stage = (size_t)tp->npad * 128 * tp->ksub;
-  tp->stages_b = b_stage <= 16384 ? 4 : 2;
+  tp->stages_b = shared ? FDL_LM_SHARED_STAGES_B : (b_stage <= 16384 ? 4 : 2);
   const size_t b_bytes = (size_t)tp->stages_b * b_stage;
-  const size_t budget = 200 * 1024;
+  const size_t budget = (shared ? FDL_LM_SHARED_RING_KB : 200) * 1024;
+  if (b_bytes + 2 * a_stage > budget) return false;
   int sa = (int)((budget - b_bytes) / a_stage);
   if (sa > 12) sa = 12;
   if (sa < 2) return false;
   tp->stages_a = sa;
   const size_t bars = 8 * (size_t)(2 * sa + 2 * tp->stages_b + 5) + 16;
   *smem = 1024 + (size_t)sa * a_stage + b_bytes + bars + 4 * (size_t)tp->npad * sizeof(MSI);
+  if (shared) {
+    if (*smem > 152 * 1024) return false;
+    if (*smem < 114 * 1024) *smem = 114 * 1024;
+  }
   return true;
 }
 
-cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s) {
+bool lmhead_tc_shared_ok(const LmArgs& a) {
   TcParams tp;
   size_t smem = 0;
-  if (!lmhead_tc_params(a.R, a.H, a.rows_per_cta, &tp, &smem)) return cudaErrorInvalidValue;
+  return lmhead_tc_params(a.R, a.H, a.rows_per_cta, true, &tp, &smem);
+}
+
+cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, bool shared,
+                             bool after_producer) {
+  TcParams tp;
+  size_t smem = 0;
+  if (!lmhead_tc_params(a.R, a.H, a.rows_per_cta, shared, &tp, &smem))
+    return cudaErrorInvalidValue;
   CUtensorMap wf, wp, x;
   if (!make_map(&wf, a.w, a.H, a.V, kKChunk, kTileM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
       !make_map(&wp, a.w, a.H, a.V, kKChunk, kBoxPart, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
@@ -369,9 +445,9 @@ cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
 #define FDL_LM_CASE(NCH)                                                   \
   case NCH:                                                                \
-    if (tp.ksub == 4) return launch_nch<NCH, 4>(wf, wp, x, a, tp, smem, s); \
-    if (tp.ksub == 2) return launch_nch<NCH, 2>(wf, wp, x, a, tp, smem, s); \
-    return launch_nch<NCH, 1>(wf, wp, x, a, tp, smem, s);
+    if (tp.ksub == 4) return launch_nch<NCH, 4>(wf, wp, x, a, tp, smem, s, after_producer); \
+    if (tp.ksub == 2) return launch_nch<NCH, 2>(wf, wp, x, a, tp, smem, s, after_producer); \
+    return launch_nch<NCH, 1>(wf, wp, x, a, tp, smem, s, after_producer);
   switch (tp.npad / 32) {
     FDL_LM_CASE(1)
     FDL_LM_CASE(2)

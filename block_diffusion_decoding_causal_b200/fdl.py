@@ -19,13 +19,15 @@ LIB_PATH = os.path.join(_HERE, "libfdl.so")
 F32, BF16 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_STATUS = (
     0, -1, -2, -3, -4, -5)
-DEV_BAD_PREFIX_LEN, DEV_BAD_SUFFIX_LEN = 1, 2
+DEV_BAD_PREFIX_LEN, DEV_BAD_SUFFIX_LEN, DEV_TIMEOUT = 1, 2, 4
+SELECT_THRESHOLD, SELECT_FACTOR, SELECT_BUDGET = 0, 1, 2
 
 # Every symbol include/fdl.h declares.
 SYMBOLS = ["fdl_version", "fdl_last_error", "fdl_workspace_size",
            "fdl_reset_workspace", "fdl_block_attn", "fdl_dualcache_attn",
            "fdl_lmhead_confidence", "fdl_threshold_commit", "fdl_denoise_step",
-           "fdl_get_status", "fdl_lmhead_confidence_noalloc"]
+           "fdl_get_status", "fdl_lmhead_confidence_noalloc", "fdl_select_commit",
+           "fdl_unit_status", "fdl_append_block", "fdl_prefixcache_attn"]
 
 
 class StepCfg(ctypes.Structure):
@@ -74,10 +76,17 @@ def lib() -> ctypes.CDLL:
             _P, ctypes.c_size_t, _P]
         L.fdl_get_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
         L.fdl_lmhead_confidence_noalloc.argtypes = [ctypes.POINTER(StepCfg)] + [_P] * 5 + [_P]
+        L.fdl_select_commit.argtypes = [ctypes.POINTER(StepCfg), ctypes.c_int, ctypes.c_float] + [
+            _P] * 6 + [_P]
+        L.fdl_unit_status.argtypes = [ctypes.POINTER(StepCfg), _P, _P, _P, ctypes.c_ulonglong, _P]
+        L.fdl_prefixcache_attn.argtypes = [ctypes.POINTER(StepCfg)] + [_P] * 7 + [
+            _P, ctypes.c_size_t, _P]
+        L.fdl_append_block.argtypes = [ctypes.POINTER(StepCfg)] + [_P] * 5 + [_P, ctypes.c_size_t, _P]
         for name in ["fdl_reset_workspace", "fdl_block_attn", "fdl_dualcache_attn",
                      "fdl_lmhead_confidence", "fdl_threshold_commit",
                      "fdl_denoise_step", "fdl_get_status",
-                     "fdl_lmhead_confidence_noalloc"]:
+                     "fdl_lmhead_confidence_noalloc", "fdl_select_commit",
+                     "fdl_unit_status", "fdl_append_block", "fdl_prefixcache_attn"]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -143,6 +152,12 @@ def dualcache_attn(cfg, q, k_pre, v_pre, len_pre, k_blk, v_blk, k_suf, v_suf,
                                     ws.numel(), stream_ptr(stream)))
 
 
+def prefixcache_attn(cfg, q, k_pre, v_pre, len_pre, k_fresh, v_fresh, out, ws, stream=None):
+    _check(lib().fdl_prefixcache_attn(ctypes.byref(cfg), ptr(q), ptr(k_pre), ptr(v_pre),
+                                      ptr(len_pre), ptr(k_fresh), ptr(v_fresh), ptr(out),
+                                      ptr(ws), ws.numel(), stream_ptr(stream)))
+
+
 def lmhead_confidence(cfg, rows, w_lm, row_active, conf, tok, ws, stream=None):
     _check(lib().fdl_lmhead_confidence(ctypes.byref(cfg), ptr(rows), ptr(w_lm),
                                        ptr(row_active), ptr(conf), ptr(tok), ptr(ws),
@@ -164,6 +179,25 @@ def threshold_commit(cfg, conf, tok, block_tokens, committed, n_committed,
                                       ptr(block_tokens), ptr(committed),
                                       ptr(n_committed), ptr(n_masked_left),
                                       stream_ptr(stream)))
+
+
+def select_commit(cfg, policy, param, conf, tok, block_tokens, committed, n_committed,
+                  n_masked_left, stream=None):
+    _check(lib().fdl_select_commit(ctypes.byref(cfg), int(policy), float(param), ptr(conf),
+                                   ptr(tok), ptr(block_tokens), ptr(committed),
+                                   ptr(n_committed), ptr(n_masked_left), stream_ptr(stream)))
+
+
+def unit_status(cfg, n_masked_left, any_masked=None, step_count=None, while_handle=0,
+                stream=None):
+    _check(lib().fdl_unit_status(ctypes.byref(cfg), ptr(n_masked_left), ptr(any_masked),
+                                 ptr(step_count), int(while_handle), stream_ptr(stream)))
+
+
+def append_block(cfg, k_blk, v_blk, k_pre, v_pre, len_pre, ws, stream=None):
+    _check(lib().fdl_append_block(ctypes.byref(cfg), ptr(k_blk), ptr(v_blk), ptr(k_pre),
+                                  ptr(v_pre), ptr(len_pre), ptr(ws), ws.numel(),
+                                  stream_ptr(stream)))
 
 
 def denoise_step(cfg, q, k_pre, v_pre, len_pre, k_blk, v_blk, k_suf, v_suf, len_suf,

@@ -63,6 +63,10 @@ typedef enum {
 /* Device status bits (fdl_get_status). */
 #define FDL_DEV_BAD_PREFIX_LEN 1u  /* len_pre[b] outside [0, cap_prefix] */
 #define FDL_DEV_BAD_SUFFIX_LEN 2u  /* len_suf[b] outside [0, cap_suffix] */
+#define FDL_DEV_TIMEOUT 4u         /* a kernel's bounded wait (about 1 s) ran out;
+                                      its outputs are invalid and the workspace
+                                      counters may be left non-zero: call
+                                      fdl_reset_workspace before reusing it */
 
 /*
  * Geometry and decoding parameters of one step.
@@ -78,15 +82,22 @@ typedef enum {
  * Lp and Ls are per sequence and live on the device (len_pre / len_suf);
  * cap_prefix / cap_suffix are the cache capacities (rows per (sequence, KV
  * head)).
+ * Limits.  The fused step, the LM head and the commit entry points take
+ * block_size <= 64, q_len <= 32 and batch * q_len <= 4096 (beyond 256 rows
+ * the LM head makes one pass over the weight per group of whole sequences
+ * that fits in 256 rows).  The attention entry points also take block_size
+ * and q_len up to 4096 (PrefixCache: the recomputed rows), on the bf16,
+ * head_dim 128 path with batch <= 256.
  */
 typedef struct {
   int32_t batch;       /* B >= 1                                               */
   int32_t n_q_heads;   /* Hq; Hq % Hkv == 0                                    */
   int32_t n_kv_heads;  /* Hkv; query head h reads KV head h / (Hq / Hkv)       */
   int32_t head_dim;    /* d in {32, 64, 128}; softmax scale 1/sqrt(d)          */
-  int32_t block_size;  /* D, 1..64                                             */
+  int32_t block_size;  /* D, 1..64 (attention entry points: up to 4096)      */
   int32_t q_off;       /* first block position of the active unit             */
-  int32_t q_len;       /* unit length, 1..32, q_off + q_len <= D               */
+  int32_t q_len;       /* unit length, 1..32, q_off + q_len <= D (attention
+                          entry points: up to 4096)                           */
   int32_t cap_prefix;  /* prefix cache rows per (b, kv head), >= 0             */
   int32_t cap_suffix;  /* suffix cache rows per (b, kv head), >= 0 (DualCache) */
   int32_t hidden;      /* H: LM-head input width                               */
@@ -144,6 +155,27 @@ int fdl_dualcache_attn(const fdl_step_cfg* cfg, const void* q,
                        size_t ws_bytes, void* stream);
 
 /*
+ * PrefixCache attention, v1 (technical review section 3 and the PrefixCache
+ * branch of its Algorithm 1): only the prompt and the finished answer prefix
+ * are cached; the active block and the masked suffix after it are
+ * recomputed every step, and their queries attend, with full attention, to
+ * the cached prefix and to their own fresh K/V.
+ *   n = cfg->block_size = cfg->q_len recomputed rows (the active block and
+ *   the suffix), cfg->q_off = 0 (else FDL_ERR_INVALID_ARG).  For sequence b,
+ *   query head h (KV head kvh) and recomputed row r:
+ *     out[b,r,h,:] = softmax(q[b,r,h,:] . K^T / sqrt(d)) V over
+ *     K = k_pre[b,kvh, 0:len_pre[b], :] followed by k_fresh[b,kvh, 0:n, :].
+ * Layouts: q, out [B, n, Hq, d]; k_pre, v_pre [B, Hkv, cap_prefix, d];
+ *   len_pre int32 [B]; k_fresh, v_fresh [B, Hkv, n, d].  n up to 4096 on the
+ *   bf16, head_dim 128 path (the 128-row query tiles are then full).
+ * This is fdl_block_attn with the recomputed rows in the block's place.
+ */
+int fdl_prefixcache_attn(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
+                         const void* v_pre, const int32_t* len_pre, const void* k_fresh,
+                         const void* v_fresh, void* out, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/*
  * LM head + confidence (stage b, first half; "Fast-dLLM v2" Level 2 and
  * Algorithm 2 of the technical review, section 4).
  *   For each row i of rows [B*q_len, H] (already token-shifted: row
@@ -176,6 +208,27 @@ int fdl_threshold_commit(const fdl_step_cfg* cfg, const float* conf,
                          const int32_t* tok, int32_t* block_tokens,
                          uint8_t* committed, int32_t* n_committed,
                          int32_t* n_masked_left, void* stream);
+
+/* Selection rules of fdl_select_commit. */
+#define FDL_SELECT_THRESHOLD 0 /* Algorithm 2: commit conf >= param (tau)    */
+#define FDL_SELECT_FACTOR 1    /* Algorithm 3, eq. 13: factor f = param        */
+#define FDL_SELECT_BUDGET 2    /* eq. 9: heterogeneous error budget (no param) */
+
+/*
+ * Commit with a chosen selection rule (technical review: section 4
+ * Algorithm 2; section 6 eq. (13) and Algorithm 3; section 5.1 eq. (9)).
+ * Candidates as in fdl_threshold_commit.  FDL_SELECT_THRESHOLD is
+ * fdl_threshold_commit with tau = param.  FDL_SELECT_FACTOR sorts the
+ * candidates by decreasing confidence (lower position first on ties) and
+ * commits the first n for the largest n with (n + 1)(1 - c_(n)) < param.
+ * FDL_SELECT_BUDGET commits the first n for the largest n with
+ * sum_{j<=n} (1 - c_(j)) + (1 - c_(n)) < 1.  If no n qualifies, the most
+ * confident candidate alone.  Outputs as fdl_threshold_commit.
+ */
+int fdl_select_commit(const fdl_step_cfg* cfg, int policy, float param,
+                      const float* conf, const int32_t* tok,
+                      int32_t* block_tokens, uint8_t* committed,
+                      int32_t* n_committed, int32_t* n_masked_left, void* stream);
 
 /*
  * One whole denoising step on one stream, no host synchronisation:
@@ -221,6 +274,38 @@ int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
 int fdl_lmhead_confidence_noalloc(const fdl_step_cfg* cfg, const void* rows,
                                   const void* w_lm, const uint8_t* row_active,
                                   float* conf, int32_t* tok, void* stream);
+
+/*
+ * Loop control of the block decode (technical review Algorithm 1: repeat
+ * steps "while the current block contains masks"; "Fast-dLLM v2" Level 2).
+ * Reads n_masked_left [B] (device) after a step and, each only if given:
+ *   any_masked (device int32): 1 if any sequence still has a masked unit
+ *     position, else 0;
+ *   step_count (device int32): incremented by one;
+ *   while_handle: a cudaGraphConditionalHandle (cast to integer, 0 = none)
+ *     of the WHILE node that wraps the step in a CUDA graph; it is set to 1
+ *     while a masked position is left AND the incremented step_count is
+ *     below q_len, so the graph keeps stepping without the host and never
+ *     loops more than q_len times (each step commits at least one position;
+ *     only a committed token equal to mask_id can leave one masked).  A
+ *     non-zero while_handle requires step_count (else FDL_ERR_INVALID_ARG),
+ *     zeroed by the caller before each graph launch.
+ * One tiny kernel; capturable.
+ */
+int fdl_unit_status(const fdl_step_cfg* cfg, const int32_t* n_masked_left,
+                    int32_t* any_masked, int32_t* step_count,
+                    unsigned long long while_handle, void* stream);
+
+/*
+ * Block-level KV cache append ("Fast-dLLM v2" Level 3): after the block is
+ * fully decoded, copy its rows k_blk/v_blk [B, Hkv, D, d] into the prefix
+ * cache k_pre/v_pre [B, Hkv, cap_prefix, d] at rows len_pre[b] .. +D, then
+ * len_pre[b] += D, on the device.  A sequence whose cache would overflow is
+ * left unchanged and flagged (FDL_DEV_BAD_PREFIX_LEN in the workspace).
+ */
+int fdl_append_block(const fdl_step_cfg* cfg, const void* k_blk,
+                     const void* v_blk, void* k_pre, void* v_pre,
+                     int32_t* len_pre, void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, read the workspace status word into *status (bits
  * FDL_DEV_*) and clear it.  Returns FDL_ERR_DEVICE_STATUS if any bit was

@@ -155,6 +155,31 @@ def attention_step(q, k_pre, v_pre, len_pre, prompt_len, k_blk, v_blk, q_off,
     return out
 
 
+def prefixcache_attention(q, k_pre, v_pre, len_pre, k_fresh, v_fresh) -> np.ndarray:
+    """PrefixCache attention of v1 (technical review, section 3 and
+    Algorithm 1, the PrefixCache branch), fp64, [B, n, Hq, d].
+
+    Only the prompt and the finished answer prefix are cached; the active
+    block and the still-masked suffix after it (n positions in all) are
+    recomputed every step.  Their queries attend, with full (bidirectional)
+    attention, to the cached prefix rows [0, len_pre[b]) followed by the n
+    recomputed rows' own fresh K/V.
+    """
+    B, n, Hq, d = q.shape
+    Hkv = k_pre.shape[1]
+    group = Hq // Hkv
+    out = np.empty((B, n, Hq, d), dtype=np.float64)
+    for b in range(B):
+        Lp = int(len_pre[b])
+        vis = np.ones((n, Lp + n), dtype=bool)
+        for h in range(Hq):
+            kvh = h // group
+            K = np.concatenate([k_pre[b, kvh, :Lp], k_fresh[b, kvh]], axis=0)
+            Vv = np.concatenate([v_pre[b, kvh, :Lp], v_fresh[b, kvh]], axis=0)
+            out[b, :, h, :] = masked_attention(q[b, :, h, :], K, Vv, vis)
+    return out
+
+
 # ------------------------------------------------------- LM head + commit
 
 
@@ -230,6 +255,28 @@ def threshold_commit(block_tokens, conf, tok, q_off: int, q_len: int,
     for b in range(B):
         M = [p for p in range(q_off, q_off + q_len) if bt[b, p] == mask_id]
         S = threshold_select(M, lambda p: conf[b, p - q_off], tau)
+        for p in S:
+            new[b, p] = tok[b, p - q_off]
+            committed[b, p] = 1
+        n_comm[b] = len(S)
+        n_left[b] = sum(1 for p in range(q_off, q_off + q_len) if new[b, p] == mask_id)
+    return new, committed, n_comm, n_left
+
+
+def select_commit(block_tokens, conf, tok, q_off: int, q_len: int, mask_id: int,
+                  select):
+    """Commit step with any selection rule ``select(masked, conf_of)`` over
+    the unit's still-masked positions (technical review, Algorithms 2 and 3;
+    eq. 9).  Same outputs as ``threshold_commit``."""
+    bt = np.array(block_tokens, dtype=np.int64)
+    B, D = bt.shape
+    new = bt.copy()
+    committed = np.zeros((B, D), dtype=np.uint8)
+    n_comm = np.zeros(B, dtype=np.int64)
+    n_left = np.zeros(B, dtype=np.int64)
+    for b in range(B):
+        M = [p for p in range(q_off, q_off + q_len) if bt[b, p] == mask_id]
+        S = select(M, lambda p: conf[b, p - q_off]) if M else []
         for p in S:
             new[b, p] = tok[b, p - q_off]
             committed[b, p] = 1

@@ -95,6 +95,21 @@ def factor_select(masked_positions, conf_of, f: float):
     return order[:best]
 
 
+def budget_select(masked_positions, conf_of):
+    """Selection by the heterogeneous error budget of eq. (9): sort the masked
+    positions by decreasing confidence (ties: lower position first), with
+    eps_j = 1 - c_j; keep the largest n whose first n positions satisfy
+    sum eps + max eps < 1; if no n qualifies, the first position alone."""
+    order = sorted(masked_positions, key=lambda p: (-conf_of(p), p))
+    best = 0
+    for n in range(1, len(order) + 1):
+        if heterogeneous_budget_ok([1.0 - conf_of(q) for q in order[:n]]):
+            best = n
+    if best == 0:
+        return order[:1]
+    return order[:best]
+
+
 def all_assignments(n: int, k: int):
     """Every string of length n over an alphabet of size k."""
     return itertools.product(range(k), repeat=n)

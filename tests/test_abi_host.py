@@ -38,6 +38,28 @@ def test_library_exports_every_declared_symbol(L):
     assert set(fdl.SYMBOLS) <= declared
 
 
+def _declared_arity():
+    """Parameter count of every fdl_* function include/*.h declares."""
+    out = {}
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            for name, params in re.findall(r"\b(fdl_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", src):
+                params = params.strip()
+                out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header(L):
+    arity = _declared_arity()
+    assert set(fdl.SYMBOLS) <= set(arity)
+    for name in fdl.SYMBOLS:
+        fn = getattr(L, name)
+        if fn.argtypes is not None:
+            assert len(fn.argtypes) == arity[name], name
+
+
 def test_version(L):
     assert L.fdl_version() == 1
 
@@ -58,7 +80,7 @@ def _cfg(**kw):
     (dict(shift=2), "shift"),
     (dict(tau=float("nan")), "tau"),
     (dict(hidden=100), "hidden"),
-    (dict(batch=33), "256"),
+    (dict(block_size=5000), "block_size"),
     (dict(dtype=""), "dtype"),
 ])
 def test_invalid_configs_are_rejected(L, bad, msg):
@@ -139,3 +161,48 @@ def test_last_error_is_cleared_by_success(L):
     assert fdl.last_error() != ""
     assert L.fdl_workspace_size(ctypes.byref(_cfg())) > 0
     assert fdl.last_error() == ""
+
+
+def test_loop_control_and_append_reject_bad_arguments(L):
+    cfg = _cfg()
+    nl = ctypes.c_void_p(16)        # never dereferenced: rejected before any launch
+    rc = L.fdl_unit_status(ctypes.byref(cfg), None, None, None, 0, None)
+    assert rc == fdl.ERR_INVALID_ARG and "n_masked_left" in fdl.last_error()
+    rc = L.fdl_unit_status(ctypes.byref(cfg), nl, None, None, 12345, None)
+    assert rc == fdl.ERR_INVALID_ARG and "step_count" in fdl.last_error()
+    rc = L.fdl_append_block(ctypes.byref(cfg), None, nl, nl, nl, nl, nl, 1 << 30, None)
+    assert rc == fdl.ERR_INVALID_ARG
+    small = _cfg(cap_prefix=16)
+    rc = L.fdl_append_block(ctypes.byref(small), nl, nl, nl, nl, nl, nl, 1 << 30, None)
+    assert rc == fdl.ERR_INVALID_ARG and "cap_prefix" in fdl.last_error()
+    rc = L.fdl_select_commit(ctypes.byref(cfg), 7, 1.0, nl, nl, nl, nl, nl, nl, None)
+    assert rc == fdl.ERR_INVALID_ARG
+
+
+def test_prefixcache_needs_every_recomputed_row_as_a_query(L):
+    c = dict(synth.CONFIGS["llada"], block_size=288, q_len=280, q_off=8, cap_suffix=0)
+    cfg = fdl.make_cfg(c)
+    rc = L.fdl_prefixcache_attn(ctypes.byref(cfg), *([None] * 7), None, 0, None)
+    assert rc == fdl.ERR_INVALID_ARG and "q_off = 0" in fdl.last_error()
+
+
+def test_wide_attention_shapes_only_on_the_tensor_core_path(L):
+    big = dict(synth.CONFIGS["llada"], block_size=768, q_len=768, q_off=0, cap_suffix=0)
+    assert L.fdl_workspace_size(ctypes.byref(fdl.make_cfg(big))) > 0
+    assert L.fdl_workspace_size(ctypes.byref(fdl.make_cfg(dict(big, dtype="f32")))) == 0
+    assert "bf16" in fdl.last_error()
+    assert L.fdl_workspace_size(ctypes.byref(fdl.make_cfg(dict(big, head_dim=64)))) == 0
+    # the fused step keeps its own limits
+    nl = ctypes.c_void_p(16)
+    rc = L.fdl_threshold_commit(ctypes.byref(fdl.make_cfg(big)), nl, nl, nl, nl, nl, nl, None)
+    assert rc == fdl.ERR_INVALID_ARG and "block_size" in fdl.last_error()
+
+
+def test_step_rows_beyond_one_lm_pass_are_accepted_up_to_4096(L):
+    ok = _cfg(batch=512, q_len=8, q_off=0)
+    assert L.fdl_workspace_size(ctypes.byref(ok)) > 0
+    too_many = _cfg(batch=513, q_len=8, q_off=0)
+    assert L.fdl_workspace_size(ctypes.byref(too_many)) > 0      # attention-level only
+    nl = ctypes.c_void_p(16)
+    rc = L.fdl_threshold_commit(ctypes.byref(too_many), nl, nl, nl, nl, nl, nl, None)
+    assert rc == fdl.ERR_INVALID_ARG and "4096" in fdl.last_error()

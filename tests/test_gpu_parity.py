@@ -235,9 +235,14 @@ EDGE = dict(batch=1, n_q_heads=1, n_kv_heads=1, head_dim=128, block_size=32,
     dict(batch=2, n_q_heads=6, n_kv_heads=3, q_len=3, prefix=(60, 70), cap_prefix=80,
          suffix=130, cap_suffix=130),                          # DualCache, short
 ])
-def test_attention_split_extremes(over):
+@pytest.mark.parametrize("path", ["entry", "step"])
+def test_attention_split_extremes(over, path):
     """Stream-K partition edges: fewer chunks than CTAs, one item spread over
-    most CTAs, row tiles of 128 (group 32 x 4 positions), DualCache."""
+    most CTAs, row tiles of 128 (group 32 x 4 positions), DualCache.  "entry":
+    the attention entry points (two CTAs per SM, merge kernel); "step": the
+    fused step, where the attention runs beside the LM head (one CTA per SM,
+    partials merged inside the kernel); only its attention output is checked
+    here."""
     cfg = dict(EDGE, **over)
     case = synth.make_case("edge", 3, cfg=cfg)
     c = fdl.make_cfg(case.cfg)
@@ -245,6 +250,13 @@ def test_attention_split_extremes(over):
     out = torch.empty_like(d["q"])
     ws = fdl.workspace(c)
     for _ in range(2):
+        if path == "step":
+            gh.run_denoise_step(case, ws=ws, d=d)
+            res = gh.run_denoise_step(case, ws=ws, d=d)
+            ref = cases.run_oracle(case)
+            gh.assert_close_scaled(res["attn"].double().numpy(), ref["attn"], 2e-2, "attn")
+            assert res["status"] == 0
+            continue
         if case.k_suf is None:
             fdl.block_attn(c, d["q"], d["k_pre"], d["v_pre"], d["len_pre"], d["k_blk"],
                            d["v_blk"], out, ws)
@@ -254,3 +266,136 @@ def test_attention_split_extremes(over):
         ref = cases.run_oracle(case)
         gh.assert_close_scaled(out.double().cpu().numpy(), ref["attn"], 2e-2, "attn")
     assert fdl.get_status(ws) == 0
+
+
+# ------------------------------------------- factor / budget selection
+
+def _ranked_margin_ok(conf_row, masked, policy, f):
+    cs = sorted((float(conf_row[i]) for i in masked), reverse=True)
+    run = 0.0
+    for n, c in enumerate(cs, start=1):
+        e = 1.0 - c
+        run += e
+        v = (n + 1) * e - f if policy == fdl.SELECT_FACTOR else run + e - 1.0
+        if abs(v) < 1e-4:
+            return False
+    return True
+
+
+@pytest.mark.parametrize("policy,f", [(1, 1.0), (1, 0.5), (1, 2.5), (2, 0.0)])
+def test_select_commit_factor_and_budget(policy, f):
+    """Algorithm 3 / eq. 13 and eq. 9 against the oracle on random units
+    (decisions kept 1e-4 away from their boundaries), including an exact
+    confidence tie and units with nothing or one thing masked."""
+    rng = np.random.default_rng(policy * 10 + int(f * 10))
+    B, D, q_off, q_len, mask = 16, 32, 8, 16, 77
+    conf = np.zeros((B, q_len), dtype=np.float32)
+    bt = np.zeros((B, D), dtype=np.int32)
+    for b in range(B):
+        while True:
+            row = rng.uniform(0.3, 1.0, q_len).astype(np.float32) ** rng.uniform(0.2, 3)
+            row = row.astype(np.float32)
+            if b == 0:
+                row[1] = row[5]                      # exact tie
+            masked = np.flatnonzero(rng.random(q_len) < rng.uniform(0, 1))
+            if b == 1:
+                masked = np.array([], dtype=int)
+            if b == 2:
+                masked = np.array([3])
+            if _ranked_margin_ok(row, masked, policy, f):
+                break
+        conf[b] = row
+        bt[b] = rng.integers(0, 70, D)
+        bt[b, q_off + masked] = mask
+    tok = rng.integers(100, 200, (B, q_len)).astype(np.int32)
+    cfg = fdl.make_cfg(dict(batch=B, n_q_heads=1, n_kv_heads=1, head_dim=32,
+                            block_size=D, q_off=q_off, q_len=q_len, cap_prefix=0,
+                            hidden=8, vocab=1000, mask_id=mask, shift=0, tau=0.9, dtype="f32"))
+    d_bt = torch.from_numpy(bt).cuda()
+    comm = torch.empty((B, D), dtype=torch.uint8, device="cuda")
+    n_c = torch.empty(B, dtype=torch.int32, device="cuda")
+    n_l = torch.empty(B, dtype=torch.int32, device="cuda")
+    fdl.select_commit(cfg, policy, f, torch.from_numpy(conf).cuda(), torch.from_numpy(tok).cuda(),
+                      d_bt, comm, n_c, n_l)
+    from oracle import theory
+    sel = ((lambda M, c: theory.factor_select(M, c, f)) if policy == fdl.SELECT_FACTOR
+           else theory.budget_select)
+    want = step.select_commit(bt, conf.astype(np.float64), tok, q_off, q_len, mask, sel)
+    assert np.array_equal(d_bt.cpu().numpy(), want[0])
+    assert np.array_equal(comm.cpu().numpy(), want[1])
+    assert np.array_equal(n_c.cpu().numpy(), want[2])
+    assert np.array_equal(n_l.cpu().numpy(), want[3])
+    assert want[2][1] == 0 and want[2][2] == 1
+
+
+# ------------------------------------------------ PrefixCache (queries = block + suffix)
+
+@pytest.mark.parametrize("B,Hq,Hkv,n,lens", [
+    (1, 32, 32, 288, [768]),          # LLaDA-like: block 32 + suffix 256 recomputed
+    (2, 28, 4, 100, [0, 1500]),       # GQA 7, ragged: empty prefix, 100 rows (2 chunks)
+    (3, 8, 8, 200, [64, 65, 300]),    # MHA, prefixes on and off the 64-key chunk grid
+])
+def test_prefixcache_attn_against_oracle(B, Hq, Hkv, n, lens):
+    """PrefixCache attention: the recomputed rows (several 64-key chunks and
+    several 128-row query tiles) over [prefix | their own fresh K/V]."""
+    d = 128
+    cap = max(max(lens), 1)
+    g = torch.Generator().manual_seed(B * 100 + n)
+    rn = lambda *s: torch.randn(s, generator=g).to(torch.bfloat16)
+    q, kp, vp, kn, vn = rn(B, n, Hq, d), rn(B, Hkv, cap, d), rn(B, Hkv, cap, d), \
+        rn(B, Hkv, n, d), rn(B, Hkv, n, d)
+    len_pre = torch.tensor(lens, dtype=torch.int32)
+    cfg = fdl.make_cfg(dict(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, block_size=n,
+                            q_off=0, q_len=n, cap_prefix=cap, hidden=128, vocab=1000,
+                            mask_id=999, shift=0, tau=0.9, dtype="bf16"))
+    ws = fdl.workspace(cfg)
+    out = torch.empty((B, n, Hq, d), dtype=torch.bfloat16, device="cuda")
+    dv = [t.cuda() for t in (q, kp, vp, len_pre, kn, vn)]
+    f64 = lambda t: t.double().numpy()
+    ref = step.prefixcache_attention(f64(q), f64(kp), f64(vp), lens, f64(kn), f64(vn))
+    for _ in range(2):                        # the second call reuses the workspace
+        fdl.prefixcache_attn(cfg, *dv, out, ws)
+        torch.cuda.synchronize()
+        gh.assert_close_scaled(out.double().cpu().numpy(), ref, 2e-2, "prefixcache attn")
+    assert fdl.get_status(ws) == 0
+
+
+# ---------------------------------------- more LM-head rows than one pass holds
+
+def test_lmhead_more_rows_than_one_pass():
+    """batch * q_len = 600 rows: passes of 256, 256 and 88 rows over the
+    weight, against the oracle (tokens where the top-2 gap exceeds 1e-3)."""
+    B, q_len, V, H = 75, 8, 20000, 256
+    g = torch.Generator().manual_seed(600)
+    rows = torch.randn((B * q_len, H), generator=g).to(torch.bfloat16)
+    w = (torch.randn((V, H), generator=g) * (8.0 / H ** 0.5)).to(torch.bfloat16)
+    active = (torch.rand(B * q_len, generator=g) < 0.8).to(torch.uint8)
+    cfg = fdl.make_cfg(dict(batch=B, n_q_heads=1, n_kv_heads=1, head_dim=32, block_size=q_len,
+                            q_off=0, q_len=q_len, cap_prefix=0, hidden=H, vocab=V,
+                            mask_id=V - 1, shift=0, tau=0.9, dtype="bf16"))
+    conf = torch.empty(B * q_len, dtype=torch.float32, device="cuda")
+    tok = torch.empty(B * q_len, dtype=torch.int32, device="cuda")
+    ws = fdl.workspace(cfg)
+    fdl.lmhead_confidence(cfg, rows.cuda(), w.cuda(), active.cuda(), conf, tok, ws)
+    torch.cuda.synchronize()
+    t_ref, c_ref, gap = step.lmhead_confidence(rows.double().numpy(), w.float().numpy())
+    act = active.numpy().astype(bool)
+    t_gpu, c_gpu = tok.cpu().numpy(), conf.cpu().numpy().astype(np.float64)
+    sure = (gap > 1e-3) & act
+    assert np.array_equal(t_gpu[sure], t_ref[sure])
+    np.testing.assert_allclose(c_gpu[act], c_ref[act], rtol=1e-3)
+    assert (c_gpu[~act] == -1).all() and (t_gpu[~act] == -1).all()
+    assert fdl.get_status(ws) == 0
+
+
+LARGE_BATCH = dict(batch=40, n_q_heads=8, n_kv_heads=2, head_dim=128, block_size=32,
+                   q_len=8, q_off=None, prefix=(100, 400), cap_prefix=400, suffix=0,
+                   cap_suffix=0, hidden=256, vocab=5000, mask_id=4999, shift=1, tau=0.8,
+                   w_scale=8.0, dtype="bf16", masked=(1, 8))
+
+
+def test_fused_step_with_two_lm_passes():
+    """A fused step with 320 LM-head rows (passes of 256 and 64 rows, each
+    committing its own sequences) against the oracle, bit-exact commits."""
+    case, ref, _ = cases.parity_case("large_batch", 0, cfg=LARGE_BATCH)
+    gh.compare_step(case, gh.run_denoise_step(case), ref)

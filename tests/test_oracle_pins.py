@@ -67,6 +67,43 @@ def test_attention_zero_query_averages_visible_values():
     np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-14)
 
 
+def _prefixcache_inputs(B=2, Hq=6, Hkv=2, d=16, cap=40, n=20, D=8):
+    q = RNG.standard_normal((B, n, Hq, d))
+    k_pre, v_pre = RNG.standard_normal((2, B, Hkv, cap, d))
+    k_new, v_new = RNG.standard_normal((2, B, Hkv, n, d))
+    lens = np.array([cap - 7, 0][:B])
+    return q, k_pre, v_pre, lens, k_new, v_new, D
+
+
+def test_prefixcache_attention_matches_torch_sdpa_with_gqa():
+    """Full attention of every recomputed row over [prefix | fresh rows]
+    against SDPA with the KV heads repeated for their query groups."""
+    q, k_pre, v_pre, lens, k_new, v_new, _ = _prefixcache_inputs()
+    got = step.prefixcache_attention(q, k_pre, v_pre, lens, k_new, v_new)
+    group = q.shape[2] // k_pre.shape[1]
+    for b in range(q.shape[0]):
+        K = np.concatenate([k_pre[b, :, :lens[b]], k_new[b]], axis=1).repeat(group, axis=0)
+        V = np.concatenate([v_pre[b, :, :lens[b]], v_new[b]], axis=1).repeat(group, axis=0)
+        want = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[b].transpose(1, 0, 2)), torch.from_numpy(K),
+            torch.from_numpy(V)).numpy().transpose(1, 0, 2)
+        np.testing.assert_allclose(got[b], want, rtol=1e-12, atol=1e-13)
+
+
+def test_prefixcache_block_rows_equal_dualcache_with_the_same_suffix():
+    """When the suffix cache holds exactly the K/V that PrefixCache
+    recomputes, the active block's rows see the same keys under both schemes
+    (technical review, section 3: the two differ only in what is refreshed)."""
+    q, k_pre, v_pre, lens, k_new, v_new, D = _prefixcache_inputs()
+    pc = step.prefixcache_attention(q, k_pre, v_pre, lens, k_new, v_new)
+    q_off, q_len = 2, 4
+    dc = step.attention_step(q[:, q_off:q_off + q_len], k_pre, v_pre, lens, lens,
+                             k_new[:, :, :D], v_new[:, :, :D], q_off,
+                             k_suf=k_new[:, :, D:], v_suf=v_new[:, :, D:],
+                             len_suf=np.full(q.shape[0], q.shape[1] - D))
+    np.testing.assert_allclose(pc[:, q_off:q_off + q_len], dc, rtol=1e-13, atol=1e-14)
+
+
 # ------------------------------------------------------------------ masks
 
 def test_training_mask_truth_table(golden_dir):
@@ -408,3 +445,30 @@ def test_teaching_roofline_constants(golden_dir):
     # 2 * 7e9 / 989e12 s = 0.0141557 ms; the page prints it cut to 0.01415
     assert per_pos_ms == pytest.approx(g["ms_per_position"], abs=1e-5)
     assert floor_ms / per_pos_ms == pytest.approx(g["crossover_positions"], abs=1.0)
+
+
+def test_budget_rule_eq9_selection():
+    # eps sorted: 0.01, 0.02, 0.05, 0.3 -> n=1: .01+.01; n=2: .03+.02; n=3: .08+.05;
+    # n=4: .38+.3 = .68 < 1 -> all four admissible
+    c = {0: 0.95, 1: 0.99, 2: 0.7, 3: 0.98}.__getitem__
+    assert theory.budget_select([0, 1, 2, 3], c) == [1, 3, 0, 2]
+    c2 = {0: 0.6, 1: 0.99, 2: 0.55}.__getitem__
+    # n=2: eps .01+.4 = .41 + max .4 = .81 < 1; n=3: .86 + .45 = 1.31
+    assert theory.budget_select([0, 1, 2], c2) == [1, 0]
+    c3 = {0: 0.4, 1: 0.3}.__getitem__
+    assert theory.budget_select([0, 1], c3) == [0]       # 0.6 + 0.6 >= 1: first alone
+    # the certificate it uses implies agreement (eq. 8 generalised), by brute force
+    assert theory.heterogeneous_budget_ok([0.01, 0.02, 0.05, 0.3])
+
+
+def test_select_commit_matches_threshold_commit_for_algorithm_2():
+    rng = np.random.default_rng(3)
+    for _ in range(50):
+        conf = rng.uniform(0, 1, (3, 8))
+        tok = rng.integers(0, 100, (3, 8))
+        bt = np.where(rng.random((3, 16)) < 0.5, 99, rng.integers(0, 99, (3, 16)))
+        a = step.threshold_commit(bt, conf, tok, 4, 8, 99, 0.7)
+        b = step.select_commit(bt, conf, tok, 4, 8, 99,
+                               lambda M, cf: step.threshold_select(M, cf, 0.7))
+        for x, y in zip(a, b):
+            assert np.array_equal(x, y)
