@@ -315,6 +315,10 @@ def main():
         attn(i)
     t_attn = max_over_ranks(timed(attn, args.steps), world) / args.steps
     pc = prefixcache_leg(torch, fdl, stream, timed, world, args.steps, peaks)
+    try:
+        blk = block_decode_leg(torch, fdl, c, sets[0], w, stream, world)
+    except Exception as e:  # reported in the JSON line; the headline legs stand
+        blk = {"error": f"{type(e).__name__}: {e}"}
     lm_big = large_batch_lm_leg(torch, fdl, synth, stream, timed, world, args.steps, peaks)
 
     # End to end through the public API: per step, pinned host inputs copied
@@ -385,6 +389,7 @@ def main():
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": step_bytes / (t_step / args.steps) / 1e9,
                           "frac": step_bytes / (t_step / args.steps) / 1e9 / peaks["hbm_gbs"]},
         "prefixcache": pc,
+        "block_decode": blk,
         "lmhead_large_batch": lm_big,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e / args.steps * 1e3},
@@ -399,6 +404,89 @@ def main():
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def block_decode_leg(torch, fdl, c, x, w, stream, world, blocks: int = 5) -> dict:
+    """One whole block (4 sub-blocks of 8) decoded by repeated fused steps
+    until no position is masked, then appended to the prefix cache: as one
+    CUDA graph with a device-side WHILE loop per sub-block, and driven from
+    the host (one synchronisation per step).  The step inputs stay fixed
+    (no model between steps), so the confidences repeat and each sub-block
+    takes 1 + (positions left below tau) steps."""
+    from block_diffusion_decoding_causal_b200 import driver
+    B, D, q_len = c["batch"], c["block_size"], c["q_len"]
+    units = D // q_len
+    cap = x["k_pre"].shape[2] + 2 * D
+    cfgs = [fdl.make_cfg(dict(c, q_off=u * q_len, cap_prefix=cap)) for u in range(units)]
+    Hkv, d = c["n_kv_heads"], c["head_dim"]
+    with torch.cuda.stream(stream):
+        k_pre = torch.zeros((B, Hkv, cap, d), dtype=torch.bfloat16, device="cuda")
+        v_pre = torch.zeros_like(k_pre)
+        cap0 = x["k_pre"].shape[2]
+        k_pre[:, :, :cap0].copy_(x["k_pre"])
+        v_pre[:, :, :cap0].copy_(x["v_pre"])
+        len0 = x["len_pre"].clone()
+        lens = len0.clone()
+        bt0 = torch.full((B, D), c["mask_id"], dtype=torch.int32, device="cuda")
+        bt = bt0.clone()
+        o = dict(attn=torch.empty_like(x["q"]),
+                 conf=torch.empty((B, q_len), dtype=torch.float32, device="cuda"),
+                 tok=torch.empty((B, q_len), dtype=torch.int32, device="cuda"),
+                 comm=torch.empty((B, D), dtype=torch.uint8, device="cuda"),
+                 n_c=torch.empty(B, dtype=torch.int32, device="cuda"),
+                 n_l=torch.empty(B, dtype=torch.int32, device="cuda"),
+                 any=torch.zeros(1, dtype=torch.int32, device="cuda"),
+                 steps=torch.zeros(units, dtype=torch.int32, device="cuda"))
+        ws = fdl.workspace(cfgs[0])
+    stream.synchronize()
+
+    def step(u, s):
+        fdl.denoise_step(cfgs[u], x["q"], k_pre, v_pre, lens, x["k_blk"], x["v_blk"], None, None,
+                         None, x["hidden"], x["h_prev"], w, bt, o["attn"], o["conf"], o["tok"],
+                         o["comm"], o["n_c"], o["n_l"], ws, stream=s)
+
+    def append(s):
+        fdl.append_block(cfgs[0], x["k_blk"], x["v_blk"], k_pre, v_pre, lens, ws, stream=s)
+
+    def reset():
+        with torch.cuda.stream(stream):
+            bt.copy_(bt0)
+            lens.copy_(len0)
+            o["steps"].zero_()
+
+    g = driver.BlockGraph(cfgs, step, o["n_l"], o["steps"], append=append)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for _ in range(2):
+        reset()
+        g.launch(stream)
+    stream.synchronize()
+    ev[0].record(stream)
+    for _ in range(blocks):
+        reset()
+        g.launch(stream)
+    ev[1].record(stream)
+    stream.synchronize()
+    steps_graph = o["steps"].cpu().tolist()
+    ok = bool((bt != c["mask_id"]).all())
+    ev[2].record(stream)
+    steps_host = []
+    for _ in range(blocks):
+        reset()
+        steps_host = []
+        driver.run_host_loop(cfgs, step, o["n_l"], o["any"], steps_host, stream=stream)
+        append(stream)
+    ev[3].record(stream)
+    stream.synchronize()
+    t_graph = max_over_ranks(ev[0].elapsed_time(ev[1]) / blocks, world)
+    t_host = max_over_ranks(ev[2].elapsed_time(ev[3]) / blocks, world)
+    n_steps = sum(steps_graph)
+    assert fdl.get_status(ws, stream) == 0
+    return {"workload": f"one block of {D} positions, {units} sub-blocks of {q_len}, batch {B}",
+            "steps_per_block": n_steps, "steps_per_sub_block": steps_graph,
+            "host_loop_steps": steps_host, "block_decoded": ok,
+            "graph_us_per_block": t_graph * 1e3, "host_loop_us_per_block": t_host * 1e3,
+            "graph_us_per_step": t_graph * 1e3 / max(n_steps, 1),
+            "positions_per_s_graph": B * D / (t_graph * 1e-3)}
 
 
 PREFIXCACHE = dict(batch=1, n_q_heads=32, n_kv_heads=32, head_dim=128, prefix=768, rows=768)

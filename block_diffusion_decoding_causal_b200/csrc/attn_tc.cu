@@ -41,7 +41,11 @@ using namespace sm100;
 
 constexpr int kCh = 64;                  // keys per chunk
 constexpr int kQRegion = 128 * 128;      // 128 rows x 64 bf16 (16 KB)
-constexpr int kQBuf = 2 * kQRegion;      // d 0-63 and 64-127
+// Rows of an item at most 64: the Q halves (d 0-63, 64-127) sit 8 KB apart
+// and the buffer is 16 KB.  The MMA still reads 128 rows per half; rows 64+
+// then fall on the other half or the K/V stage that follows, which only
+// feeds S rows no softmax thread reads (rows of an item never mix).
+constexpr int kQRegionCompact = 64 * 128;
 constexpr int kKVRegion = kCh * 128;     // 64 keys x 64 bf16 (8 KB)
 constexpr int kKVSlot = 4 * kKVRegion;   // K lo, K hi, V lo, V hi: one 32 KB stage
 // K/V stages of the attention alone on the GPU (two CTAs per SM at 2) and
@@ -71,6 +75,7 @@ struct TcArgs {
   float* part_o;          // [2 * n_cta][128][128]
   float2* part_ml;        // [2 * n_cta][128]
   int inline_merge;       // the last CTA to finish a row of an item merges it
+  int q_region;           // bytes between the two d-halves of the Q buffer
 };
 
 struct Maps {
@@ -243,8 +248,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_smem = base;                          // kQBufs x 32 KB
-  uint8_t* kv_smem = q_smem + kQBufs * kQBuf;      // STAGES x 32 KB
+  uint8_t* q_smem = base;                               // kQBufs x 2 x q_region
+  uint8_t* kv_smem = q_smem + kQBufs * 2 * a.q_region;  // STAGES x 32 KB
   Smem& S = *reinterpret_cast<Smem*>(kv_smem + STAGES * kKVSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -308,12 +313,13 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
     }
     if (lane == 0) S.cb[a.B] = run;
   }
-  // Padding rows of both Q buffers are never written by TMA: zero them once.
-  for (int t = threadIdx.x; t < kQBufs * 2 * (128 - rows_full) * 8; t += kThreads) {
-    const int per_region = (128 - rows_full) * 8;
+  // Padding rows of the Q halves are never written by TMA: zero them once.
+  const int q_rows = a.q_region / 128;
+  for (int t = threadIdx.x; t < kQBufs * 2 * (q_rows - rows_full) * 8; t += kThreads) {
+    const int per_region = (q_rows - rows_full) * 8;
     const int region = t / per_region, w = t % per_region;
     const int row = rows_full + w / 8, chunk = w % 8;
-    *reinterpret_cast<uint4*>(q_smem + region * kQRegion + row * 128 + chunk * 16) =
+    *reinterpret_cast<uint4*>(q_smem + region * a.q_region + row * 128 + chunk * 16) =
         make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async_smem();
@@ -361,8 +367,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
           if (!mbar_wait(&S.q_empty[qb], ((q_i / kQBufs) & 1) ^ 1)) { failed = true; break; }
           mbar_arrive_expect_tx(&S.q_full[qb], 2u * 128u * (uint32_t)rows_full);
           const int z = c.b * a.q_len + rt * a.qpt;
-          tma_load_3d(q_smem + qb * kQBuf, &maps.q, 0, kvh * a.group, z, &S.q_full[qb]);
-          tma_load_3d(q_smem + qb * kQBuf + kQRegion, &maps.q, 64, kvh * a.group, z,
+          tma_load_3d(q_smem + qb * 2 * a.q_region, &maps.q, 0, kvh * a.group, z,
+                      &S.q_full[qb]);
+          tma_load_3d(q_smem + qb * 2 * a.q_region + a.q_region, &maps.q, 64, kvh * a.group, z,
                       &S.q_full[qb]);
           ++q_i;
           prev_x = x;
@@ -403,12 +410,12 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
             const int qb = (q_s - 1) % kQBufs;
             const bool last = (is + 1 == n_my) || (cs.j + 1 == S.nc[cs.b]);
             tc_fence_after();
-            const uint32_t q_base = smem_u32(q_smem + qb * kQBuf);
+            const uint32_t q_base = smem_u32(q_smem + qb * 2 * a.q_region);
             const uint32_t k_base = smem_u32(kv_smem + slot * kKVSlot);
             const uint32_t d_s = tmem + (uint32_t)sb * kCh;
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              mma_bf16(d_s, desc_k_sw128(q_base + (k >> 2) * kQRegion + (k & 3) * 32),
+              mma_bf16(d_s, desc_k_sw128(q_base + (k >> 2) * a.q_region + (k & 3) * 32),
                        desc_k_sw128(k_base + (k >> 2) * kKVRegion + (k & 3) * 32), id_s,
                        k ? 1u : 0u);
             mma_commit(&S.s_full[sb]);
@@ -648,26 +655,28 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
 }
 
 // Merge of the partials of every item the split spread over several CTAs.
-// A warp per (item, tile row); its lanes are PG partial groups x (32 / PG)
-// column groups, so the partials are read in parallel (PG ~ the expected
-// number of partials per item) and combined with the usual (max, sum)
-// rescaling, then reduced across the partial groups by shuffles.  A CTA
-// holds 8 rows of one item.  Launched as a programmatic dependent of the
-// attention grid: scheduled as its CTAs retire, it waits for the whole grid
-// before reading anything.
-template <int PG>
+// A CTA holds 8 / WPR rows of one item, WPR warps per row (WPR follows the
+// expected number of partials per item): warp w of a row combines partials
+// cta_lo + w, + WPR, ... with the usual (max, sum) rescaling, each lane
+// holding four of the 128 columns (one coalesced 512-byte read per partial
+// and warp); the row's warps then combine through shared memory.  Launched
+// as a programmatic dependent of the attention grid: scheduled as its CTAs
+// retire, it waits for the whole grid before reading anything.
+template <int WPR>
 __global__ void __launch_bounds__(256)
 attn_merge_kernel(const TcArgs a) {
-  constexpr int CGL = 32 / PG;      // column groups per warp
-  constexpr int COLS = 128 / CGL;   // columns per lane
+  constexpr int RPC = 8 / WPR;  // rows per CTA
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ float s_m[RPC][WPR], s_l[RPC][WPR];
+  __shared__ float4 s_acc[RPC][WPR][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = warp / WPR, wq = warp % WPR;
   const int per_seq = a.Hkv * a.n_rt;
-  const int x = blockIdx.x, r = blockIdx.y * 8 + warp;
+  const int x = blockIdx.x, r = blockIdx.y * RPC + half;
   const int b = x / per_seq, it = x % per_seq;
   const int kvh = it / a.n_rt, rt = it % a.n_rt;
   const int qpt_eff = min(a.qpt, a.q_len - rt * a.qpt);
-  if (r >= qpt_eff * a.group) return;
+  const bool row_ok = r < qpt_eff * a.group;
   // The split, recomputed exactly as the attention kernel did.
   long long T = 0, cb = 0;
   int ncb = 0;
@@ -699,62 +708,56 @@ attn_merge_kernel(const TcArgs a) {
   const int n = a.n_cta;
   const long long x_start = cb + (long long)it * ncb, x_end = x_start + ncb;
   const int cta_lo = cta_of(x_start, T, n), cta_hi = cta_of(x_end - 1, T, n);
-  if (cta_lo == cta_hi) return;  // written directly by its only CTA
-  const int cg = lane % CGL, pg = lane / CGL;
-  float M = kEmptyMax, L = 0.f, acc[COLS];
-#pragma unroll
-  for (int t = 0; t < COLS; ++t) acc[t] = 0.f;
-  for (int j = cta_lo + pg; j <= cta_hi; j += PG) {
-    if (!cta_nonempty(j, T, n)) continue;
-    const int sl = partial_slot(j, cta_lo, x_start, T, n);
-    const float2 ml = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
-    const float4* src =
-        reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128 + cg * COLS);
-    float4 v[COLS / 4];
-#pragma unroll
-    for (int t = 0; t < COLS / 4; ++t) v[t] = __ldcg(src + t);
-    const float m_new = fmaxf(M, ml.x);
-    const float f_old = exp2f(M - m_new), w = exp2f(ml.x - m_new);
-    L = L * f_old + ml.y * w;
-#pragma unroll
-    for (int t = 0; t < COLS / 4; ++t) {
-      acc[4 * t] = acc[4 * t] * f_old + v[t].x * w;
-      acc[4 * t + 1] = acc[4 * t + 1] * f_old + v[t].y * w;
-      acc[4 * t + 2] = acc[4 * t + 2] * f_old + v[t].z * w;
-      acc[4 * t + 3] = acc[4 * t + 3] * f_old + v[t].w * w;
-    }
-    M = m_new;
-  }
-  // Combine the partial groups: lanes with the same cg, strides CGL.
-  float Mall = M;
-#pragma unroll
-  for (int o = CGL; o < 32; o <<= 1) Mall = fmaxf(Mall, __shfl_xor_sync(0xffffffffu, Mall, o));
-  const float f = exp2f(M - Mall);
-  L *= f;
-#pragma unroll
-  for (int o = CGL; o < 32; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-#pragma unroll
-  for (int t = 0; t < COLS; ++t) {
-    float v = acc[t] * f;
-#pragma unroll
-    for (int o = CGL; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    acc[t] = v;
-  }
-  if (pg == 0) {
-    const float inv = 1.f / L;
-    const int pq = r / a.group, jq = r % a.group;
-    bf16* dst = a.out + (((size_t)b * a.q_len + rt * a.qpt + pq) * a.Hq + kvh * a.group + jq) * 128 +
-                cg * COLS;
-#pragma unroll
-    for (int t = 0; t < COLS / 8; ++t) {
-      uint4 v;
-      v.x = pack_bf16(acc[8 * t + 0] * inv, acc[8 * t + 1] * inv);
-      v.y = pack_bf16(acc[8 * t + 2] * inv, acc[8 * t + 3] * inv);
-      v.z = pack_bf16(acc[8 * t + 4] * inv, acc[8 * t + 5] * inv);
-      v.w = pack_bf16(acc[8 * t + 6] * inv, acc[8 * t + 7] * inv);
-      reinterpret_cast<uint4*>(dst)[t] = v;
+  if (cta_lo == cta_hi) return;  // written directly by its only CTA (uniform in the CTA)
+  float M = kEmptyMax, L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (row_ok) {
+#pragma unroll 4
+    for (int j = cta_lo + wq; j <= cta_hi; j += WPR) {
+      if (!cta_nonempty(j, T, n)) continue;
+      const int sl = partial_slot(j, cta_lo, x_start, T, n);
+      const float2 ml = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
+      const float4 v =
+          __ldcg(reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128) + lane);
+      const float m_new = fmaxf(M, ml.x);
+      const float f_old = exp2f(M - m_new), w = exp2f(ml.x - m_new);
+      L = L * f_old + ml.y * w;
+      acc.x = acc.x * f_old + v.x * w;
+      acc.y = acc.y * f_old + v.y * w;
+      acc.z = acc.z * f_old + v.z * w;
+      acc.w = acc.w * f_old + v.w * w;
+      M = m_new;
     }
   }
+  if (lane == 0) {
+    s_m[half][wq] = M;
+    s_l[half][wq] = L;
+  }
+  s_acc[half][wq][lane] = acc;
+  __syncthreads();
+  if (wq != 0 || !row_ok) return;
+  float Mall = s_m[half][0];
+#pragma unroll
+  for (int w = 1; w < WPR; ++w) Mall = fmaxf(Mall, s_m[half][w]);
+  float Lall = 0.f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int w = 0; w < WPR; ++w) {
+    const float f = exp2f(s_m[half][w] - Mall);
+    const float4 v = s_acc[half][w][lane];
+    Lall += s_l[half][w] * f;
+    o.x += v.x * f;
+    o.y += v.y * f;
+    o.z += v.z * f;
+    o.w += v.w * f;
+  }
+  const float inv = 1.f / Lall;
+  const int pq = r / a.group, jq = r % a.group;
+  bf16* dst = a.out + (((size_t)b * a.q_len + rt * a.qpt + pq) * a.Hq + kvh * a.group + jq) * 128;
+  uint2 packed;
+  packed.x = pack_bf16(o.x * inv, o.y * inv);
+  packed.y = pack_bf16(o.z * inv, o.w * inv);
+  reinterpret_cast<uint2*>(dst)[lane] = packed;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -807,9 +810,17 @@ int attn_tc_qpt(int q_len, int group) {
   return qpt < q_len ? qpt : q_len;
 }
 
-size_t attn_tc_smem_bytes(int stages) {
-  return 1024 + kQBufs * kQBuf + stages * kKVSlot + sizeof(Smem);
+size_t attn_tc_smem_bytes(int stages, int q_region) {
+  return 1024 + kQBufs * 2 * (size_t)q_region + stages * kKVSlot + sizeof(Smem);
 }
+
+// Shared memory of one attention CTA (beside the LM head: one K/V stage).
+size_t attn_tc_smem_for(int q_len, int group, bool beside) {
+  const int qpt = attn_tc_qpt(q_len, group);
+  return attn_tc_smem_bytes(beside ? 1 : kAloneStages,
+                            qpt * group <= 64 ? kQRegionCompact : kQRegion);
+}
+
 
 cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
                            unsigned int* tickets, int n_cta, cudaStream_t s,
@@ -857,10 +868,11 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   t.part_o = part_o;
   t.part_ml = part_ml;
   t.inline_merge = beside_prior ? 1 : 0;
+  t.q_region = qpt * a.group <= 64 ? kQRegionCompact : kQRegion;
   // Beside the LM head: one K/V stage, so the SM's remaining shared memory
   // goes to that kernel's weight ring.
   const int stages = beside_prior ? 1 : kAloneStages;
-  const size_t smem = attn_tc_smem_bytes(stages);
+  const size_t smem = attn_tc_smem_bytes(stages, t.q_region);
   auto kern = beside_prior ? attn_tc_kernel<1> : attn_tc_kernel<kAloneStages>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
@@ -885,18 +897,18 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   if (beside_prior) return cudaSuccess;  // merged inside the kernel
   cudaLaunchConfig_t lc = {};
   const int n_items = a.B * a.Hkv * t.n_rt;
-  lc.gridDim = dim3(n_items, (qpt * a.group + 7) / 8, 1);
+  // Warps per row ~ partials per split item (about n_cta / n_items + 1).
+  const int est = n_cta / n_items + 1;
+  const int wpr = est <= 2 ? 1 : (est <= 6 ? 2 : 4);
+  lc.gridDim = dim3(n_items, (qpt * a.group + 8 / wpr - 1) / (8 / wpr), 1);
   lc.blockDim = dim3(256, 1, 1);
   lc.dynamicSmemBytes = 0;
   lc.stream = s;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  // Partials per split item are about n_cta / n_items + 1 (the split is
-  // even); the lanes spread over that many partial groups.
-  const int est = n_cta / n_items + 1;
-  e = est <= 4 ? cudaLaunchKernelEx(&lc, attn_merge_kernel<4>, t)
-               : (est <= 8 ? cudaLaunchKernelEx(&lc, attn_merge_kernel<8>, t)
-                           : cudaLaunchKernelEx(&lc, attn_merge_kernel<16>, t));
+  e = wpr == 1 ? cudaLaunchKernelEx(&lc, attn_merge_kernel<1>, t)
+               : (wpr == 2 ? cudaLaunchKernelEx(&lc, attn_merge_kernel<2>, t)
+                           : cudaLaunchKernelEx(&lc, attn_merge_kernel<4>, t));
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -162,9 +162,9 @@ int check_lmhead_supported(const fdl_step_cfg& c) {
   return FDL_OK;
 }
 
-int run_lmhead(const LmArgs& a, const fdl_step_cfg& c, cudaStream_t s, bool shared = false,
+int run_lmhead(const LmArgs& a, const fdl_step_cfg& c, cudaStream_t s, size_t beside_smem = 0,
                bool after_gather = false) {
-  cudaError_t e = c.dtype == FDL_BF16 ? launch_lmhead_tc(a, s, shared, after_gather)
+  cudaError_t e = c.dtype == FDL_BF16 ? launch_lmhead_tc(a, s, beside_smem, after_gather)
                                       : launch_lmhead_simt(a, (fdl_dtype)c.dtype, s);
   if (e != cudaSuccess) return cuda_fail(e, "lm-head launch");
   return FDL_OK;
@@ -175,8 +175,8 @@ int run_lmhead(const LmArgs& a, const fdl_step_cfg& c, cudaStream_t s, bool shar
 // at the ridge (as many FLOPs per weight byte as the tensor cores have per
 // HBM byte), so beyond it the passes cost what the arithmetic does.
 int run_lmhead_passes(const LmArgs& a, const fdl_step_cfg& c, const Plan& p, cudaStream_t s,
-                      bool shared = false, bool after_gather = false) {
-  if (a.R <= p.lm_pass_rows) return run_lmhead(a, c, s, shared, after_gather);
+                      bool after_gather = false) {
+  if (a.R <= p.lm_pass_rows) return run_lmhead(a, c, s, 0, after_gather);
   const size_t row_bytes = (size_t)c.hidden * p.elem;
   for (int r0 = 0; r0 < a.R; r0 += p.lm_pass_rows) {
     LmArgs pa = a;
@@ -194,7 +194,7 @@ int run_lmhead_passes(const LmArgs& a, const fdl_step_cfg& c, const Plan& p, cud
       pa.n_committed = a.n_committed + b0;
       pa.n_masked_left = a.n_masked_left + b0;
     }
-    const int rc = run_lmhead(pa, c, s, shared, after_gather && r0 == 0);
+    const int rc = run_lmhead(pa, c, s, 0, after_gather && r0 == 0);
     if (rc != FDL_OK) return rc;
   }
   return FDL_OK;
@@ -482,8 +482,9 @@ int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
     rc = lm_rows(hidden, &rows);
     if (rc != FDL_OK) return rc;
     LmArgs a = lm_fused(rows);
-    if (lmhead_tc_shared_ok(a)) {
-      rc = run_lmhead(a, c, s, true, c.shift != 0);
+    const size_t attn_smem = attn_tc_smem_for(c.q_len, c.n_q_heads / c.n_kv_heads, true);
+    if (lmhead_tc_shared_ok(a, attn_smem)) {
+      rc = run_lmhead(a, c, s, attn_smem, c.shift != 0);
       if (rc != FDL_OK) return rc;
       rc = run_attention(c, p, dual, q, k_pre, v_pre, len_pre, k_blk, v_blk, k_suf, v_suf,
                          len_suf, out, ws, s, true);
@@ -502,7 +503,7 @@ int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
   const void* rows = nullptr;
   rc = lm_rows(hidden != nullptr ? hidden : out, &rows);
   if (rc != FDL_OK) return rc;
-  rc = run_lmhead_passes(lm_fused(rows), c, p, s, false, c.shift != 0);
+  rc = run_lmhead_passes(lm_fused(rows), c, p, s, c.shift != 0);
   return rc != FDL_OK ? rc : ok();
 }
 

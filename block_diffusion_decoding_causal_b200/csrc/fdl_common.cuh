@@ -268,13 +268,16 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
                            unsigned int* tickets, int n_cta, cudaStream_t s,
                            bool beside_prior = false);
 cudaError_t launch_lmhead_simt(const LmArgs& a, fdl_dtype dt, cudaStream_t s);
-// shared: leave room on every SM for one attention CTA (see lmhead_tc.cu).
+// beside_smem > 0: the shared form, leaving room on every SM for one
+// attention CTA of that many bytes of shared memory (see lmhead_tc.cu).
 // after_producer: a programmatic dependent of the kernel before it (the
 // token-shift gather that writes its rows), which it waits for only before
 // its first read of the rows.
-cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, bool shared = false,
+cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem = 0,
                              bool after_producer = false);
-bool lmhead_tc_shared_ok(const LmArgs& a);
+bool lmhead_tc_shared_ok(const LmArgs& a, size_t beside_smem);
+// Shared memory of one tensor-core attention CTA for these shapes.
+size_t attn_tc_smem_for(int q_len, int group, bool beside);
 cudaError_t launch_commit(const float* conf, const int32_t* tok,
                           int32_t* block_tokens, uint8_t* committed,
                           int32_t* n_committed, int32_t* n_masked_left, int B,

@@ -352,42 +352,29 @@ cudaError_t launch_nch(const CUtensorMap& wf, const CUtensorMap& wp, const CUten
 
 // Tiles per CTA, group size, ring depths and TMEM columns for a call.
 //
-// Shared mode: the CTA leaves room on its SM for one attention CTA of the
-// same step in its one-stage form (71 KB shared memory, 256 TMEM columns,
-// 192 threads of 168 registers), so the two kernels stream HBM side by side.
-// Its shared memory stays between 114 and 152 KB: two LM-head CTAs never fit
-// on one SM, one LM-head CTA and one attention CTA always do; TMEM stays
-// within 256 columns and registers within 168 per thread (R <= 64).
-bool lmhead_tc_params(int R, int H, int rows_per_cta, bool shared, TcParams* tp,
+// Shared mode (beside_smem > 0): the CTA leaves room on its SM for one
+// attention CTA of the same step that needs beside_smem bytes of shared
+// memory, 256 TMEM columns and 192 threads of 168 registers, so the two
+// kernels stream HBM side by side.  Its shared memory is what is left of
+// the SM's 228 KB after that CTA and the two per-CTA reservations, and must
+// exceed half the SM (so two LM-head CTAs never share one); TMEM stays within
+// 256 columns and registers within 168 per thread (R <= 64).  The widest K
+// stage (4, 2 or 1 boxes of 64) that still fits two weight stages is taken.
+bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcParams* tp,
                       size_t* smem);
 
-// Shared-mode ring: K width per stage (boxes of 64), X stages, and the bytes
-// of both rings together.
-#ifndef FDL_LM_SHARED_KSUB
-#define FDL_LM_SHARED_KSUB 2
-#endif
-#ifndef FDL_LM_SHARED_STAGES_B
-#define FDL_LM_SHARED_STAGES_B 2
-#endif
-#ifndef FDL_LM_SHARED_RING_KB
-#define FDL_LM_SHARED_RING_KB 144
-#endif
+namespace {
+constexpr size_t kSmPerSM = 228 * 1024;  // unified shared memory of one SM
+constexpr size_t kSmReserve = 1024;      // reserved by the system per CTA
+}  // namespace
 
-bool lmhead_tc_params(int R, int H, int rows_per_cta, bool shared, TcParams* tp,
+bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcParams* tp,
                       size_t* smem) {
+  const bool shared = beside_smem > 0;
   int nch = 1;
   while (nch * 32 < R) nch *= 2;
   if (nch > (shared ? 2 : 8)) return false;
   tp->npad = nch * 32;
-  // K width per stage: up to 4 boxes (512 contiguous bytes of each weight
-  // row), as long as the B stage stays within 16 KB; 2 boxes when shared.
-  const int kchunks = H / kKChunk;
-  int kmax = 16384 / (tp->npad * 128);
-  if (shared && kmax > FDL_LM_SHARED_KSUB) kmax = FDL_LM_SHARED_KSUB;
-  if (kmax < 1) kmax = 1;
-  tp->ksub = 1;
-  for (int k = 4; k >= 2; k >>= 1)
-    if (k <= kmax && kchunks % k == 0) { tp->ksub = k; break; }
   // Tiles per TMEM buffer: about half a CTA's range, so each X chunk serves
   // several weight tiles and the epilogue of one group hides under the next
   // group's stream (both buffers together stay within TMEM's 512 columns, or
@@ -401,42 +388,53 @@ bool lmhead_tc_params(int R, int H, int rows_per_cta, bool shared, TcParams* tp,
   }
   if (G < 1) G = 1;
   tp->group = G;
-  if (kchunks % tp->ksub != 0) return false;
   const int col_limit = shared ? 256 : 512;
-  if (tp->group < 1 || 2 * tp->group * tp->npad > col_limit) return false;
+  if (2 * tp->group * tp->npad > col_limit) return false;
   uint32_t cols = 32;
   while (cols < (uint32_t)(2 * tp->group * tp->npad)) cols *= 2;
   tp->tmem_cols = cols;
-  const size_t a_stage = (size_t)kStageA * tp->ksub;
-  const size_t b_stage = (size_t)tp->npad * 128 * tp->ksub;
-  tp->stages_b = shared ? FDL_LM_SHARED_STAGES_B : (b_stage <= 16384 ? 4 : 2);
-  const size_t b_bytes = (size_t)tp->stages_b * b_stage;
-  const size_t budget = (shared ? FDL_LM_SHARED_RING_KB : 200) * 1024;
-  if (b_bytes + 2 * a_stage > budget) return false;
-  int sa = (int)((budget - b_bytes) / a_stage);
-  if (sa > 12) sa = 12;
-  if (sa < 2) return false;
-  tp->stages_a = sa;
-  const size_t bars = 8 * (size_t)(2 * sa + 2 * tp->stages_b + 5) + 16;
-  *smem = 1024 + (size_t)sa * a_stage + b_bytes + bars + 4 * (size_t)tp->npad * sizeof(MSI);
-  if (shared) {
-    if (*smem > 152 * 1024) return false;
-    if (*smem < 114 * 1024) *smem = 114 * 1024;
+  // Shared memory: the full form keeps 200 KB of rings; the shared form
+  // what the SM has left.
+  const size_t cap = shared ? (beside_smem + 2 * kSmReserve < kSmPerSM
+                                   ? kSmPerSM - beside_smem - 2 * kSmReserve : 0)
+                            : 227 * 1024;
+  const int kchunks = H / kKChunk;
+  for (int ksub = 4; ksub >= 1; ksub >>= 1) {
+    if (kchunks % ksub != 0) continue;
+    const size_t b_stage = (size_t)tp->npad * 128 * ksub;
+    if (b_stage > 16384 && ksub > 1) continue;  // X stage within 16 KB when possible
+    const size_t a_stage = (size_t)kStageA * ksub;
+    const int sb = shared ? 2 : (b_stage <= 16384 ? 4 : 2);
+    const size_t b_bytes = (size_t)sb * b_stage;
+    const size_t fixed = 1024 + 8 * (size_t)(2 * 12 + 2 * sb + 5) + 16 +
+                         4 * (size_t)tp->npad * sizeof(MSI);
+    const size_t ring_cap = shared ? cap : fixed + 200 * 1024;
+    if (ring_cap < fixed + b_bytes + 2 * a_stage) continue;
+    int sa = (int)((ring_cap - fixed - b_bytes) / a_stage);
+    if (sa > 12) sa = 12;
+    tp->ksub = ksub;
+    tp->stages_b = sb;
+    tp->stages_a = sa;
+    const size_t bars = 8 * (size_t)(2 * sa + 2 * sb + 5) + 16;
+    *smem = 1024 + (size_t)sa * a_stage + b_bytes + bars + 4 * (size_t)tp->npad * sizeof(MSI);
+    if (shared && 2 * (*smem + kSmReserve) <= kSmPerSM) *smem = kSmPerSM / 2;  // one per SM
+    if (*smem > cap) return false;
+    return true;
   }
-  return true;
+  return false;
 }
 
-bool lmhead_tc_shared_ok(const LmArgs& a) {
+bool lmhead_tc_shared_ok(const LmArgs& a, size_t beside_smem) {
   TcParams tp;
   size_t smem = 0;
-  return lmhead_tc_params(a.R, a.H, a.rows_per_cta, true, &tp, &smem);
+  return lmhead_tc_params(a.R, a.H, a.rows_per_cta, beside_smem, &tp, &smem);
 }
 
-cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, bool shared,
+cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem,
                              bool after_producer) {
   TcParams tp;
   size_t smem = 0;
-  if (!lmhead_tc_params(a.R, a.H, a.rows_per_cta, shared, &tp, &smem))
+  if (!lmhead_tc_params(a.R, a.H, a.rows_per_cta, beside_smem, &tp, &smem))
     return cudaErrorInvalidValue;
   CUtensorMap wf, wp, x;
   if (!make_map(&wf, a.w, a.H, a.V, kKChunk, kTileM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||

@@ -171,3 +171,61 @@ def test_block_graph_with_fused_step_and_append():
     assert int(dcase["len_pre"][0]) == len0 + D
     assert torch.equal(dcase["k_pre"][0, :, len0:len0 + D].cpu(), case.k_blk[0])
     assert fdl.get_status(ws) == 0
+
+
+def test_block_graph_on_the_tensor_core_step_matches_the_host_loop():
+    """The bf16 / head-dim-128 fused step (LM head first, attention beside it
+    through programmatic launches, token-shift gather before them) captured
+    in the WHILE-node graph: same tokens, step counts and appended cache as
+    the host-driven loop."""
+    c = dict(synth.CONFIGS["qwen7b"], batch=2, prefix=(300, 500), cap_prefix=600, q_off=0,
+             vocab=8000, mask_id=7999, hidden=512, masked=(8, 8), tau=0.9)
+    for seed in range(20):          # a case whose argmax is never the mask token
+        case = synth.make_case("graph_tc", seed, cfg=dict(c))
+        if (cases.run_oracle(case)["tok"] != c["mask_id"]).all():
+            break
+    B, D, q_len = c["batch"], c["block_size"], c["q_len"]
+    units = D // q_len
+    cfgs = [fdl.make_cfg(dict(case.cfg, q_off=u * q_len)) for u in range(units)]
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in vars(case).items()}
+
+    def run(use_graph):
+        kp, vp, lens = d["k_pre"].clone(), d["v_pre"].clone(), d["len_pre"].clone()
+        bt = torch.full((B, D), c["mask_id"], dtype=torch.int32, device="cuda")
+        o = dict(attn=torch.empty_like(d["q"]),
+                 conf=torch.empty((B, q_len), dtype=torch.float32, device="cuda"),
+                 tok=torch.empty((B, q_len), dtype=torch.int32, device="cuda"),
+                 comm=torch.empty((B, D), dtype=torch.uint8, device="cuda"),
+                 n_c=torch.empty(B, dtype=torch.int32, device="cuda"),
+                 n_l=torch.empty(B, dtype=torch.int32, device="cuda"))
+        steps = torch.zeros(units, dtype=torch.int32, device="cuda")
+        ws = fdl.workspace(cfgs[0])
+
+        def one_step(u, s):
+            fdl.denoise_step(cfgs[u], d["q"], kp, vp, lens, d["k_blk"], d["v_blk"], None, None,
+                             None, d["hidden"], d["h_prev"], d["w_lm"], bt, o["attn"], o["conf"],
+                             o["tok"], o["comm"], o["n_c"], o["n_l"], ws, stream=s)
+
+        def append(s):
+            fdl.append_block(cfgs[0], d["k_blk"], d["v_blk"], kp, vp, lens, ws, stream=s)
+
+        if use_graph:
+            g = driver.BlockGraph(cfgs, one_step, o["n_l"], steps, append=append)
+            g.launch()
+            torch.cuda.synchronize()
+            n = steps.cpu().tolist()
+        else:
+            n = []
+            driver.run_host_loop(cfgs, one_step, o["n_l"],
+                                 torch.zeros(1, dtype=torch.int32, device="cuda"), n)
+            append(torch.cuda.current_stream())
+            torch.cuda.synchronize()
+        assert fdl.get_status(ws) == 0
+        return bt.cpu(), n, lens.cpu(), kp.cpu()
+
+    bt_h, n_h, len_h, kp_h = run(False)
+    bt_g, n_g, len_g, kp_g = run(True)
+    assert not (bt_h == c["mask_id"]).any()
+    assert torch.equal(bt_g, bt_h) and n_g == n_h
+    assert torch.equal(len_g, len_h) and torch.equal(len_h, case.len_pre + D)
+    assert torch.equal(kp_g, kp_h)
