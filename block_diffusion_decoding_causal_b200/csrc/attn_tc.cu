@@ -177,6 +177,15 @@ __device__ __forceinline__ ChunkInfo chunk_info(int j, int Lp, int Ls, int D) {
 
 
 
+// 2^x with the PTX ex2.approx instruction (relative error near 2^-22,
+// subnormal results flushed to zero): the softmax weights are rounded to
+// bf16 right after, so the approximation is far below what is kept.
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -507,18 +516,29 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
       }
       const int pb = sb;
       if (warp_active) {
-        float xs[64];
-        float cmax = kEmptyMax;
+        // Row maximum on the raw scores (the scale is positive); keys past
+        // the chunk's valid count get the empty value, whose weight is 0.
+        const float sc = a.scale_log2;
+        if (ci.nvalid != kCh) {
 #pragma unroll
-        for (int jj = 0; jj < 64; ++jj) {
-          xs[jj] = jj < ci.nvalid ? __uint_as_float(sr[jj]) * a.scale_log2 : kEmptyMax;
-          cmax = fmaxf(cmax, xs[jj]);
+          for (int jj = 0; jj < 64; ++jj)
+            if (jj >= ci.nvalid) sr[jj] = __float_as_uint(kEmptyMax);
         }
+        // Eight independent partial maxima, then a tree: short dependency
+        // chains instead of one of 64.
+        float pm[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) pm[t] = __uint_as_float(sr[t]);
+#pragma unroll
+        for (int jj = 8; jj < 64; ++jj) pm[jj & 7] = fmaxf(pm[jj & 7], __uint_as_float(sr[jj]));
+        const float rmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        const float cmax = rmax * sc;
         float alpha = 1.f;
         if (first) {
           m_used = cmax;
         } else if (cmax > m_used + kRescale) {
-          alpha = exp2f(m_used - cmax);
+          alpha = ex2_fast(m_used - cmax);
           m_used = cmax;
         }
         // O rescale (warp-collective TMEM access) when any row needs it.
@@ -543,16 +563,16 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
           tmem_st_wait();
         }
         l *= alpha;
-        float psum = 0.f;
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
         uint32_t pk[32];
 #pragma unroll
         for (int jj = 0; jj < 64; jj += 2) {
-          const float p0 = exp2f(xs[jj] - m_used);
-          const float p1 = exp2f(xs[jj + 1] - m_used);
-          psum += p0 + p1;
+          const float p0 = ex2_fast(fmaf(__uint_as_float(sr[jj]), sc, -m_used));
+          const float p1 = ex2_fast(fmaf(__uint_as_float(sr[jj + 1]), sc, -m_used));
+          ps[(jj >> 1) & 3] += p0 + p1;
           pk[jj >> 1] = pack_bf16(p0, p1);
         }
-        l += psum;
+        l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         // P (bf16 pairs) over the first 32 columns of this chunk's S.
         tmem_st_32x32b_x32(tmem + lane_addr + (uint32_t)pb * kCh, pk);
         tmem_st_wait();

@@ -404,7 +404,10 @@ bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcPara
     const size_t b_stage = (size_t)tp->npad * 128 * ksub;
     if (b_stage > 16384 && ksub > 1) continue;  // X stage within 16 KB when possible
     const size_t a_stage = (size_t)kStageA * ksub;
-    const int sb = shared ? 2 : (b_stage <= 16384 ? 4 : 2);
+    // Four X stages in the full form: at 256 rows an X chunk (32 KB) is
+    // twice a weight stage and is staged again for every vocabulary tile, so
+    // its ring needs the deeper prefetch.
+    const int sb = shared ? 2 : 4;
     const size_t b_bytes = (size_t)sb * b_stage;
     const size_t fixed = 1024 + 8 * (size_t)(2 * 12 + 2 * sb + 5) + 16 +
                          4 * (size_t)tp->npad * sizeof(MSI);

@@ -18,7 +18,9 @@ from block_diffusion_decoding_causal_b200 import fdl, synth
 def main() -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", default="lmhead",
-                    choices=["lmhead", "attn", "dualcache", "step"])
+                    choices=["lmhead", "attn", "dualcache", "step", "prefixcache"])
+    ap.add_argument("--rows", type=int, default=768,
+                    help="prefixcache: recomputed rows (block + suffix)")
     ap.add_argument("--workload", default="qwen7b")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--prefix", type=int, default=None)
@@ -31,6 +33,9 @@ def main() -> int:
     if args.prefix is not None:
         c.update(prefix=(args.prefix, args.prefix), cap_prefix=args.prefix)
     c["q_off"] = c["q_off"] or 0
+    if args.kernel == "prefixcache":
+        # the recomputed rows take the block's place: queries = keys = rows
+        c.update(block_size=args.rows, q_len=args.rows, q_off=0, cap_suffix=0, suffix=0)
     B, q_len, H, V = c["batch"], c["q_len"], c["hidden"], c["vocab"]
     Hq, Hkv, d, D = c["n_q_heads"], c["n_kv_heads"], c["head_dim"], c["block_size"]
     dt = synth.torch_dtype(c["dtype"])
@@ -45,7 +50,7 @@ def main() -> int:
     len_pre = torch.randint(lo, hi + 1, (B,), generator=g, device="cuda", dtype=torch.int32)
     q = rn(B, q_len, Hq, d)
     out = torch.empty_like(q)
-    if args.kernel in ("attn", "dualcache", "step"):
+    if args.kernel in ("attn", "dualcache", "step", "prefixcache"):
         kp, vp = rn(B, Hkv, cap_p, d), rn(B, Hkv, cap_p, d)
         kb, vb = rn(B, Hkv, D, d), rn(B, Hkv, D, d)
         if cap_s:
@@ -57,6 +62,8 @@ def main() -> int:
     for _ in range(args.launches):
         if args.kernel == "lmhead":
             fdl.lmhead_confidence(cfg, rows, w, None, conf, tok, ws)
+        elif args.kernel == "prefixcache":
+            fdl.prefixcache_attn(cfg, q, kp, vp, len_pre, kb, vb, out, ws)
         elif args.kernel == "attn":
             fdl.block_attn(cfg, q, kp, vp, len_pre, kb, vb, out, ws)
         elif args.kernel == "dualcache":
