@@ -63,6 +63,7 @@ constexpr int kThreads = 192;
 constexpr float kRescale = 8.0f;         // log2-domain growth forcing a rescale
 constexpr unsigned kDevTimeout = FDL_DEV_TIMEOUT;
 constexpr int kMaxSeq = 256;
+constexpr int kMaxMergeParts = 512;      // >= CTAs of any attention grid
 
 struct TcArgs {
   int B, Hq, Hkv, q_len, D, cap_p, cap_s, group, qpt, n_rt, n_cta, dual;
@@ -682,22 +683,13 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
 // and warp); the row's warps then combine through shared memory.  Launched
 // as a programmatic dependent of the attention grid: scheduled as its CTAs
 // retire, it waits for the whole grid before reading anything.
-template <int WPR>
-__global__ void __launch_bounds__(256)
-attn_merge_kernel(const TcArgs a) {
-  constexpr int RPC = 8 / WPR;  // rows per CTA
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ float s_m[RPC][WPR], s_l[RPC][WPR];
-  __shared__ float4 s_acc[RPC][WPR][32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = warp / WPR, wq = warp % WPR;
+// Warp-collective: the partial slots of item (b, it), in CTA order, into
+// slot[] (at most kMaxMergeParts) and their count into *n_out (lane 0); the
+// split recomputed exactly as the attention kernel did.
+__device__ __noinline__ void item_partial_slots(const TcArgs& a, int b, int it, int* slot,
+                                                int* n_out) {
+  const int lane = threadIdx.x & 31;
   const int per_seq = a.Hkv * a.n_rt;
-  const int x = blockIdx.x, r = blockIdx.y * RPC + half;
-  const int b = x / per_seq, it = x % per_seq;
-  const int kvh = it / a.n_rt, rt = it % a.n_rt;
-  const int qpt_eff = min(a.qpt, a.q_len - rt * a.qpt);
-  const bool row_ok = r < qpt_eff * a.group;
-  // The split, recomputed exactly as the attention kernel did.
   long long T = 0, cb = 0;
   int ncb = 0;
   for (int b0 = 0; b0 < a.B; b0 += 32) {
@@ -728,14 +720,49 @@ attn_merge_kernel(const TcArgs a) {
   const int n = a.n_cta;
   const long long x_start = cb + (long long)it * ncb, x_end = x_start + ncb;
   const int cta_lo = cta_of(x_start, T, n), cta_hi = cta_of(x_end - 1, T, n);
-  if (cta_lo == cta_hi) return;  // written directly by its only CTA (uniform in the CTA)
+  // Lanes take CTAs cta_lo + lane, + 32, ...; the nonempty ones keep their
+  // order through a ballot prefix count.  One CTA alone: no partials.
+  int count = 0;
+  if (cta_lo != cta_hi) {
+    for (int j0 = cta_lo; j0 <= cta_hi; j0 += 32) {
+      const int j = j0 + lane;
+      const bool have = j <= cta_hi && cta_nonempty(j, T, n);
+      const unsigned m = __ballot_sync(0xffffffffu, have);
+      const int pos = count + __popc(m & ((1u << lane) - 1u));
+      if (have && pos < kMaxMergeParts) slot[pos] = partial_slot(j, cta_lo, x_start, T, n);
+      count += __popc(m);
+    }
+  }
+  if (lane == 0) *n_out = count < kMaxMergeParts ? count : kMaxMergeParts;
+}
+
+template <int WPR>
+__global__ void __launch_bounds__(256)
+attn_merge_kernel(const TcArgs a) {
+  constexpr int RPC = 8 / WPR;  // rows per CTA
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ float s_m[RPC][WPR], s_l[RPC][WPR];
+  __shared__ float4 s_acc[RPC][WPR][32];
+  __shared__ int s_slot[kMaxMergeParts];  // partial slots of the item, in order
+  __shared__ int s_n;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = warp / WPR, wq = warp % WPR;
+  const int per_seq = a.Hkv * a.n_rt;
+  const int x = blockIdx.x, r = blockIdx.y * RPC + half;
+  const int b = x / per_seq, it = x % per_seq;
+  const int kvh = it / a.n_rt, rt = it % a.n_rt;
+  const int qpt_eff = min(a.qpt, a.q_len - rt * a.qpt);
+  const bool row_ok = r < qpt_eff * a.group;
+  if (warp == 0) item_partial_slots(a, b, it, s_slot, &s_n);
+  __syncthreads();
+  const int n_parts = s_n;
+  if (n_parts == 0) return;  // written directly by its only CTA (uniform in the CTA)
   float M = kEmptyMax, L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (row_ok) {
 #pragma unroll 4
-    for (int j = cta_lo + wq; j <= cta_hi; j += WPR) {
-      if (!cta_nonempty(j, T, n)) continue;
-      const int sl = partial_slot(j, cta_lo, x_start, T, n);
+    for (int q = wq; q < n_parts; q += WPR) {
+      const int sl = s_slot[q];
       const float2 ml = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
       const float4 v =
           __ldcg(reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128) + lane);
@@ -778,6 +805,74 @@ attn_merge_kernel(const TcArgs a) {
   packed.x = pack_bf16(o.x * inv, o.y * inv);
   packed.y = pack_bf16(o.z * inv, o.w * inv);
   reinterpret_cast<uint2*>(dst)[lane] = packed;
+}
+
+// Merge for items with few partials (about two each, the usual case when
+// there are more items than CTAs): a CTA holds 32 rows of one item, each warp
+// four rows whose partial reads are all in flight together; lanes hold four
+// of the 128 columns.
+__global__ void __launch_bounds__(256)
+attn_merge_few_kernel(const TcArgs a) {
+  constexpr int RW = 4;  // rows per warp
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ int s_slot[kMaxMergeParts];
+  __shared__ int s_n;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per_seq = a.Hkv * a.n_rt;
+  const int x = blockIdx.x;
+  const int b = x / per_seq, it = x % per_seq;
+  const int kvh = it / a.n_rt, rt = it % a.n_rt;
+  const int qpt_eff = min(a.qpt, a.q_len - rt * a.qpt);
+  const int rows = qpt_eff * a.group;
+  if (warp == 0) item_partial_slots(a, b, it, s_slot, &s_n);
+  __syncthreads();
+  const int n_parts = s_n;
+  const int r0 = blockIdx.y * 32 + warp * RW;
+  if (n_parts == 0 || r0 >= rows) return;
+  float M[RW], L[RW];
+  float4 acc[RW];
+#pragma unroll
+  for (int k = 0; k < RW; ++k) {
+    M[k] = kEmptyMax;
+    L[k] = 0.f;
+    acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int q = 0; q < n_parts; ++q) {
+    const int sl = s_slot[q];
+    float2 ml[RW];
+    float4 v[RW];
+#pragma unroll
+    for (int k = 0; k < RW; ++k) {  // rows past the item read a valid slot row, unused
+      const int r = min(r0 + k, 127);
+      ml[k] = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
+      v[k] = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128) +
+                    lane);
+    }
+#pragma unroll
+    for (int k = 0; k < RW; ++k) {
+      const float m_new = fmaxf(M[k], ml[k].x);
+      const float f_old = exp2f(M[k] - m_new), w = exp2f(ml[k].x - m_new);
+      L[k] = L[k] * f_old + ml[k].y * w;
+      acc[k].x = acc[k].x * f_old + v[k].x * w;
+      acc[k].y = acc[k].y * f_old + v[k].y * w;
+      acc[k].z = acc[k].z * f_old + v[k].z * w;
+      acc[k].w = acc[k].w * f_old + v[k].w * w;
+      M[k] = m_new;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < RW; ++k) {
+    const int r = r0 + k;
+    if (r >= rows) break;
+    const float inv = 1.f / L[k];
+    const int pq = r / a.group, jq = r % a.group;
+    bf16* dst =
+        a.out + (((size_t)b * a.q_len + rt * a.qpt + pq) * a.Hq + kvh * a.group + jq) * 128;
+    uint2 packed;
+    packed.x = pack_bf16(acc[k].x * inv, acc[k].y * inv);
+    packed.y = pack_bf16(acc[k].z * inv, acc[k].w * inv);
+    reinterpret_cast<uint2*>(dst)[lane] = packed;
+  }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -917,16 +1012,18 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   if (beside_prior) return cudaSuccess;  // merged inside the kernel
   cudaLaunchConfig_t lc = {};
   const int n_items = a.B * a.Hkv * t.n_rt;
-  // Warps per row ~ partials per split item (about n_cta / n_items + 1).
+  // Partials per split item are about n_cta / n_items + 1: few, and a CTA
+  // takes 32 rows (4 per warp); more, and 1, 2 or 4 warps share a row.
   const int est = n_cta / n_items + 1;
-  const int wpr = est <= 2 ? 1 : (est <= 6 ? 2 : 4);
-  lc.gridDim = dim3(n_items, (qpt * a.group + 8 / wpr - 1) / (8 / wpr), 1);
+  const int wpr = est <= 3 ? 0 : (est <= 6 ? 2 : 4);
+  const int rows_per_cta = wpr == 0 ? 32 : 8 / wpr;
+  lc.gridDim = dim3(n_items, (qpt * a.group + rows_per_cta - 1) / rows_per_cta, 1);
   lc.blockDim = dim3(256, 1, 1);
   lc.dynamicSmemBytes = 0;
   lc.stream = s;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  e = wpr == 1 ? cudaLaunchKernelEx(&lc, attn_merge_kernel<1>, t)
+  e = wpr == 0 ? cudaLaunchKernelEx(&lc, attn_merge_few_kernel, t)
                : (wpr == 2 ? cudaLaunchKernelEx(&lc, attn_merge_kernel<2>, t)
                            : cudaLaunchKernelEx(&lc, attn_merge_kernel<4>, t));
   if (e != cudaSuccess) return e;
