@@ -41,20 +41,22 @@ using namespace sm100;
 
 constexpr int kCh = 64;                  // keys per chunk
 constexpr int kQRegion = 128 * 128;      // 128 rows x 64 bf16 (16 KB)
-// Rows of an item at most 64: the Q halves (d 0-63, 64-127) sit 8 KB apart
-// and the buffer is 16 KB.  The MMA still reads 128 rows per half; rows 64+
-// then fall on the other half or the K/V stage that follows, which only
-// feeds S rows no softmax thread reads (rows of an item never mix).
-constexpr int kQRegionCompact = 64 * 128;
+// Rows of an item at most 64: the Q halves (d 0-63, 64-127) sit only the
+// rows (rounded to 8) apart, 16 KB at most for both.  The MMA still reads 128
+// rows per half; the rows past the item then fall on the other half or the
+// K/V stage that follows, which only feeds S rows no softmax thread reads
+// (rows of an M = 128 tile never mix).
+constexpr int kQRegionMaxCompact = 64 * 128;
+// Bytes between the two d-halves of the Q buffer: the item's rows rounded up
+// to the 8-row swizzle atom when they are at most 64, else 128 rows.
+__host__ __device__ constexpr int q_region_for(int rows) {
+  return rows <= 64 ? ((rows + 7) / 8) * 8 * 128 : 128 * 128;
+}
 constexpr int kKVRegion = kCh * 128;     // 64 keys x 64 bf16 (8 KB)
 constexpr int kKVSlot = 4 * kKVRegion;   // K lo, K hi, V lo, V hi: one 32 KB stage
 // K/V stages of the attention alone on the GPU (two CTAs per SM at 2) and
 // beside the LM head (1).
-#ifndef FDL_ATTN_ALONE_STAGES
-#define FDL_ATTN_ALONE_STAGES 2
-#endif
-constexpr int kAloneStages = FDL_ATTN_ALONE_STAGES;
-constexpr int kMaxStages = kAloneStages > 1 ? kAloneStages : 1;
+constexpr int kMaxStages = 3;            // two CTAs per SM fit three stages when Q is small
 constexpr int kQBufs = 1;                // Q is reloaded per item
 constexpr int kSB = 2;                   // S buffers in TMEM; P overwrites its S
 constexpr uint32_t kTmemCols = 256;      // S 2 x 64 columns, O 128 columns
@@ -92,10 +94,8 @@ struct Smem {
   uint64_t drain;
   uint32_t tmem;
   int flag;
-  int cb[kMaxSeq + 1];  // first global chunk of sequence b
-  int nc[kMaxSeq];      // chunks per item of sequence b
-  int lp[kMaxSeq];
-  int ls[kMaxSeq];
+  // followed by the sequence table: cb [B + 1] (first global chunk of
+  // sequence b), nc [B] (chunks per item), lp [B], ls [B] (lengths)
 };
 
 // Position in the chunk sequence of one CTA.
@@ -103,23 +103,22 @@ struct Cursor {
   int b, it, j;  // sequence, item within sequence, chunk within item
 };
 
-__device__ __forceinline__ Cursor locate(const Smem& S, int B, int per_seq, long long g) {
+__device__ __forceinline__ Cursor locate(const int* cb, const int* nc, int B, long long g) {
   int lo = 0, hi = B - 1;
   while (lo < hi) {  // last b with cb[b] <= g
     const int mid = (lo + hi + 1) >> 1;
-    if (S.cb[mid] <= g) lo = mid; else hi = mid - 1;
+    if (cb[mid] <= g) lo = mid; else hi = mid - 1;
   }
-  const int rem = (int)(g - S.cb[lo]);
+  const int rem = (int)(g - cb[lo]);
   Cursor c;
   c.b = lo;
-  c.it = rem / S.nc[lo];
-  c.j = rem % S.nc[lo];
-  (void)per_seq;
+  c.it = rem / nc[lo];
+  c.j = rem % nc[lo];
   return c;
 }
 
-__device__ __forceinline__ void advance(Cursor& c, const Smem& S, int per_seq) {
-  if (++c.j == S.nc[c.b]) {
+__device__ __forceinline__ void advance(Cursor& c, const int* nc, int per_seq) {
+  if (++c.j == nc[c.b]) {
     c.j = 0;
     if (++c.it == per_seq) {
       c.it = 0;
@@ -261,6 +260,10 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   uint8_t* q_smem = base;                               // kQBufs x 2 x q_region
   uint8_t* kv_smem = q_smem + kQBufs * 2 * a.q_region;  // STAGES x 32 KB
   Smem& S = *reinterpret_cast<Smem*>(kv_smem + STAGES * kKVSlot);
+  int* const cb = reinterpret_cast<int*>(&S + 1);  // sequence table, sized by B
+  int* const nc = cb + a.B + 1;
+  int* const lp = nc + a.B;
+  int* const ls = lp + a.B;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_seq = a.Hkv * a.n_rt;  // items per sequence
@@ -291,7 +294,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
     int run = 0;
     for (int b0 = 0; b0 < a.B; b0 += 32) {
       const int b = b0 + lane;
-      int Lp = 0, Ls = 0, nc = 0;
+      int Lp = 0, Ls = 0, n_ch = 0;
       if (b < a.B) {
         Lp = a.len_pre[b];
         if (Lp < 0 || Lp > a.cap_p) {
@@ -305,23 +308,23 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
             Ls = 0;
           }
         }
-        nc = item_chunks(Lp, Ls, a.D);
+        n_ch = item_chunks(Lp, Ls, a.D);
       }
-      int incl = nc * per_seq;
+      int incl = n_ch * per_seq;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += v;
       }
       if (b < a.B) {
-        S.lp[b] = Lp;
-        S.ls[b] = Ls;
-        S.nc[b] = nc;
-        S.cb[b] = run + incl - nc * per_seq;
+        lp[b] = Lp;
+        ls[b] = Ls;
+        nc[b] = n_ch;
+        cb[b] = run + incl - n_ch * per_seq;
       }
       run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) S.cb[a.B] = run;
+    if (lane == 0) cb[a.B] = run;
   }
   // Padding rows of the Q halves are never written by TMA: zero them once.
   const int q_rows = a.q_region / 128;
@@ -339,7 +342,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   tc_fence_after();
   const uint32_t tmem = S.tmem;
 
-  const long long T = S.cb[a.B];
+  const long long T = cb[a.B];
   const int n = a.n_cta;
   const long long c_begin = cta_start(blockIdx.x, T, n);
   const long long c_end = cta_start(blockIdx.x + 1, T, n);
@@ -352,13 +355,13 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
     if (lane == 0) {
       const int n_my = (int)(c_end - c_begin);
       int q_i = 0, prev_x = -1;
-      Cursor c = locate(S, a.B, per_seq, c_begin);
-      for (int i = 0; i < n_my && !failed; ++i, advance(c, S, per_seq)) {
+      Cursor c = locate(cb, nc, a.B, c_begin);
+      for (int i = 0; i < n_my && !failed; ++i, advance(c, nc, per_seq)) {
         const int x = c.b * per_seq + c.it;
         const int kvh = c.it / a.n_rt, rt = c.it % a.n_rt;
         const int slot = i % STAGES;
         if (!mbar_wait(&S.kv_empty[slot], ((i / STAGES) & 1) ^ 1)) { failed = true; break; }
-        const ChunkInfo ci = chunk_info(c.j, S.lp[c.b], S.ls[c.b], a.D);
+        const ChunkInfo ci = chunk_info(c.j, lp[c.b], ls[c.b], a.D);
         const int bk = c.b * a.Hkv + kvh;
         const CUtensorMap* mk = ci.seg == 0 ? &maps.kp : (ci.seg == 1 ? &maps.kb : &maps.ks);
         const CUtensorMap* mv = ci.seg == 0 ? &maps.vp : (ci.seg == 1 ? &maps.vb : &maps.vs);
@@ -401,7 +404,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
       const uint32_t id_pv = idesc_bf16_f32(128, 128) | (1u << 16);  // V is MN-major
       const int n_my = (int)(c_end - c_begin);
       int is = 0, ip = 0, q_s = 0, o_i = 0, prev_xs = -1, prev_xp = -1;
-      Cursor cs = locate(S, a.B, per_seq, c_begin), cp = cs;
+      Cursor cs = locate(cb, nc, a.B, c_begin), cp = cs;
       long long t_last = clock64();
       while (ip < n_my) {
         bool progress = false;
@@ -418,7 +421,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
               prev_xs = x;
             }
             const int qb = (q_s - 1) % kQBufs;
-            const bool last = (is + 1 == n_my) || (cs.j + 1 == S.nc[cs.b]);
+            const bool last = (is + 1 == n_my) || (cs.j + 1 == nc[cs.b]);
             tc_fence_after();
             const uint32_t q_base = smem_u32(q_smem + qb * 2 * a.q_region);
             const uint32_t k_base = smem_u32(kv_smem + slot * kKVSlot);
@@ -430,7 +433,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
                        k ? 1u : 0u);
             mma_commit(&S.s_full[sb]);
             if (last) mma_commit(&S.q_empty[qb]);
-            advance(cs, S, per_seq);
+            advance(cs, nc, per_seq);
             ++is;
             progress = true;
           }
@@ -443,7 +446,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
           if (first) ready = ready && mbar_test(&S.o_empty[0], (o_i & 1) ^ 1);
           if (ready) {
             if (first) prev_xp = x;
-            const bool last = (ip + 1 == n_my) || (cp.j + 1 == S.nc[cp.b]);
+            const bool last = (ip + 1 == n_my) || (cp.j + 1 == nc[cp.b]);
             tc_fence_after();
             const uint32_t v_base = smem_u32(kv_smem + vslot * kKVSlot + 2 * kKVRegion);
             const uint32_t p_tmem = tmem + (uint32_t)pb * kCh;  // P over its S columns
@@ -458,7 +461,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
               mma_commit(&S.o_full[0]);
               ++o_i;
             }
-            advance(cp, S, per_seq);
+            advance(cp, nc, per_seq);
             ++ip;
             progress = true;
           }
@@ -486,14 +489,14 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
     float m_used = kEmptyMax, l = 0.f;
     int s_i = 0, o_i = 0, prev_x = -1;
     const int first_x = [&] {
-      const Cursor c0 = locate(S, a.B, per_seq, c_begin);
+      const Cursor c0 = locate(cb, nc, a.B, c_begin);
       return c0.b * per_seq + c0.it;
     }();
-    Cursor c = locate(S, a.B, per_seq, c_begin);
-    for (long long g = c_begin; g < c_end && !failed; ++g, advance(c, S, per_seq)) {
+    Cursor c = locate(cb, nc, a.B, c_begin);
+    for (long long g = c_begin; g < c_end && !failed; ++g, advance(c, nc, per_seq)) {
       const int x = c.b * per_seq + c.it;
       const int first = x != prev_x;
-      const int last = (g + 1 == c_end) || (c.j + 1 == S.nc[c.b]);
+      const int last = (g + 1 == c_end) || (c.j + 1 == nc[c.b]);
       const int kvh = c.it / a.n_rt, rt = c.it % a.n_rt;
       const int qpt_eff = min(a.qpt, a.q_len - rt * a.qpt);
       const int rows = qpt_eff * a.group;
@@ -503,7 +506,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
         l = 0.f;
         prev_x = x;
       }
-      const ChunkInfo ci = chunk_info(c.j, S.lp[c.b], S.ls[c.b], a.D);
+      const ChunkInfo ci = chunk_info(c.j, lp[c.b], ls[c.b], a.D);
       const int sb = s_i % kSB;
       if (!mbar_wait(&S.s_full[sb], (s_i / kSB) & 1)) { failed = true; break; }
       tc_fence_after();
@@ -587,8 +590,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
       // ----------------------------------------------------- item epilogue
       if (!mbar_wait(&S.o_full[0], o_i & 1)) { failed = true; break; }
       tc_fence_after();
-      const long long x_start = S.cb[c.b] + (long long)c.it * S.nc[c.b];
-      const long long x_end = x_start + S.nc[c.b];
+      const long long x_start = cb[c.b] + (long long)c.it * nc[c.b];
+      const long long x_end = x_start + nc[c.b];
       const int cta_lo = cta_of(x_start, T, n), cta_hi = cta_of(x_end - 1, T, n);
       const int p_pos = r / a.group, jh = r % a.group;
       const int qi = rt * a.qpt + p_pos;
@@ -925,15 +928,22 @@ int attn_tc_qpt(int q_len, int group) {
   return qpt < q_len ? qpt : q_len;
 }
 
-size_t attn_tc_smem_bytes(int stages, int q_region) {
-  return 1024 + kQBufs * 2 * (size_t)q_region + stages * kKVSlot + sizeof(Smem);
+size_t attn_tc_smem_bytes(int stages, int q_region, int B) {
+  return 1024 + kQBufs * 2 * (size_t)q_region + stages * kKVSlot + sizeof(Smem) +
+         sizeof(int) * (4 * (size_t)B + 1);
 }
 
 // Shared memory of one attention CTA (beside the LM head: one K/V stage).
-size_t attn_tc_smem_for(int q_len, int group, bool beside) {
+// Stages of the attention alone on the GPU: three when two CTAs with three
+// still fit on one SM (228 KB less a 1 KB reservation each), else two.
+int attn_tc_alone_stages(int q_region, int B) {
+  return 2 * (attn_tc_smem_bytes(3, q_region, B) + 1024) <= 228 * 1024 ? 3 : 2;
+}
+
+size_t attn_tc_smem_for(int q_len, int group, int B, bool beside) {
   const int qpt = attn_tc_qpt(q_len, group);
-  return attn_tc_smem_bytes(beside ? 1 : kAloneStages,
-                            qpt * group <= 64 ? kQRegionCompact : kQRegion);
+  const int q_region = q_region_for(qpt * group);
+  return attn_tc_smem_bytes(beside ? 1 : attn_tc_alone_stages(q_region, B), q_region, B);
 }
 
 
@@ -983,12 +993,13 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   t.part_o = part_o;
   t.part_ml = part_ml;
   t.inline_merge = beside_prior ? 1 : 0;
-  t.q_region = qpt * a.group <= 64 ? kQRegionCompact : kQRegion;
+  t.q_region = q_region_for(qpt * a.group);
   // Beside the LM head: one K/V stage, so the SM's remaining shared memory
   // goes to that kernel's weight ring.
-  const int stages = beside_prior ? 1 : kAloneStages;
-  const size_t smem = attn_tc_smem_bytes(stages, t.q_region);
-  auto kern = beside_prior ? attn_tc_kernel<1> : attn_tc_kernel<kAloneStages>;
+  const int stages = beside_prior ? 1 : attn_tc_alone_stages(t.q_region, a.B);
+  const size_t smem = attn_tc_smem_bytes(stages, t.q_region, a.B);
+  auto kern = stages == 1 ? attn_tc_kernel<1> : (stages == 2 ? attn_tc_kernel<2>
+                                                             : attn_tc_kernel<3>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

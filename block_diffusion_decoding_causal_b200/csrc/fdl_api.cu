@@ -482,7 +482,8 @@ int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
     rc = lm_rows(hidden, &rows);
     if (rc != FDL_OK) return rc;
     LmArgs a = lm_fused(rows);
-    const size_t attn_smem = attn_tc_smem_for(c.q_len, c.n_q_heads / c.n_kv_heads, true);
+    const size_t attn_smem =
+        attn_tc_smem_for(c.q_len, c.n_q_heads / c.n_kv_heads, c.batch, true);
     if (lmhead_tc_shared_ok(a, attn_smem)) {
       rc = run_lmhead(a, c, s, attn_smem, c.shift != 0);
       if (rc != FDL_OK) return rc;

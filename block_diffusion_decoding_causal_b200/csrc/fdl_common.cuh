@@ -277,7 +277,7 @@ cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem
                              bool after_producer = false);
 bool lmhead_tc_shared_ok(const LmArgs& a, size_t beside_smem);
 // Shared memory of one tensor-core attention CTA for these shapes.
-size_t attn_tc_smem_for(int q_len, int group, bool beside);
+size_t attn_tc_smem_for(int q_len, int group, int B, bool beside);
 cudaError_t launch_commit(const float* conf, const int32_t* tok,
                           int32_t* block_tokens, uint8_t* committed,
                           int32_t* n_committed, int32_t* n_masked_left, int B,
