@@ -5,6 +5,8 @@
 #include <cstring>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "fdl_common.cuh"
 #include "fdl_plan.h"
 
@@ -200,6 +202,13 @@ int run_lmhead_passes(const LmArgs& a, const fdl_step_cfg& c, const Plan& p, cud
   return FDL_OK;
 }
 
+// An NVTX range around an entry point (visible to profilers; no cost when
+// none is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 }  // namespace
 
 // Error reporting for entry points defined in other files.
@@ -269,6 +278,7 @@ int fdl_block_attn(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
                    const void* v_pre, const int32_t* len_pre, const void* k_blk,
                    const void* v_blk, void* out, void* ws, size_t ws_bytes,
                    void* stream) {
+  NvtxRange nvtx_range("fdl_block_attn");
   return attn_common(cfg, false, q, k_pre, v_pre, len_pre, k_blk, v_blk, nullptr,
                      nullptr, nullptr, out, ws, ws_bytes, stream);
 }
@@ -278,6 +288,7 @@ int fdl_dualcache_attn(const fdl_step_cfg* cfg, const void* q, const void* k_pre
                        const void* k_blk, const void* v_blk, const void* k_suf,
                        const void* v_suf, const int32_t* len_suf, void* out,
                        void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("fdl_dualcache_attn");
   return attn_common(cfg, true, q, k_pre, v_pre, len_pre, k_blk, v_blk, k_suf,
                      v_suf, len_suf, out, ws, ws_bytes, stream);
 }
@@ -286,6 +297,7 @@ int fdl_prefixcache_attn(const fdl_step_cfg* cfg, const void* q, const void* k_p
                          const void* v_pre, const int32_t* len_pre, const void* k_fresh,
                          const void* v_fresh, void* out, void* ws, size_t ws_bytes,
                          void* stream) {
+  NvtxRange nvtx_range("fdl_prefixcache_attn");
   if (cfg != nullptr && (cfg->q_off != 0 || cfg->q_len != cfg->block_size))
     return fail(FDL_ERR_INVALID_ARG,
                 "PrefixCache queries are all recomputed rows: need q_off = 0 and "
@@ -300,6 +312,7 @@ int fdl_lmhead_confidence(const fdl_step_cfg* cfg, const void* rows,
                           const void* w_lm, const uint8_t* row_active,
                           float* conf, int32_t* tok, void* ws, size_t ws_bytes,
                           void* stream) {
+  NvtxRange nvtx_range("fdl_lmhead_confidence");
   Plan p;
   std::string why;
   if (!make_plan(cfg, &p, &why)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
@@ -320,6 +333,7 @@ int fdl_threshold_commit(const fdl_step_cfg* cfg, const float* conf,
                          const int32_t* tok, int32_t* block_tokens,
                          uint8_t* committed, int32_t* n_committed,
                          int32_t* n_masked_left, void* stream) {
+  NvtxRange nvtx_range("fdl_threshold_commit");
   Plan p;
   std::string why;
   if (!make_plan(cfg, &p, &why)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
@@ -340,6 +354,7 @@ int fdl_threshold_commit(const fdl_step_cfg* cfg, const float* conf,
 int fdl_select_commit(const fdl_step_cfg* cfg, int policy, float param, const float* conf,
                       const int32_t* tok, int32_t* block_tokens, uint8_t* committed,
                       int32_t* n_committed, int32_t* n_masked_left, void* stream) {
+  NvtxRange nvtx_range("fdl_select_commit");
   Plan p;
   std::string why;
   if (!make_plan(cfg, &p, &why)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
@@ -368,6 +383,7 @@ int fdl_select_commit(const fdl_step_cfg* cfg, int policy, float param, const fl
 int fdl_unit_status(const fdl_step_cfg* cfg, const int32_t* n_masked_left,
                     int32_t* any_masked, int32_t* step_count,
                     unsigned long long while_handle, void* stream) {
+  NvtxRange nvtx_range("fdl_unit_status");
   Plan p;
   std::string why;
   if (!make_plan(cfg, &p, &why)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
@@ -382,6 +398,7 @@ int fdl_unit_status(const fdl_step_cfg* cfg, const int32_t* n_masked_left,
 
 int fdl_append_block(const fdl_step_cfg* cfg, const void* k_blk, const void* v_blk, void* k_pre,
                      void* v_pre, int32_t* len_pre, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("fdl_append_block");
   Plan p;
   std::string why;
   if (!make_plan(cfg, &p, &why, false)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
@@ -410,6 +427,7 @@ int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
                      void* attn_out, float* conf, int32_t* tok, uint8_t* committed,
                      int32_t* n_committed, int32_t* n_masked_left, void* ws,
                      size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("fdl_denoise_step");
   Plan p;
   std::string why;
   if (!make_plan(cfg, &p, &why)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());

@@ -27,7 +27,8 @@ SYMBOLS = ["fdl_version", "fdl_last_error", "fdl_workspace_size",
            "fdl_reset_workspace", "fdl_block_attn", "fdl_dualcache_attn",
            "fdl_lmhead_confidence", "fdl_threshold_commit", "fdl_denoise_step",
            "fdl_get_status", "fdl_lmhead_confidence_noalloc", "fdl_select_commit",
-           "fdl_unit_status", "fdl_append_block", "fdl_prefixcache_attn"]
+           "fdl_unit_status", "fdl_append_block", "fdl_prefixcache_attn",
+           "fdl_check_wait_timeout"]
 
 
 class StepCfg(ctypes.Structure):
@@ -81,12 +82,14 @@ def lib() -> ctypes.CDLL:
         L.fdl_unit_status.argtypes = [ctypes.POINTER(StepCfg), _P, _P, _P, ctypes.c_ulonglong, _P]
         L.fdl_prefixcache_attn.argtypes = [ctypes.POINTER(StepCfg)] + [_P] * 7 + [
             _P, ctypes.c_size_t, _P]
+        L.fdl_check_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_longlong, _P]
         L.fdl_append_block.argtypes = [ctypes.POINTER(StepCfg)] + [_P] * 5 + [_P, ctypes.c_size_t, _P]
         for name in ["fdl_reset_workspace", "fdl_block_attn", "fdl_dualcache_attn",
                      "fdl_lmhead_confidence", "fdl_threshold_commit",
                      "fdl_denoise_step", "fdl_get_status",
                      "fdl_lmhead_confidence_noalloc", "fdl_select_commit",
-                     "fdl_unit_status", "fdl_append_block", "fdl_prefixcache_attn"]:
+                     "fdl_unit_status", "fdl_append_block", "fdl_prefixcache_attn",
+                     "fdl_check_wait_timeout"]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -209,6 +212,11 @@ def denoise_step(cfg, q, k_pre, v_pre, len_pre, k_blk, v_blk, k_suf, v_suf, len_
         ptr(w_lm), ptr(block_tokens), ptr(attn_out), ptr(conf), ptr(tok),
         ptr(committed), ptr(n_committed), ptr(n_masked_left), ptr(ws), ws.numel(),
         stream_ptr(stream)))
+
+
+def check_wait_timeout(ws, limit_cycles=1_000_000, stream=None):
+    _check(lib().fdl_check_wait_timeout(ptr(ws), ws.numel(), int(limit_cycles),
+                                        stream_ptr(stream)))
 
 
 def get_status(ws, stream=None) -> int:

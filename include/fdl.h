@@ -312,6 +312,18 @@ int fdl_append_block(const fdl_step_cfg* cfg, const void* k_blk,
  * set, FDL_OK otherwise. */
 int fdl_get_status(void* ws, void* stream, uint32_t* status);
 
+/*
+ * Failure-detection self-check (no counterpart on the pages; a diagnostic of
+ * this library).  Launches one CTA that waits on an mbarrier nothing ever
+ * arrives on, with the same bounded wait every kernel uses but a bound of
+ * limit_cycles SM clocks (1e3 .. 2e9; 1e6 is about half a millisecond), so
+ * the wait runs out: the kernel sets FDL_DEV_TIMEOUT in the workspace status
+ * word and returns.  fdl_get_status then reports FDL_ERR_DEVICE_STATUS with
+ * that bit, and the CUDA context stays usable.  ws: at least 256 bytes,
+ * 256-byte aligned (only its control words are touched).
+ */
+int fdl_check_wait_timeout(void* ws, size_t ws_bytes, long long limit_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -206,3 +206,10 @@ def test_step_rows_beyond_one_lm_pass_are_accepted_up_to_4096(L):
     nl = ctypes.c_void_p(16)
     rc = L.fdl_threshold_commit(ctypes.byref(too_many), nl, nl, nl, nl, nl, nl, None)
     assert rc == fdl.ERR_INVALID_ARG and "4096" in fdl.last_error()
+
+
+def test_wait_timeout_check_rejects_bad_arguments(L):
+    rc = L.fdl_check_wait_timeout(None, 256, 1000000, None)
+    assert rc == fdl.ERR_WORKSPACE
+    rc = L.fdl_check_wait_timeout(ctypes.c_void_p(256), 256, 10, None)
+    assert rc == fdl.ERR_INVALID_ARG and "limit_cycles" in fdl.last_error()

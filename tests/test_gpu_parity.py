@@ -399,3 +399,18 @@ def test_fused_step_with_two_lm_passes():
     committing its own sequences) against the oracle, bit-exact commits."""
     case, ref, _ = cases.parity_case("large_batch", 0, cfg=LARGE_BATCH)
     gh.compare_step(case, gh.run_denoise_step(case), ref)
+
+
+# ------------------------------------------------------ failure detection
+
+def test_bounded_wait_times_out_into_the_status_word():
+    """A wait that nothing satisfies runs out after its bound: the timeout
+    bit lands in the workspace status word, the context stays usable, and
+    the next step through the same workspace is correct."""
+    cfg = fdl.make_cfg(synth.CONFIGS["tiny"] | dict(q_off=0))
+    ws = fdl.workspace(cfg)
+    fdl.check_wait_timeout(ws, limit_cycles=1_000_000)
+    assert fdl.get_status(ws) == fdl.DEV_TIMEOUT
+    assert fdl.get_status(ws) == 0                     # read and cleared
+    case, ref, _ = cases.parity_case("tiny", 0)
+    gh.compare_step(case, gh.run_denoise_step(case, ws=ws), ref)
