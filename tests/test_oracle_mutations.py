@@ -93,3 +93,46 @@ def test_shift_in_wrong_direction_is_caught(monkeypatch):
         return rows
     monkeypatch.setattr(step, "shifted_rows", wrong)
     _expect_pin_failure(pins.test_token_shift_rows)
+
+
+def test_prefixcache_with_block_causal_mask_is_caught(monkeypatch):
+    """PrefixCache computed as if the recomputed rows were one block under a
+    causal-across-blocks mask (suffix rows hidden from earlier rows)."""
+    def causal(q, k_pre, v_pre, len_pre, k_fresh, v_fresh):
+        B, n, Hq, d = q.shape
+        group = Hq // k_pre.shape[1]
+        out = np.empty((B, n, Hq, d))
+        for b in range(B):
+            Lp = int(len_pre[b])
+            vis = np.ones((n, Lp + n), bool)
+            vis[:, Lp:] = np.tril(np.ones((n, n), bool))
+            for h in range(Hq):
+                K = np.concatenate([k_pre[b, h // group, :Lp], k_fresh[b, h // group]])
+                V = np.concatenate([v_pre[b, h // group, :Lp], v_fresh[b, h // group]])
+                out[b, :, h] = step.masked_attention(q[b, :, h], K, V, vis)
+        return out
+    monkeypatch.setattr(step, "prefixcache_attention", causal)
+    _expect_pin_failure(pins.test_prefixcache_attention_matches_torch_sdpa_with_gqa)
+
+
+def test_factor_rule_with_n_instead_of_n_plus_1_is_caught(monkeypatch):
+    """Eq. 13 with the group-size factor off by one: n (1 - c_(n)) < f."""
+    from oracle import theory
+
+    def off_by_one(masked_positions, conf_of, f):
+        order = sorted(masked_positions, key=lambda p: (-conf_of(p), p))
+        best = 0
+        for n in range(1, len(order) + 1):
+            if n * (1.0 - conf_of(order[n - 1])) < f:
+                best = n
+        return order[:best] if best else order[:1]
+    monkeypatch.setattr(theory, "factor_select", off_by_one)
+    _expect_pin_failure(pins.test_factor_rule_eq13)
+
+
+def test_budget_rule_without_the_max_term_is_caught(monkeypatch):
+    """Eq. 9 with the max_j eps_j term dropped (sum only)."""
+    from oracle import theory
+    monkeypatch.setattr(theory, "heterogeneous_budget_ok",
+                        lambda eps: sum(float(e) for e in eps) < 1.0)
+    _expect_pin_failure(pins.test_budget_rule_eq9_selection)
