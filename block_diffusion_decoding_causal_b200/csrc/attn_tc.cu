@@ -40,13 +40,11 @@ namespace {
 using namespace sm100;
 
 constexpr int kCh = 64;                  // keys per chunk
-constexpr int kQRegion = 128 * 128;      // 128 rows x 64 bf16 (16 KB)
 // Rows of an item at most 64: the Q halves (d 0-63, 64-127) sit only the
 // rows (rounded to 8) apart, 16 KB at most for both.  The MMA still reads 128
 // rows per half; the rows past the item then fall on the other half or the
 // K/V stage that follows, which only feeds S rows no softmax thread reads
 // (rows of an M = 128 tile never mix).
-constexpr int kQRegionMaxCompact = 64 * 128;
 // Bytes between the two d-halves of the Q buffer: the item's rows rounded up
 // to the 8-row swizzle atom when they are at most 64, else 128 rows.
 __host__ __device__ constexpr int q_region_for(int rows) {
@@ -93,7 +91,6 @@ struct Smem {
   uint64_t o_full[2], o_empty[2];
   uint64_t drain;
   uint32_t tmem;
-  int flag;
   // followed by the sequence table: cb [B + 1] (first global chunk of
   // sequence b), nc [B] (chunks per item), lp [B], ls [B] (lengths)
 };
