@@ -108,7 +108,7 @@ namespace fdl {
 namespace {
 
 // Loop control of the sub-block iteration (technical review Algorithm 1:
-// "while the current block contains masks"): any[0] = 1 if any sequence still
+// steps repeat while masked positions remain): any[0] = 1 if any sequence still
 // has a masked position in the unit; optionally sets a CUDA-graph conditional
 // (the WHILE node around one denoising step) and counts steps.
 // The WHILE condition also stops after `limit` steps (the unit length: every

@@ -277,7 +277,7 @@ int fdl_lmhead_confidence_noalloc(const fdl_step_cfg* cfg, const void* rows,
 
 /*
  * Loop control of the block decode (technical review Algorithm 1: repeat
- * steps "while the current block contains masks"; "Fast-dLLM v2" Level 2).
+ * steps for as long as masked positions remain in the block; "Fast-dLLM v2" Level 2).
  * Reads n_masked_left [B] (device) after a step and, each only if given:
  *   any_masked (device int32): 1 if any sequence still has a masked unit
  *     position, else 0;

@@ -240,7 +240,7 @@ def threshold_commit(block_tokens, conf, tok, q_off: int, q_len: int,
     """Commit step over the active unit [q_off, q_off + q_len) of each block.
 
     Candidates are the unit's positions still holding the mask token (v2
-    digest Level 1: positions are "set to [MASK]").  The sub-block is the
+    digest Level 1: undecoded positions hold the mask token).  The sub-block is the
     thresholding unit (v2 digest, "Sub-block size as a decoding granularity
     knob").  conf / tok are [B, q_len], indexed by unit position.
     Returns new block tokens, the committed bitmap over the whole block,
