@@ -326,6 +326,12 @@ def main():
         blk = block_decode_leg(torch, fdl, c, sets[0], w, stream, world)
     except Exception as e:  # reported in the JSON line; the headline legs stand
         blk = {"error": f"{type(e).__name__}: {e}"}
+    # Every rank takes part in these reductions, whatever its leg did.
+    for k in ("graph_us_per_block", "host_loop_us_per_block", "graph_us_per_step"):
+        blk[k] = max_over_ranks(float(blk.get(k, float("nan"))), world)
+    if "graph_us_per_block" in blk and blk["graph_us_per_block"] == blk["graph_us_per_block"]:
+        blk["positions_per_s_graph"] = c["batch"] * c["block_size"] / (
+            blk["graph_us_per_block"] * 1e-6)
     lm_big = large_batch_lm_leg(torch, fdl, synth, stream, timed, world, args.steps, peaks)
 
     # End to end through the public API: per step, pinned host inputs copied
@@ -514,8 +520,8 @@ def block_decode_leg(torch, fdl, c, x, w, stream, world, blocks: int = 5) -> dic
         append(stream)
     ev[3].record(stream)
     stream.synchronize()
-    t_graph = max_over_ranks(ev[0].elapsed_time(ev[1]) / blocks, world)
-    t_host = max_over_ranks(ev[2].elapsed_time(ev[3]) / blocks, world)
+    t_graph = ev[0].elapsed_time(ev[1]) / blocks  # this rank's; reduced by the caller
+    t_host = ev[2].elapsed_time(ev[3]) / blocks
     n_steps = sum(steps_graph)
     assert fdl.get_status(ws, stream) == 0
     return {"workload": f"one block of {D} positions, {units} sub-blocks of {q_len}, batch {B}",
