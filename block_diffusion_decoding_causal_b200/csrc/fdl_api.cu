@@ -113,6 +113,7 @@ LmArgs lm_args(const fdl_step_cfg& c, const Plan& p, const void* rows,
   const bool tc = c.dtype == FDL_BF16;
   a.n_cta = tc ? p.lm_tc_cta : p.lm_cta;
   a.rows_per_cta = tc ? p.lm_tc_rows_per_cta : p.lm_rows_per_cta;
+  a.w_packed = c.w_layout == FDL_W_PACKED;
   a.commit = 0;
   a.B = c.batch;
   a.D = c.block_size;
@@ -161,6 +162,8 @@ int run_attention(const fdl_step_cfg& c, const Plan& p, bool dual, const void* q
 int check_lmhead_supported(const fdl_step_cfg& c) {
   if (c.dtype == FDL_BF16 && c.hidden % 64 != 0)
     return fail(FDL_ERR_UNSUPPORTED, "bf16 LM head needs hidden %% 64 == 0 (got %d)", c.hidden);
+  if (c.w_layout == FDL_W_PACKED && c.dtype != FDL_BF16)
+    return fail(FDL_ERR_UNSUPPORTED, "the tiled weight layout is bf16 only");
   return FDL_OK;
 }
 
@@ -327,6 +330,34 @@ int fdl_lmhead_confidence(const fdl_step_cfg* cfg, const void* rows,
   LmArgs a = lm_args(*cfg, p, rows, w_lm, row_active, conf, tok, ws);
   rc = run_lmhead_passes(a, *cfg, p, (cudaStream_t)stream);
   return rc != FDL_OK ? rc : ok();
+}
+
+int fdl_lmhead_pack_weight(const fdl_step_cfg* cfg, const void* w_lm, void* w_packed,
+                           void* stream) {
+  NvtxRange nvtx_range("fdl_lmhead_pack_weight");
+  if (cfg == nullptr) return fail(FDL_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->dtype != FDL_BF16)
+    return fail(FDL_ERR_UNSUPPORTED, "the tiled weight layout is bf16 only");
+  if (cfg->vocab < 1 || cfg->hidden < 64)
+    return fail(FDL_ERR_INVALID_ARG, "need vocab >= 1 and hidden >= 64 (got %d, %d)", cfg->vocab,
+                cfg->hidden);
+  if (cfg->hidden % 64 != 0)
+    return fail(FDL_ERR_UNSUPPORTED, "the tiled weight layout needs hidden %% 64 == 0 (got %d)",
+                cfg->hidden);
+  if ((long)cfg->vocab * (cfg->hidden / 64) > 0x7fffffffL)
+    return fail(FDL_ERR_INVALID_ARG, "vocab * hidden / 64 exceeds 2^31 - 1");
+  FDL_CHECK_PTR(w_lm);
+  FDL_CHECK_PTR(w_packed);
+  const uintptr_t src = reinterpret_cast<uintptr_t>(w_lm);
+  const uintptr_t dst = reinterpret_cast<uintptr_t>(w_packed);
+  const uintptr_t bytes = (uintptr_t)cfg->vocab * (uintptr_t)cfg->hidden * 2u;
+  if (src < dst + bytes && dst < src + bytes)
+    return fail(FDL_ERR_INVALID_ARG, "w_lm and w_packed overlap");
+  const cudaError_t e =
+      launch_pack_weight(w_lm, w_packed, cfg->vocab, cfg->hidden,
+                         (int)lm_tc_rows_per_cta(cfg->vocab), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "weight pack launch");
+  return ok();
 }
 
 int fdl_threshold_commit(const fdl_step_cfg* cfg, const float* conf,

@@ -111,6 +111,7 @@ struct LmArgs {
   int R, H, V;
   int n_cta;
   int rows_per_cta;          // vocab rows per CTA (multiple of 16)
+  int w_packed;              // w in the tiled layout of fdl_lmhead_pack_weight
   // fused commit (when commit != 0)
   int commit;
   int32_t* block_tokens;
@@ -276,6 +277,10 @@ cudaError_t launch_lmhead_simt(const LmArgs& a, fdl_dtype dt, cudaStream_t s);
 cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem = 0,
                              bool after_producer = false);
 bool lmhead_tc_shared_ok(const LmArgs& a, size_t beside_smem);
+// Rewrites the bf16 weight [V, H] into the tiled layout the LM head reads
+// when LmArgs::w_packed is set (see lmhead_tc.cu).
+cudaError_t launch_pack_weight(const void* w, void* out, int V, int H, int rows_per_cta,
+                               cudaStream_t s);
 // Shared memory of one tensor-core attention CTA for these shapes.
 size_t attn_tc_smem_for(int q_len, int group, int B, bool beside);
 cudaError_t launch_commit(const float* conf, const int32_t* tok,

@@ -43,6 +43,14 @@ struct Plan {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Vocabulary rows per CTA of the tensor-core LM head: V over one CTA per SM,
+// rounded up to 16 rows.  Depends on V alone, so it also fixes the tiled
+// weight layout (FDL_W_PACKED) whatever the number of rows of a call.
+inline long lm_tc_rows_per_cta(long vocab) {
+  long per = (vocab + kPlanCTAs - 1) / kPlanCTAs;
+  return (per + 15) / 16 * 16;
+}
+
 // Split the (b, kv head, row tile) key sequences so that about two CTAs per
 // SM are in flight.
 inline AttnSplit plan_split(long keys_cap, long items) {
@@ -65,6 +73,9 @@ inline AttnSplit plan_split(long keys_cap, long items) {
 inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why, bool step = true) {
   if (c == nullptr) { *why = "cfg is NULL"; return false; }
   if (c->dtype != FDL_F32 && c->dtype != FDL_BF16) { *why = "dtype must be FDL_F32 or FDL_BF16"; return false; }
+  if (c->w_layout != FDL_W_ROW_MAJOR && c->w_layout != FDL_W_PACKED) {
+    *why = "w_layout must be FDL_W_ROW_MAJOR or FDL_W_PACKED"; return false;
+  }
   if (c->batch < 1) { *why = "batch must be >= 1"; return false; }
   if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads != 0) {
     *why = "n_q_heads must be a positive multiple of n_kv_heads"; return false;
@@ -122,8 +133,7 @@ inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why, bool ste
   per = (per + 15) / 16 * 16;
   p->lm_rows_per_cta = (int)per;
   p->lm_cta = (int)(((long)c->vocab + per - 1) / per);
-  long per_tc = ((long)c->vocab + kPlanCTAs - 1) / kPlanCTAs;
-  per_tc = (per_tc + 15) / 16 * 16;
+  const long per_tc = lm_tc_rows_per_cta(c->vocab);
   p->lm_tc_rows_per_cta = (int)per_tc;
   p->lm_tc_cta = (int)(((long)c->vocab + per_tc - 1) / per_tc);
 

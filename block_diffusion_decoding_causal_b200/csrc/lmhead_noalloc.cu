@@ -100,6 +100,8 @@ extern "C" int fdl_lmhead_confidence_noalloc(const fdl_step_cfg* cfg, const void
   }
   if (cfg->dtype == FDL_BF16 && cfg->hidden % 64 != 0)
     return record_error(FDL_ERR_UNSUPPORTED, "bf16 LM head needs hidden % 64 == 0");
+  if (cfg->w_layout == FDL_W_PACKED && cfg->dtype != FDL_BF16)
+    return record_error(FDL_ERR_UNSUPPORTED, "the tiled weight layout is bf16 only");
   const int rc = lmhead_static_check(p, *cfg, &why);
   if (rc != FDL_OK) return record_error(rc, why);
   LmArgs a;
@@ -118,6 +120,7 @@ extern "C" int fdl_lmhead_confidence_noalloc(const fdl_step_cfg* cfg, const void
   a.V = cfg->vocab;
   a.n_cta = tc ? p.lm_tc_cta : p.lm_cta;
   a.rows_per_cta = tc ? p.lm_tc_rows_per_cta : p.lm_rows_per_cta;
+  a.w_packed = cfg->w_layout == FDL_W_PACKED;
   a.B = cfg->batch;
   a.D = cfg->block_size;
   a.q_off = cfg->q_off;

@@ -10,7 +10,9 @@
 // vocabulary range of ~V/148 rows and streams it once:
 //   warp 0   TMA producer: W tiles [128 x 64*KSUB] (KSUB boxes of 128-byte
 //            swizzled rows, so each weight row is read 512 contiguous bytes at
-//            a time) through an A ring, X chunks [N x 64*KSUB] through a B ring;
+//            a time; with the tiled weight layout each box is one contiguous
+//            16 KB block) through an A ring, X chunks [N x 64*KSUB] through a
+//            B ring;
 //   warp 1   MMA issuer: tcgen05.mma kind::f16, accumulators in TMEM; tiles
 //            are processed in groups of G, K-outer inside a group so each X
 //            chunk is reused by G tiles; two TMEM buffers let the epilogue
@@ -103,6 +105,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
   const int G = tp.group;
   const int n_groups = (n_tiles + G - 1) / G;
   const int KC = a.H / (kKChunk * KSUB);
+  const int KCT = a.H / kKChunk;  // 64-wide chunks of one weight row
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SA; ++i) {
@@ -171,17 +174,33 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
             if (rows == kTileM) {
               mbar_arrive_expect_tx(&full_a[slot_a], SA_BYTES);
 #pragma unroll
-              for (int u = 0; u < KSUB; ++u)
-                tma_load_2d_hint(dst + u * kStageA, &tm_w_full, (kc * KSUB + u) * kKChunk,
-                                 row0, &full_a[slot_a], pol_w);
+              for (int u = 0; u < KSUB; ++u) {
+                const int kk = kc * KSUB + u;
+                if (a.w_packed)
+                  tma_load_2d_hint(dst + u * kStageA, &tm_w_full, 0, row0 * KCT + kk * kTileM,
+                                   &full_a[slot_a], pol_w);
+                else
+                  tma_load_2d_hint(dst + u * kStageA, &tm_w_full, kk * kKChunk, row0,
+                                   &full_a[slot_a], pol_w);
+              }
             } else {
               const int nbox = (rows + kBoxPart - 1) / kBoxPart;
               mbar_arrive_expect_tx(&full_a[slot_a], KSUB * nbox * kBoxPart * 128);
-              for (int u = 0; u < KSUB; ++u)
-                for (int j = 0; j < nbox; ++j)
-                  tma_load_2d_hint(dst + u * kStageA + j * kBoxPart * 128, &tm_w_part,
-                                   (kc * KSUB + u) * kKChunk, row0 + j * kBoxPart,
-                                   &full_a[slot_a], pol_w);
+              for (int u = 0; u < KSUB; ++u) {
+                const int kk = kc * KSUB + u;
+                for (int j = 0; j < nbox; ++j) {
+                  // Box rows past the tile's last row read neighbouring
+                  // weight rows (or the zero fill past the end); the
+                  // epilogue masks their logits.
+                  if (a.w_packed)
+                    tma_load_2d_hint(dst + u * kStageA + j * kBoxPart * 128, &tm_w_part, 0,
+                                     row0 * KCT + kk * rows + j * kBoxPart, &full_a[slot_a],
+                                     pol_w);
+                  else
+                    tma_load_2d_hint(dst + u * kStageA + j * kBoxPart * 128, &tm_w_part,
+                                     kk * kKChunk, row0 + j * kBoxPart, &full_a[slot_a], pol_w);
+                }
+              }
             }
             ++ia;
           }
@@ -322,6 +341,29 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tiled weight layout.  The vocabulary is cut into the CTA ranges of the LM
+// head (per rows each) and each range into tiles of up to 128 rows; tile
+// (first row row0, rt rows) occupies rt * KCT consecutive 128-byte rows
+// starting at row0 * KCT, chunk kk's rt rows (columns 64 kk .. 64 kk + 63 of
+// every row of the tile) at row0 * KCT + kk * rt.  A weight row's 128-byte
+// piece (v, kk) thus moves from v * KCT + kk to the row computed here.
+// One thread per 16 bytes; reads are coalesced, writes 128 bytes per eight
+// threads.
+__global__ void pack_weight_kernel(const uint4* __restrict__ w, uint4* __restrict__ out,
+                                   int V, int KCT, int per) {
+  const long n = (long)V * KCT * 8;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n;
+       i += (long)gridDim.x * blockDim.x) {
+    const long seg = i >> 3;
+    const int v = (int)(seg / KCT), kk = (int)(seg % KCT);
+    const int v_lo = v / per * per;
+    const int v_hi = min(V, v_lo + per);
+    const int row0 = v_lo + (v - v_lo) / kTileM * kTileM;
+    const int rt = min(kTileM, v_hi - row0);
+    out[((long)row0 * KCT + (long)kk * rt + (v - row0)) * 8 + (i & 7)] = w[i];
+  }
+}
+
 template <int NCH, int KSUB>
 cudaError_t launch_nch(const CUtensorMap& wf, const CUtensorMap& wp, const CUtensorMap& x,
                        const LmArgs& a, const TcParams& tp, size_t smem, cudaStream_t s,
@@ -440,8 +482,11 @@ cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem
   if (!lmhead_tc_params(a.R, a.H, a.rows_per_cta, beside_smem, &tp, &smem))
     return cudaErrorInvalidValue;
   CUtensorMap wf, wp, x;
-  if (!make_map(&wf, a.w, a.H, a.V, kKChunk, kTileM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
-      !make_map(&wp, a.w, a.H, a.V, kKChunk, kBoxPart, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+  // Row-major: [V][H]; tiled: [V * H / 64][64], one 128-byte row per piece.
+  const uint64_t w_inner = a.w_packed ? kKChunk : a.H;
+  const uint64_t w_outer = a.w_packed ? (uint64_t)a.V * (a.H / kKChunk) : a.V;
+  if (!make_map(&wf, a.w, w_inner, w_outer, kKChunk, kTileM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+      !make_map(&wp, a.w, w_inner, w_outer, kKChunk, kBoxPart, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
       !make_map(&x, a.rows, a.H, a.R, kKChunk, tp.npad, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
     return cudaErrorInvalidValue;
 #define FDL_LM_CASE(NCH)                                                   \
@@ -457,6 +502,14 @@ cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem
   }
 #undef FDL_LM_CASE
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_pack_weight(const void* w, void* out, int V, int H, int rows_per_cta,
+                               cudaStream_t s) {
+  pack_weight_kernel<<<4 * kPlanSMs, 256, 0, s>>>(static_cast<const uint4*>(w),
+                                                  static_cast<uint4*>(out), V, H / kKChunk,
+                                                  rows_per_cta);
+  return cudaGetLastError();
 }
 
 }  // namespace fdl

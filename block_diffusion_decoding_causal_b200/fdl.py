@@ -21,6 +21,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_STATUS
     0, -1, -2, -3, -4, -5)
 DEV_BAD_PREFIX_LEN, DEV_BAD_SUFFIX_LEN, DEV_TIMEOUT = 1, 2, 4
 SELECT_THRESHOLD, SELECT_FACTOR, SELECT_BUDGET = 0, 1, 2
+W_ROW_MAJOR, W_PACKED = 0, 1
 
 # Every symbol include/fdl.h declares.
 SYMBOLS = ["fdl_version", "fdl_last_error", "fdl_workspace_size",
@@ -28,7 +29,7 @@ SYMBOLS = ["fdl_version", "fdl_last_error", "fdl_workspace_size",
            "fdl_lmhead_confidence", "fdl_threshold_commit", "fdl_denoise_step",
            "fdl_get_status", "fdl_lmhead_confidence_noalloc", "fdl_select_commit",
            "fdl_unit_status", "fdl_append_block", "fdl_prefixcache_attn",
-           "fdl_check_wait_timeout"]
+           "fdl_check_wait_timeout", "fdl_lmhead_pack_weight"]
 
 
 class StepCfg(ctypes.Structure):
@@ -40,7 +41,7 @@ class StepCfg(ctypes.Structure):
                 ("cap_suffix", ctypes.c_int32), ("hidden", ctypes.c_int32),
                 ("vocab", ctypes.c_int32), ("mask_id", ctypes.c_int32),
                 ("shift", ctypes.c_int32), ("tau", ctypes.c_float),
-                ("dtype", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("w_layout", ctypes.c_int32)]
 
 
 class FdlError(RuntimeError):
@@ -83,13 +84,14 @@ def lib() -> ctypes.CDLL:
         L.fdl_prefixcache_attn.argtypes = [ctypes.POINTER(StepCfg)] + [_P] * 7 + [
             _P, ctypes.c_size_t, _P]
         L.fdl_check_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_longlong, _P]
+        L.fdl_lmhead_pack_weight.argtypes = [ctypes.POINTER(StepCfg), _P, _P, _P]
         L.fdl_append_block.argtypes = [ctypes.POINTER(StepCfg)] + [_P] * 5 + [_P, ctypes.c_size_t, _P]
         for name in ["fdl_reset_workspace", "fdl_block_attn", "fdl_dualcache_attn",
                      "fdl_lmhead_confidence", "fdl_threshold_commit",
                      "fdl_denoise_step", "fdl_get_status",
                      "fdl_lmhead_confidence_noalloc", "fdl_select_commit",
                      "fdl_unit_status", "fdl_append_block", "fdl_prefixcache_attn",
-                     "fdl_check_wait_timeout"]:
+                     "fdl_check_wait_timeout", "fdl_lmhead_pack_weight"]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -112,7 +114,8 @@ def make_cfg(c: dict) -> StepCfg:
                    cap_prefix=c["cap_prefix"], cap_suffix=c.get("cap_suffix", 0),
                    hidden=c["hidden"], vocab=c["vocab"], mask_id=c["mask_id"],
                    shift=c["shift"], tau=c["tau"],
-                   dtype=BF16 if c["dtype"] == "bf16" else F32)
+                   dtype=BF16 if c["dtype"] == "bf16" else F32,
+                   w_layout=c.get("w_layout", W_ROW_MAJOR))
 
 
 def ptr(t: Optional[torch.Tensor]):
@@ -212,6 +215,11 @@ def denoise_step(cfg, q, k_pre, v_pre, len_pre, k_blk, v_blk, k_suf, v_suf, len_
         ptr(w_lm), ptr(block_tokens), ptr(attn_out), ptr(conf), ptr(tok),
         ptr(committed), ptr(n_committed), ptr(n_masked_left), ptr(ws), ws.numel(),
         stream_ptr(stream)))
+
+
+def lmhead_pack_weight(cfg, w_lm, w_packed, stream=None):
+    _check(lib().fdl_lmhead_pack_weight(ctypes.byref(cfg), ptr(w_lm), ptr(w_packed),
+                                        stream_ptr(stream)))
 
 
 def check_wait_timeout(ws, limit_cycles=1_000_000, stream=None):

@@ -25,6 +25,8 @@ def main() -> int:
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--prefix", type=int, default=None)
     ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--packed", action="store_true",
+                    help="lmhead / step: the LM-head weight in the tiled layout")
     args = ap.parse_args()
 
     c = dict(synth.CONFIGS[args.workload])
@@ -59,6 +61,11 @@ def main() -> int:
     if args.kernel in ("lmhead", "step"):
         w = (torch.randn((V, H), generator=g, device="cuda") * (c["w_scale"] / H ** 0.5)).to(dt)
         rows = rn(B * q_len, H)
+        if args.packed:
+            w_rm, w = w, torch.empty_like(w)
+            fdl.lmhead_pack_weight(cfg, w_rm, w)
+            del w_rm
+            cfg.w_layout = fdl.W_PACKED
     for _ in range(args.launches):
         if args.kernel == "lmhead":
             fdl.lmhead_confidence(cfg, rows, w, None, conf, tok, ws)

@@ -107,7 +107,13 @@ typedef struct {
                           p - 1 (v2 token shift); 0: from p itself             */
   float tau;           /* commit iff confidence >= tau                         */
   int32_t dtype;       /* fdl_dtype of every floating tensor                   */
+  int32_t w_layout;    /* FDL_W_ROW_MAJOR, or FDL_W_PACKED: w_lm as rewritten by
+                          fdl_lmhead_pack_weight (bf16 only)                   */
 } fdl_step_cfg;
+
+/* Layouts of the LM-head weight (fdl_step_cfg.w_layout). */
+#define FDL_W_ROW_MAJOR 0  /* w_lm [V, H] row-major                            */
+#define FDL_W_PACKED 1     /* the tiled layout of fdl_lmhead_pack_weight         */
 
 /* Library version (FDL_VERSION) and a thread-local description of the last
  * error returned on this thread ("" if none). */
@@ -191,6 +197,23 @@ int fdl_lmhead_confidence(const fdl_step_cfg* cfg, const void* rows,
                           const void* w_lm, const uint8_t* row_active,
                           float* conf, int32_t* tok, void* ws, size_t ws_bytes,
                           void* stream);
+
+/*
+ * LM-head weight in its tiled form (no counterpart on the pages: a load-time
+ * layout choice of this library, like a GEMM library's pre-transformed
+ * weights).  Rewrites w_lm [V, H] row-major (bf16) into w_packed, the same
+ * number of bytes (2 V H), so that every block the LM head streams — 128
+ * vocabulary rows x 64 hidden columns of one CTA's range — is contiguous in
+ * memory instead of 128 strided 128-byte pieces.  Call it once when the
+ * weight is loaded; then pass w_packed as w_lm with cfg->w_layout =
+ * FDL_W_PACKED to fdl_lmhead_confidence, fdl_lmhead_confidence_noalloc and
+ * fdl_denoise_step.  The results are bit-identical to the row-major layout.
+ * Only the vocabulary size and hidden width of cfg matter (the split of the
+ * vocabulary over the CTAs is fixed by V); w_lm and w_packed must not
+ * overlap.  bf16 and hidden % 64 == 0 only (else FDL_ERR_UNSUPPORTED).
+ */
+int fdl_lmhead_pack_weight(const fdl_step_cfg* cfg, const void* w_lm, void* w_packed,
+                           void* stream);
 
 /*
  * Threshold commit (stage b, second half; technical review Algorithm 2

@@ -32,16 +32,22 @@ def outputs(case):
         n_masked_left=torch.empty((B,), dtype=torch.int32, device="cuda"))
 
 
-def run_denoise_step(case, ws=None, d=None, keep_attn=True):
-    """fdl_denoise_step on a case; returns CPU copies of every output."""
+def run_denoise_step(case, ws=None, d=None, keep_attn=True, packed=False):
+    """fdl_denoise_step on a case; returns CPU copies of every output.
+    packed: the LM-head weight is first rewritten into the tiled layout."""
     cfg = fdl.make_cfg(case.cfg)
     d = device_case(case) if d is None else d
     o = outputs(case)
     ws = fdl.workspace(cfg) if ws is None else ws
     bt = d["block_tokens"].clone()
+    w_lm = d["w_lm"]
+    if packed:
+        w_lm = torch.empty_like(d["w_lm"])
+        fdl.lmhead_pack_weight(cfg, d["w_lm"], w_lm)
+        cfg.w_layout = fdl.W_PACKED
     fdl.denoise_step(cfg, d["q"], d["k_pre"], d["v_pre"], d["len_pre"], d["k_blk"],
                      d["v_blk"], d["k_suf"], d["v_suf"], d["len_suf"], d["hidden"],
-                     d["h_prev"], d["w_lm"], bt, o["attn"] if keep_attn else None,
+                     d["h_prev"], w_lm, bt, o["attn"] if keep_attn else None,
                      o["conf"], o["tok"], o["committed"], o["n_committed"],
                      o["n_masked_left"], ws)
     torch.cuda.synchronize()

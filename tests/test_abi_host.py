@@ -213,3 +213,29 @@ def test_wait_timeout_check_rejects_bad_arguments(L):
     assert rc == fdl.ERR_WORKSPACE
     rc = L.fdl_check_wait_timeout(ctypes.c_void_p(256), 256, 10, None)
     assert rc == fdl.ERR_INVALID_ARG and "limit_cycles" in fdl.last_error()
+
+
+def test_weight_layout_rules(L):
+    bad = _cfg()
+    bad.w_layout = 2
+    assert L.fdl_workspace_size(ctypes.byref(bad)) == 0
+    assert "w_layout" in fdl.last_error()
+    p = _fake(2)
+    assert L.fdl_lmhead_pack_weight(None, *p, None) == fdl.ERR_INVALID_ARG
+    f32 = _cfg(dtype="f32")
+    assert L.fdl_lmhead_pack_weight(ctypes.byref(f32), *p, None) == fdl.ERR_UNSUPPORTED
+    assert L.fdl_lmhead_pack_weight(ctypes.byref(_cfg(hidden=96)), *p, None) == \
+        fdl.ERR_UNSUPPORTED
+    rc = L.fdl_lmhead_pack_weight(ctypes.byref(_cfg()), None, p[1], None)
+    assert rc == fdl.ERR_INVALID_ARG and "NULL" in fdl.last_error()
+    # a 152064 x 3584 bf16 weight spans 1.09 GB: these two ranges overlap
+    rc = L.fdl_lmhead_pack_weight(ctypes.byref(_cfg()), ctypes.c_void_p(0x10000000),
+                                  ctypes.c_void_p(0x20000000), None)
+    assert rc == fdl.ERR_INVALID_ARG and "overlap" in fdl.last_error()
+    # the fp32 LM head has no tiled form
+    f32.w_layout = fdl.W_PACKED
+    q = _fake(4)
+    rc = L.fdl_lmhead_confidence(ctypes.byref(f32), q[0], q[1], None, q[2], q[3], None, 0, None)
+    assert rc == fdl.ERR_UNSUPPORTED and "bf16" in fdl.last_error()
+    rc = L.fdl_lmhead_confidence_noalloc(ctypes.byref(f32), q[0], q[1], None, q[2], q[3], None)
+    assert rc == fdl.ERR_UNSUPPORTED and "bf16" in fdl.last_error()

@@ -401,6 +401,87 @@ def test_fused_step_with_two_lm_passes():
     gh.compare_step(case, gh.run_denoise_step(case), ref)
 
 
+# ----------------------------------------------- tiled LM-head weight layout
+
+def _pack_reference(w, V, H):
+    """The tiled layout as its header states it, built here with numpy: the
+    vocabulary in ranges of round16(ceil(V / 148)) rows, each range in tiles of
+    up to 128 rows; tile (first row r0, rt rows) holds, for each 64-wide
+    column chunk kk in turn, its rt rows' 64 values of that chunk."""
+    KCT = H // 64
+    per = -(-V // 148)
+    per = -(-per // 16) * 16
+    pieces = w.reshape(V, KCT, 64)
+    out = np.empty((V * KCT, 64), dtype=w.dtype)
+    for lo in range(0, V, per):
+        hi = min(V, lo + per)
+        for r0 in range(lo, hi, 128):
+            rt = min(128, hi - r0)
+            tile = pieces[r0:r0 + rt].transpose(1, 0, 2).reshape(KCT * rt, 64)
+            out[r0 * KCT:(r0 + rt) * KCT] = tile
+    return out.reshape(V, H)
+
+
+@pytest.mark.parametrize("V,H", [(5000, 448), (7001, 64), (1, 128)])
+def test_pack_weight_matches_the_stated_layout(V, H):
+    g = torch.Generator().manual_seed(V + H)
+    w = torch.randn((V, H), generator=g).to(torch.bfloat16)
+    cfg = fdl.make_cfg(dict(batch=1, n_q_heads=1, n_kv_heads=1, head_dim=32, block_size=1,
+                            q_off=0, q_len=1, cap_prefix=0, hidden=H, vocab=V,
+                            mask_id=0, shift=0, tau=0.9, dtype="bf16"))
+    packed = torch.empty((V, H), dtype=torch.bfloat16, device="cuda")
+    fdl.lmhead_pack_weight(cfg, w.cuda(), packed)
+    torch.cuda.synchronize()
+    want = _pack_reference(w.view(torch.int16).numpy(), V, H)
+    assert np.array_equal(packed.cpu().view(torch.int16).numpy(), want)
+
+
+@pytest.mark.parametrize("R,V,H", [(32, 152064, 3584), (40, 5000, 448), (600, 20000, 256),
+                                   (256, 7001, 64)])
+@pytest.mark.parametrize("entry", ["lmhead", "noalloc"])
+def test_packed_weight_gives_identical_results(R, V, H, entry):
+    """The LM head over the tiled weight returns the very same bits as over
+    the row-major one (same MMAs, same order), and matches the oracle."""
+    if entry == "noalloc" and R > 128:
+        pytest.skip("the allocation-free entry takes at most 128 rows")
+    g = torch.Generator().manual_seed(R + V + H)
+    rows = torch.randn((R, H), generator=g).to(torch.bfloat16)
+    w = (torch.randn((V, H), generator=g) * (8.0 / H ** 0.5)).to(torch.bfloat16)
+    cfg = fdl.make_cfg(dict(batch=R, n_q_heads=1, n_kv_heads=1, head_dim=32, block_size=1,
+                            q_off=0, q_len=1, cap_prefix=0, hidden=H, vocab=V,
+                            mask_id=V - 1, shift=0, tau=0.9, dtype="bf16"))
+    w_d = w.cuda()
+    w_p = torch.empty_like(w_d)
+    fdl.lmhead_pack_weight(cfg, w_d, w_p)
+    ws = fdl.workspace(cfg)
+    got = {}
+    for layout, wt in [(fdl.W_ROW_MAJOR, w_d), (fdl.W_PACKED, w_p)]:
+        cfg.w_layout = layout
+        conf = torch.empty(R, dtype=torch.float32, device="cuda")
+        tok = torch.empty(R, dtype=torch.int32, device="cuda")
+        if entry == "lmhead":
+            fdl.lmhead_confidence(cfg, rows.cuda(), wt, None, conf, tok, ws)
+        else:
+            fdl.lmhead_confidence_noalloc(cfg, rows.cuda(), wt, None, conf, tok)
+        torch.cuda.synchronize()
+        got[layout] = (conf.cpu().numpy(), tok.cpu().numpy())
+    assert np.array_equal(got[0][0].view(np.int32), got[1][0].view(np.int32))
+    assert np.array_equal(got[0][1], got[1][1])
+    t_ref, c_ref, gap = step.lmhead_confidence(rows.double().numpy(), w.float().numpy())
+    sure = gap > 1e-3
+    assert np.array_equal(got[1][1][sure], t_ref[sure])
+    np.testing.assert_allclose(got[1][0].astype(np.float64), c_ref, rtol=1e-3)
+    assert fdl.get_status(ws) == 0
+
+
+@pytest.mark.parametrize("name,cfg", [("qwen7b", None), ("large_batch", LARGE_BATCH)])
+def test_fused_step_over_the_packed_weight(name, cfg):
+    """The fused step (LM head beside the attention, or in two passes) over
+    the tiled weight: bit-exact commits against the oracle, as row-major."""
+    case, ref, _ = cases.parity_case(name, 1, cfg=cfg) if cfg else cases.parity_case(name, 1)
+    gh.compare_step(case, gh.run_denoise_step(case, packed=True), ref)
+
+
 # ------------------------------------------------------ failure detection
 
 def test_bounded_wait_times_out_into_the_status_word():
