@@ -20,6 +20,10 @@
 //   warps 2-5  epilogue: tcgen05.ld 32 lanes x 32 columns, a warp
 //            reduce-scatter of (max, sum-exp, argmax) over the 32 vocab rows
 //            leaves column j's triple in lane j, merged into a running state.
+//            From N = 128 on, where the epilogue and not the weight stream
+//            bounds the kernel, the 32 x 32 block is transposed through
+//            shared memory instead and lane j folds column j's 32 logits into
+//            its running state one at a time (one exponential per logit).
 // The per-CTA triples go to the workspace; the last CTA to arrive merges them
 // (and, in the fused step, commits).  No thread waits on another CTA.
 #include "lm_merge.cuh"
@@ -47,6 +51,34 @@ struct TcParams {
   int stages_b;
   uint32_t tmem_cols;
 };
+
+constexpr int kTrStride = 33;  // transpose rows: 32 floats + 1 (no bank conflicts)
+constexpr int kTrBytes = 4 * 32 * kTrStride * 4;  // one 32 x 33 buffer per epilogue warp
+
+// Shared bytes of the epilogue's cross-warp region: the per-quarter states
+// of every column, which from N = 128 on also hold the transpose buffers.
+__host__ __device__ constexpr size_t red_bytes(int npad) {
+  return npad >= 128 && (size_t)kTrBytes > 4 * (size_t)npad * sizeof(MSI)
+             ? (size_t)kTrBytes : 4 * (size_t)npad * sizeof(MSI);
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Fold one logit v of vocabulary entry idx into a running state; entries
+// arrive in increasing idx, so an equal logit keeps the earlier index.  The
+// larger of the two maxima scales the other side: one exponential.
+__device__ __forceinline__ void msi_push(MSI& st, float v, int idx) {
+  const float d = v - st.m;
+  const bool up = d > 0.f;
+  const float e = ex2_approx(-fabsf(d) * kLog2e);
+  st.s = up ? fmaf(st.s, e, 1.f) : st.s + e;
+  st.m = up ? v : st.m;
+  st.i = up ? idx : st.i;
+}
 
 __device__ __forceinline__ void named_barrier_epilogue() {
   asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -256,6 +288,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
   } else {
     // ---------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may read
+    float* tr = reinterpret_cast<float*>(s_red) + (warp - 2) * (32 * kTrStride);
     MSI st[NCH];
 #pragma unroll
     for (int c = 0; c < NCH; ++c) st[c] = msi_empty();
@@ -265,8 +298,10 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
       tc_fence_after();
       const int t0 = g * G, t1 = min(n_tiles, t0 + G);
       for (int t = t0; t < t1; ++t) {
-        const int vocab = v0 + t * kTileM + q * 32 + lane;
+        const int vbase = v0 + t * kTileM + q * 32;
+        const int vocab = vbase + lane;
         const bool valid = vocab < v1;
+        const int n_valid = min(32, v1 - vbase);  // same for the whole warp
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
           uint32_t r[32];
@@ -274,16 +309,31 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
                                  (uint32_t)((buf * G + (t - t0)) * NPAD + c * 32),
                              r);
           tmem_ld_wait();
-          MSI s[32];
+          if constexpr (NCH >= 4) {
+            // Lane = vocabulary row in r; after the transpose lane j reads
+            // column j, rows in increasing vocabulary order.
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            s[j] = valid ? MSI{__uint_as_float(r[j]), 1.f, vocab} : msi_empty();
-          st[c] = msi_merge(st[c], reduce_scatter32(s, lane));
+            for (int j = 0; j < 32; ++j) tr[lane * kTrStride + j] = __uint_as_float(r[j]);
+            __syncwarp();
+            MSI m = st[c];
+            for (int k = 0; k < n_valid; ++k) msi_push(m, tr[k * kTrStride + lane], vbase + k);
+            st[c] = m;
+            __syncwarp();
+          } else {
+            MSI s[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              s[j] = valid ? MSI{__uint_as_float(r[j]), 1.f, vocab} : msi_empty();
+            st[c] = msi_merge(st[c], reduce_scatter32(s, lane));
+          }
         }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
     }
+    // From N = 128 on the transpose buffers share this region: every warp
+    // is done with its buffer before the states are written.
+    if constexpr (NCH >= 4) named_barrier_epilogue();
 #pragma unroll
     for (int c = 0; c < NCH; ++c) s_red[q * NPAD + c * 32 + lane] = st[c];
     named_barrier_epilogue();
@@ -451,8 +501,7 @@ bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcPara
     // its ring needs the deeper prefetch.
     const int sb = shared ? 2 : 4;
     const size_t b_bytes = (size_t)sb * b_stage;
-    const size_t fixed = 1024 + 8 * (size_t)(2 * 12 + 2 * sb + 5) + 16 +
-                         4 * (size_t)tp->npad * sizeof(MSI);
+    const size_t fixed = 1024 + 8 * (size_t)(2 * 12 + 2 * sb + 5) + 16 + red_bytes(tp->npad);
     const size_t ring_cap = shared ? cap : fixed + 200 * 1024;
     if (ring_cap < fixed + b_bytes + 2 * a_stage) continue;
     int sa = (int)((ring_cap - fixed - b_bytes) / a_stage);
@@ -461,7 +510,7 @@ bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcPara
     tp->stages_b = sb;
     tp->stages_a = sa;
     const size_t bars = 8 * (size_t)(2 * sa + 2 * sb + 5) + 16;
-    *smem = 1024 + (size_t)sa * a_stage + b_bytes + bars + 4 * (size_t)tp->npad * sizeof(MSI);
+    *smem = 1024 + (size_t)sa * a_stage + b_bytes + bars + red_bytes(tp->npad);
     if (shared && 2 * (*smem + kSmReserve) <= kSmPerSM) *smem = kSmPerSM / 2;  // one per SM
     if (*smem > cap) return false;
     return true;
