@@ -16,7 +16,8 @@
 //   warp 1   MMA issuer: tcgen05.mma kind::f16, accumulators in TMEM; tiles
 //            are processed in groups of G, K-outer inside a group so each X
 //            chunk is reused by G tiles; two TMEM buffers let the epilogue
-//            of group g overlap the MMAs of group g+1;
+//            of group g overlap the MMAs of group g+1 (at N = 256, one
+//            buffer of two tiles instead: half the X traffic);
 //   warps 2-5  epilogue: tcgen05.ld 32 lanes x 32 columns, a warp
 //            reduce-scatter of (max, sum-exp, argmax) over the 32 vocab rows
 //            leaves column j's triple in lane j, merged into a running state.
@@ -47,6 +48,7 @@ struct TcParams {
   int npad;        // MMA N: 32, 64, 128 or 256
   int ksub;        // 64-wide K boxes per pipeline stage
   int group;       // tiles per TMEM buffer
+  int nbuf;        // TMEM buffers: 2 (epilogue overlaps the next group) or 1
   int stages_a;
   int stages_b;
   uint32_t tmem_cols;
@@ -251,8 +253,9 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
       const uint32_t idesc = idesc_bf16_f32(kTileM, NPAD);
       int ia = 0, ib = 0;
       for (int g = 0; g < n_groups && !failed; ++g) {
-        const int buf = g & 1;
-        if (!mbar_wait(&acc_empty[buf], ((g >> 1) & 1) ^ 1)) { failed = true; break; }
+        const int buf = tp.nbuf == 2 ? (g & 1) : 0;
+        const uint32_t ph = tp.nbuf == 2 ? ((g >> 1) & 1) : (g & 1);
+        if (!mbar_wait(&acc_empty[buf], ph ^ 1)) { failed = true; break; }
         tc_fence_after();
         const int t0 = g * G, t1 = min(n_tiles, t0 + G);
         for (int kc = 0; kc < KC && !failed; ++kc) {
@@ -293,8 +296,9 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
 #pragma unroll
     for (int c = 0; c < NCH; ++c) st[c] = msi_empty();
     for (int g = 0; g < n_groups; ++g) {
-      const int buf = g & 1;
-      if (!mbar_wait(&acc_full[buf], (g >> 1) & 1)) { failed = true; break; }
+      const int buf = tp.nbuf == 2 ? (g & 1) : 0;
+      const uint32_t ph = tp.nbuf == 2 ? ((g >> 1) & 1) : (g & 1);
+      if (!mbar_wait(&acc_full[buf], ph)) { failed = true; break; }
       tc_fence_after();
       const int t0 = g * G, t1 = min(n_tiles, t0 + G);
       for (int t = t0; t < t1; ++t) {
@@ -479,11 +483,20 @@ bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcPara
     G = (n_tiles + n_groups - 1) / n_groups;
   }
   if (G < 1) G = 1;
+  tp->nbuf = 2;
+  // N = 256 (full form): two buffers hold one tile each, so every 32 KB X
+  // chunk would be staged again for each 16 KB weight box.  One buffer of
+  // two tiles halves the X traffic; the MMAs then wait for the epilogue
+  // between groups.
+  if (!shared && tp->npad == 256 && n_tiles > 1) {
+    G = 2;
+    tp->nbuf = 1;
+  }
   tp->group = G;
   const int col_limit = shared ? 256 : 512;
-  if (2 * tp->group * tp->npad > col_limit) return false;
+  if (tp->nbuf * tp->group * tp->npad > col_limit) return false;
   uint32_t cols = 32;
-  while (cols < (uint32_t)(2 * tp->group * tp->npad)) cols *= 2;
+  while (cols < (uint32_t)(tp->nbuf * tp->group * tp->npad)) cols *= 2;
   tp->tmem_cols = cols;
   // Shared memory: the full form keeps 200 KB of rings; the shared form
   // what the SM has left.
@@ -499,13 +512,25 @@ bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcPara
     // Four X stages in the full form: at 256 rows an X chunk (32 KB) is
     // twice a weight stage and is staged again for every vocabulary tile, so
     // its ring needs the deeper prefetch.
-    const int sb = shared ? 2 : 4;
+    int sb = shared ? 2 : 4;
+    int sa = 0;
+    if (tp->nbuf == 1) {
+      // Balanced rings: as many K steps in flight for the X chunks as for
+      // the G weight boxes that use each one.
+      const size_t per_step = b_stage + (size_t)G * a_stage;
+      int n = (int)((200 * 1024) / per_step);
+      if (n * G > 12) n = 12 / G;
+      if (n < 2) continue;
+      sb = n;
+      sa = n * G;
+    } else {
+      const size_t fixed = 1024 + 8 * (size_t)(2 * 12 + 2 * sb + 5) + 16 + red_bytes(tp->npad);
+      const size_t ring_cap = shared ? cap : fixed + 200 * 1024;
+      if (ring_cap < fixed + (size_t)sb * b_stage + 2 * a_stage) continue;
+      sa = (int)((ring_cap - fixed - (size_t)sb * b_stage) / a_stage);
+      if (sa > 12) sa = 12;
+    }
     const size_t b_bytes = (size_t)sb * b_stage;
-    const size_t fixed = 1024 + 8 * (size_t)(2 * 12 + 2 * sb + 5) + 16 + red_bytes(tp->npad);
-    const size_t ring_cap = shared ? cap : fixed + 200 * 1024;
-    if (ring_cap < fixed + b_bytes + 2 * a_stage) continue;
-    int sa = (int)((ring_cap - fixed - b_bytes) / a_stage);
-    if (sa > 12) sa = 12;
     tp->ksub = ksub;
     tp->stages_b = sb;
     tp->stages_a = sa;
