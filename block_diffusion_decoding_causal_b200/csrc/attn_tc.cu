@@ -979,6 +979,16 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   t.group = a.group;
   t.qpt = qpt;
   t.n_rt = (a.q_len + qpt - 1) / qpt;
+  // Items of more than 64 query rows (PrefixCache, long units), whose
+  // partials are 64 KB fp32 tiles, and at least half as many items as
+  // CTAs: one CTA per item, so that equal-length items are never split and
+  // nothing is merged (at LLaDA-8B PrefixCache shapes the merge of the
+  // stream-K split cost more than the imbalance does).  Everything else
+  // keeps the full stream-K grid.
+  const int n_items_all = a.B * a.Hkv * t.n_rt;
+  if (!beside_prior && qpt * a.group > 64 && 2 * n_items_all >= n_cta &&
+      n_items_all <= n_cta)
+    n_cta = n_items_all;
   t.n_cta = n_cta;
   t.dual = a.k_suf != nullptr;
   t.scale_log2 = a.scale_log2;

@@ -334,6 +334,9 @@ def test_select_commit_factor_and_budget(policy, f):
     (1, 32, 32, 288, [768]),          # LLaDA-like: block 32 + suffix 256 recomputed
     (2, 28, 4, 100, [0, 1500]),       # GQA 7, ragged: empty prefix, 100 rows (2 chunks)
     (3, 8, 8, 200, [64, 65, 300]),    # MHA, prefixes on and off the 64-key chunk grid
+    (1, 32, 32, 768, [768]),          # LLaDA bench shape: 192 items, one CTA each
+    (2, 8, 8, 256, [512, 512]),       # equal lengths, 32 items over the stream-K grid
+    (4, 40, 40, 128, [300, 0, 64, 1000]),  # 160 ragged items, one CTA each: merges
 ])
 def test_prefixcache_attn_against_oracle(B, Hq, Hkv, n, lens):
     """PrefixCache attention: the recomputed rows (several 64-key chunks and
