@@ -186,7 +186,9 @@ int fdl_prefixcache_attn(const fdl_step_cfg* cfg, const void* q, const void* k_p
  * Algorithm 2 of the technical review, section 4).
  *   For each row i of rows [B*q_len, H] (already token-shifted: row
  *   (b, i) predicts block position q_off + i):
- *     l = w_lm . rows[i]  over the full vocabulary (w_lm [V, H] row-major),
+ *     l = w_lm . rows[i]  over the full vocabulary (w_lm [V, H] row-major,
+ *     or, with cfg->w_layout = FDL_W_PACKED, the same weight as rewritten
+ *     by fdl_lmhead_pack_weight; the results are identical),
  *     tok[i]  = argmax_v l_v (the lowest v on a tie),
  *     conf[i] = max softmax probability = 1 / sum_v exp(l_v - l_max).
  *   Logits never leave the chip.  Rows with row_active[i] == 0 report
@@ -263,7 +265,8 @@ int fdl_select_commit(const fdl_step_cfg* cfg, int policy, float param,
  * hidden: [B, q_len, H] or NULL (then H must equal Hq*d and the attention
  *   output, rounded to cfg->dtype, is used).  h_prev: [B, H], required iff
  *   cfg->shift.  attn_out: [B, q_len, Hq, d] or NULL (then it is kept in the
- *   workspace).  k_suf, v_suf, len_suf: all NULL or all set.
+ *   workspace).  k_suf, v_suf, len_suf: all NULL or all set.  w_lm in the
+ *   layout cfg->w_layout names, as for fdl_lmhead_confidence.
  * Outputs as fdl_lmhead_confidence and fdl_threshold_commit.
  */
 int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,

@@ -11,6 +11,7 @@ import torch
 from block_diffusion_decoding_causal_b200 import fdl, synth
 from oracle import cases, step
 from tests import gpu_harness as gh
+from tests.pack_layout import pack_reference
 
 pytestmark = pytest.mark.gpu
 
@@ -406,25 +407,6 @@ def test_fused_step_with_two_lm_passes():
 
 # ----------------------------------------------- tiled LM-head weight layout
 
-def _pack_reference(w, V, H):
-    """The tiled layout as its header states it, built here with numpy: the
-    vocabulary in ranges of round16(ceil(V / 148)) rows, each range in tiles of
-    up to 128 rows; tile (first row r0, rt rows) holds, for each 64-wide
-    column chunk kk in turn, its rt rows' 64 values of that chunk."""
-    KCT = H // 64
-    per = -(-V // 148)
-    per = -(-per // 16) * 16
-    pieces = w.reshape(V, KCT, 64)
-    out = np.empty((V * KCT, 64), dtype=w.dtype)
-    for lo in range(0, V, per):
-        hi = min(V, lo + per)
-        for r0 in range(lo, hi, 128):
-            rt = min(128, hi - r0)
-            tile = pieces[r0:r0 + rt].transpose(1, 0, 2).reshape(KCT * rt, 64)
-            out[r0 * KCT:(r0 + rt) * KCT] = tile
-    return out.reshape(V, H)
-
-
 @pytest.mark.parametrize("V,H", [(5000, 448), (7001, 64), (1, 128)])
 def test_pack_weight_matches_the_stated_layout(V, H):
     g = torch.Generator().manual_seed(V + H)
@@ -435,7 +417,7 @@ def test_pack_weight_matches_the_stated_layout(V, H):
     packed = torch.empty((V, H), dtype=torch.bfloat16, device="cuda")
     fdl.lmhead_pack_weight(cfg, w.cuda(), packed)
     torch.cuda.synchronize()
-    want = _pack_reference(w.view(torch.int16).numpy(), V, H)
+    want = pack_reference(w.view(torch.int16).numpy(), V, H)
     assert np.array_equal(packed.cpu().view(torch.int16).numpy(), want)
 
 
