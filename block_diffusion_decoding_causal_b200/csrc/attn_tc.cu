@@ -1028,6 +1028,9 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
     if (e != cudaSuccess) return e;
   }
   if (beside_prior) return cudaSuccess;  // merged inside the kernel
+  // One sequence and one CTA per item: all its items have the same chunks,
+  // so each CTA's range is exactly one item and there is nothing to merge.
+  if (a.B == 1 && n_cta == n_items_all) return cudaGetLastError();
   cudaLaunchConfig_t lc = {};
   const int n_items = a.B * a.Hkv * t.n_rt;
   // Partials per split item are about n_cta / n_items + 1: few, and a CTA
