@@ -194,10 +194,13 @@ def test_sweep_full_size(batch, prefix):
 # ---------------------------------------------- LM head shapes and tails
 
 @pytest.mark.parametrize("R,V,H", [(1, 5000, 64), (32, 5000, 448), (33, 33000, 128),
-                                   (128, 20000, 256), (256, 7001, 64), (8, 151936, 1536)])
+                                   (128, 20000, 256), (256, 7001, 64), (8, 151936, 1536),
+                                   (256, 152064, 256), (200, 152064, 128)])
 def test_lmhead_shapes_against_oracle(R, V, H):
     """Every N padding (32..256), partial vocab tiles (5000 / 148 CTAs = 48
-    rows each), ragged vocab ends and several K depths.  Tokens must match
+    rows each), ragged vocab ends and several K depths; at the 7B vocabulary
+    with N = 256, nine tiles per CTA in groups of two sharing one TMEM
+    buffer, the last group a single 16-row tile.  Tokens must match
     wherever the oracle's top-2 logit gap exceeds 1e-3 (fp32 accumulation
     error is ~1e-5 at these sizes); confidences within 1e-3 relative."""
     g = torch.Generator().manual_seed(R * 7 + V + H)
