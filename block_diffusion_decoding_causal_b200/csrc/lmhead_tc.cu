@@ -509,9 +509,8 @@ bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcPara
     const size_t b_stage = (size_t)tp->npad * 128 * ksub;
     if (b_stage > 16384 && ksub > 1) continue;  // X stage within 16 KB when possible
     const size_t a_stage = (size_t)kStageA * ksub;
-    // Four X stages in the full form: at 256 rows an X chunk (32 KB) is
-    // twice a weight stage and is staged again for every vocabulary tile, so
-    // its ring needs the deeper prefetch.
+    // Four X stages in the full form (two when shared): the wider X chunks
+    // (16 KB at 128 rows, as large as a weight box) need the deeper prefetch.
     int sb = shared ? 2 : 4;
     int sa = 0;
     if (tp->nbuf == 1) {
