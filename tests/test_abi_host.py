@@ -239,3 +239,30 @@ def test_weight_layout_rules(L):
     assert rc == fdl.ERR_UNSUPPORTED and "bf16" in fdl.last_error()
     rc = L.fdl_lmhead_confidence_noalloc(ctypes.byref(f32), q[0], q[1], None, q[2], q[3], None)
     assert rc == fdl.ERR_UNSUPPORTED and "bf16" in fdl.last_error()
+
+
+def test_step_cfg_layout_matches_the_header(tmp_path):
+    """The binding's StepCfg has the size and field offsets of fdl_step_cfg
+    as the C compiler lays it out from include/fdl.h."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    names = [f[0] for f in fdl.StepCfg._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"fdl.h\"\n"
+                   "int main(void) {\n"
+                   "  printf(\"size %zu\\n\", sizeof(fdl_step_cfg));\n"
+                   + "".join(f'  printf("{n} %zu\\n", offsetof(fdl_step_cfg, {n}));\n'
+                             for n in names)
+                   + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    include = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                           "include")
+    subprocess.run([cc, "-I", include, str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    c_layout = dict(line.split() for line in out.splitlines())
+    assert int(c_layout["size"]) == ctypes.sizeof(fdl.StepCfg)
+    for n in names:
+        assert int(c_layout[n]) == getattr(fdl.StepCfg, n).offset, n
