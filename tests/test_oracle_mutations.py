@@ -136,3 +136,23 @@ def test_budget_rule_without_the_max_term_is_caught(monkeypatch):
     monkeypatch.setattr(theory, "heterogeneous_budget_ok",
                         lambda eps: sum(float(e) for e in eps) < 1.0)
     _expect_pin_failure(pins.test_budget_rule_eq9_selection)
+
+
+def test_dualcache_without_its_suffix_is_caught(monkeypatch):
+    orig = step.attention_step
+
+    def no_suffix(q, k_pre, v_pre, len_pre, prompt_len, k_blk, v_blk, q_off,
+                  k_suf=None, v_suf=None, len_suf=None):
+        return orig(q, k_pre, v_pre, len_pre, prompt_len, k_blk, v_blk, q_off)
+    monkeypatch.setattr(step, "attention_step", no_suffix)
+    _expect_pin_failure(pins.test_prefixcache_block_rows_equal_dualcache_with_the_same_suffix)
+
+
+def test_prefixcache_over_the_whole_cache_capacity_is_caught(monkeypatch):
+    orig = step.prefixcache_attention
+
+    def whole_cap(q, k_pre, v_pre, len_pre, k_fresh, v_fresh):
+        cap = np.asarray(k_pre).shape[2]
+        return orig(q, k_pre, v_pre, np.full(len(len_pre), cap), k_fresh, v_fresh)
+    monkeypatch.setattr(step, "prefixcache_attention", whole_cap)
+    _expect_pin_failure(pins.test_prefixcache_attention_matches_torch_sdpa_with_gqa)
