@@ -108,28 +108,40 @@ class ClockSampler:
 
 # ------------------------------------------------------------- CPU oracle
 
+def host_cores() -> int:
+    """Host threads this process may run on (the oracle uses one per core)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def oracle_baseline(case, min_seconds: float = 10.0, max_steps: int = 50) -> dict:
-    """Time the CPU oracle (as it stands) on this workload: whole steps,
-    repeated until ``min_seconds`` have passed."""
-    import numpy as np
-    import threadpoolctl
+    """Time the CPU oracle (the plain fp64 C++ program, as it stands) on this
+    workload: whole steps on every host core, repeated until ``min_seconds``
+    have passed, then one whole step on a single thread."""
     from oracle import cases
-    threads = max(
-        [i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
+    threads = host_cores()
     n, t0 = 0, time.perf_counter()
     while True:
-        cases.run_oracle(case)
+        cases.run_oracle(case, threads=threads)
         n += 1
         el = time.perf_counter() - t0
         if el >= min_seconds or n >= max_steps:
             break
     c = case.cfg
-    pos = n * c["batch"] * c["q_len"]
-    return {"value": pos / el, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+    per_step = c["batch"] * c["q_len"]
+    t1 = time.perf_counter()
+    cases.run_oracle(case, threads=1)
+    el1 = time.perf_counter() - t1
+    return {"value": n * per_step / el, "unit": UNIT, "cores": int(threads),
+            "kind": "oracle",
             "sample": f"{n} whole oracle step(s) of the benchmark workload "
                       f"({c['batch']} x {c['q_len']} positions each), {el:.1f} s, "
-                      f"numpy fp64 with {threads} BLAS threads",
-            "seconds": el, "steps": n}
+                      f"plain fp64 C++ (no BLAS) on {threads} threads",
+            "seconds": el, "steps": n,
+            "single_thread": {"value": per_step / el1, "unit": UNIT, "seconds": el1,
+                              "sample": "one whole oracle step on one thread"}}
 
 
 # ------------------------------------------------------------------- main
@@ -195,14 +207,13 @@ def run_reference(args):
     from oracle import cases
     case = synth.make_case(WORKLOAD, args.seed)
     c = case.cfg
+    threads = host_cores()
     for _ in range(args.warmup):
-        cases.run_oracle(case)
+        cases.run_oracle(case, threads=threads)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        cases.run_oracle(case)
+        cases.run_oracle(case, threads=threads)
     el = time.perf_counter() - t0
-    import threadpoolctl
-    threads = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
     pos = args.steps * c["batch"] * c["q_len"]
     value = pos / el
     line = {
@@ -213,7 +224,8 @@ def run_reference(args):
         "config": _config(c, args),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(threads),
                          "kind": "oracle",
-                         "sample": f"{args.steps} whole oracle steps of the workload"},
+                         "sample": f"{args.steps} whole oracle steps of the workload, "
+                                   f"plain fp64 C++ (no BLAS) on {threads} threads"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -19,8 +19,6 @@ margin holds and report how many rows were redrawn.
 from __future__ import annotations
 
 import numpy as np
-import torch
-
 from block_diffusion_decoding_causal_b200 import synth
 from . import step
 
@@ -29,25 +27,20 @@ CONF_MARGIN = 5e-3
 CAND_REL = 2e-3
 
 
-def _np(t, dtype=np.float64):
-    if t is None:
-        return None
-    if t.dtype in (torch.bfloat16, torch.float16):
-        t = t.to(torch.float32)
-    return t.numpy().astype(dtype, copy=False)
+def run_oracle(case: synth.Case, previous: dict = None, redo_q=None, redo_lm=None,
+               threads: int = 0) -> dict:
+    """The oracle's denoise step on a synthetic case (inputs as stored).
 
-
-def run_oracle(case: synth.Case) -> dict:
-    """The oracle's denoise step on a synthetic case (inputs upcast exactly)."""
+    With ``previous`` and the [B, q_len] flags ``redo_q`` / ``redo_lm`` only
+    the flagged query rows and LM-head rows are recomputed (see
+    ``step.denoise_step``)."""
     c = case.cfg
-    w = case.w_lm
-    w_np = (w.to(torch.float32) if w.dtype != torch.float32 else w).numpy()
     return step.denoise_step(
-        c, _np(case.q), _np(case.k_pre), _np(case.v_pre),
-        case.len_pre.numpy(), case.prompt_len.numpy(), _np(case.k_blk),
-        _np(case.v_blk), _np(case.hidden), _np(case.h_prev), w_np,
-        case.block_tokens.numpy(), _np(case.k_suf), _np(case.v_suf),
-        None if case.len_suf is None else case.len_suf.numpy())
+        c, case.q, case.k_pre, case.v_pre, case.len_pre.numpy(),
+        case.prompt_len.numpy(), case.k_blk, case.v_blk, case.hidden, case.h_prev,
+        case.w_lm, case.block_tokens.numpy(), case.k_suf, case.v_suf,
+        None if case.len_suf is None else case.len_suf.numpy(), threads=threads,
+        previous=previous, redo_q=redo_q, redo_lm=redo_lm)
 
 
 def _violations(case: synth.Case, res: dict):
@@ -71,34 +64,45 @@ def _violations(case: synth.Case, res: dict):
     return sorted(bad)
 
 
-def _redraw_source(case: synth.Case, b: int, i: int, attempt: int) -> None:
-    """Redraw the input row that feeds LM-head row (b, i)."""
+def _redraw_source(case: synth.Case, b: int, i: int, attempt: int, redo_q, redo_lm):
+    """Redraw the input row that feeds LM-head row (b, i) and flag the rows
+    whose results that changes."""
     shift = case.cfg["shift"]
+    q_len = case.cfg["q_len"]
     if shift and i == 0:
         synth.redraw_row(case, "h_prev", (b,), attempt)
+        redo_lm[b, 0] = 1
         return
     src = i - 1 if shift else i
     if case.hidden is not None:
         synth.redraw_row(case, "hidden", (b, src), attempt)
     else:
         synth.redraw_row(case, "q", (b, src), attempt)
+        redo_q[b, src] = 1
+    if src + shift < q_len:
+        redo_lm[b, src + shift] = 1
 
 
 def parity_case(name: str, seed: int, cfg=None, attn_as_hidden: bool = False,
                 max_rounds: int = 40, **overrides):
     """A synthetic case with every decision margin satisfied.
 
-    Returns (case, oracle result, number of redrawn rows).
+    Returns (case, oracle result, number of redrawn rows).  After the first
+    full oracle run, each round recomputes only the rows it redrew.
     """
     case = synth.make_case(name, seed, cfg=cfg, attn_as_hidden=attn_as_hidden,
                            **overrides)
     redrawn = 0
+    res = run_oracle(case)
+    B, q_len = case.cfg["batch"], case.cfg["q_len"]
     for attempt in range(max_rounds):
-        res = run_oracle(case)
         bad = _violations(case, res)
         if not bad:
             return case, res, redrawn
+        redo_q = np.zeros((B, q_len), dtype=np.uint8)
+        redo_lm = np.zeros((B, q_len), dtype=np.uint8)
         for (b, i) in bad:
-            _redraw_source(case, b, i, attempt)
+            _redraw_source(case, b, i, attempt, redo_q, redo_lm)
             redrawn += 1
+        res = run_oracle(case, previous=res, redo_q=redo_q, redo_lm=redo_lm)
     raise RuntimeError(f"margin repair did not converge for {name} seed {seed}")

@@ -1,339 +1,388 @@
-"""CPU oracle for one denoising step of the active block (fp64, numpy).
+"""CPU oracle for one denoising step of the active block: the Python face of
+the plain fp64 C++ program in ``step.cc`` (built into ``liboracle.so``).
 
-TEST INFRASTRUCTURE.  Only the tests, the smoke check and the CPU-baseline leg
-of the benchmark may import this package.  The CUDA library never calls it and
-shares no code with it.
+TEST INFRASTRUCTURE.  Only the tests, the smoke check and the benchmark's
+CPU-baseline and reference legs may import this package.  The CUDA library
+never calls it and shares no code with it.
 
-Every function below writes out the plain definition the pages give; nothing is
-blocked, fused or reordered.  Sources (page title, then the passage):
+This module only marshals arguments (numpy arrays or CPU torch tensors in,
+numpy arrays out) and sequences no arithmetic of its own: every step of the
+method, its citations and the readings taken where the pages are silent are in
+``step.cc``.  ``step_np`` holds an earlier, independent numpy restatement of
+the same definitions, kept as a second check.
 
-* "Fast-dLLM v2: Efficient Block-Diffusion LLM" (paper digest), section 3.4:
-  "Attention Mask Design" with the inference-time mask of Figure 7b;
-  "Step 5: Token shift for prediction"; "Inference Pipeline", Levels 1-3.
-* "Fast-dLLM: Reusing Bidirectional State and Spending Confidence on Parallel
-  Tokens" (technical review), section 2 eq. (3) (attention), section 3
-  (PrefixCache / DualCache), section 4 Algorithm 2 (threshold selection).
-
-Readings where the pages are silent (each is listed in the design notes):
-* GQA: query head h reads KV head h // (Hq / Hkv).
-* argmax over the full vocabulary, lowest index on a tie; confidence is the
-  largest softmax probability 1 / sum_v exp(l_v - l_max).
-* commit compares conf >= tau, with tau as the float32 the library receives;
-  the fallback picks the lowest position among equal confidences.
-* token shift: the row that predicts unit position q_off + i is the hidden state
-  of position q_off + i - 1; for i = 0 it is the caller's h_prev.
-* attention output is rounded once to the storage dtype (bf16: round to
-  nearest even) before it is used as an LM-head row.
-
-Parity of that last rounding point and of the GPU's fp32 exponentials is
-unpinned by the pages: tolerances and decision margins cover both.
+Stored inputs are passed as they are stored (bf16 bit patterns, fp32 or
+fp64) and upcast exactly inside the oracle.
 """
 from __future__ import annotations
 
+import contextlib
+import ctypes
+import os
+
 import numpy as np
+
+from . import build as _build
+
+F32, BF16, F64 = 0, 1, 2
+RULE_THRESHOLD, RULE_FACTOR, RULE_BUDGET = 0, 1, 2
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_L = ctypes.c_int64
+_D = ctypes.c_double
+
+_lib = None
+
+
+class StepCfg(ctypes.Structure):
+    """Mirror of ``orc_step_cfg`` in step.cc."""
+    _fields_ = [("B", _I), ("q_len", _I), ("Hq", _I), ("Hkv", _I), ("d", _I), ("D", _I),
+                ("q_off", _I), ("cap_pre", _L), ("cap_suf", _L), ("H", _L), ("V", _L),
+                ("mask_id", _L), ("shift", _I), ("stored", _I), ("w_stored", _I),
+                ("threads", _I), ("tau", ctypes.c_float)]
+
+
+def _declare(L):
+    L.orc_version.restype = _I
+    L.orc_round.argtypes = [_L, _P, _I, _P]
+    L.orc_training_mask.argtypes = [_L, _L, _P]
+    L.orc_block_ids.argtypes = [_L, _P, _L, _L, _P]
+    L.orc_inference_visibility.argtypes = [_L, _P, _L, _P, _L, _L, _I, _P]
+    L.orc_masked_attention.argtypes = [_L, _L, _I, _P, _P, _P, _P, _P]
+    L.orc_attention_step.argtypes = ([_I] * 6 + [_L, _L, _I, _I] + [_P] * 10 + [_P, _I])
+    L.orc_prefixcache_attention.argtypes = [_I] * 5 + [_L, _I] + [_P] * 7 + [_I]
+    L.orc_shifted_rows.argtypes = [_I, _I, _L, _I, _P, _P, _P]
+    L.orc_lmhead_confidence.argtypes = [_L, _L, _L, _P, _P, _I, _P, _P, _P, _I]
+    L.orc_select.argtypes = [_I, _D, _I, _P, _P, _P]
+    L.orc_select.restype = _I
+    L.orc_budget_ok.argtypes = [_I, _P]
+    L.orc_budget_ok.restype = _I
+    L.orc_commit.argtypes = [_I, _I, _I, _I, _L, _I, _D] + [_P] * 7
+    L.orc_denoise_step.argtypes = [ctypes.POINTER(StepCfg)] + [_P] * 28
+    L.orc_denoise_step.restype = _I
+    return L
+
+
+def load(path: str):
+    """Load an oracle library from ``path`` (the tests load mutated builds)."""
+    return _declare(ctypes.CDLL(path))
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = load(_build.build())
+    return _lib
+
+
+@contextlib.contextmanager
+def using(library):
+    """Route every call of this module to ``library`` inside the block."""
+    global _lib
+    saved = lib()
+    _lib = library
+    try:
+        yield
+    finally:
+        _lib = saved
+
+
+# ------------------------------------------------------------ marshalling
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_P)
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _i64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int64))
+
+
+def _stored(x):
+    """(contiguous numpy array, stored code) for an input kept as stored:
+    torch bf16 -> its bit patterns; fp32 stays fp32; anything else fp64."""
+    if x is None:
+        return None, None
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous()
+            if x.dtype == torch.bfloat16:
+                return x.view(torch.int16).numpy().view(np.uint16), BF16
+            x = x.numpy()
+    except ImportError:
+        pass
+    x = np.asarray(x)
+    if x.dtype == np.float32:
+        return np.ascontiguousarray(x), F32
+    return _f64(x), F64
+
+
+def _same_stored(*xs):
+    arrs, codes = zip(*(_stored(x) for x in xs))
+    kinds = {c for c in codes if c is not None}
+    if len(kinds) > 1:                       # mixed storage: compare in fp64
+        arrs = tuple(None if x is None else _f64(_as_f64(x)) for x in xs)
+        return arrs, F64
+    return arrs, (kinds.pop() if kinds else F64)
+
+
+def _as_f64(x):
+    a, code = _stored(x)
+    if code == BF16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
 
 # ----------------------------------------------------------------- rounding
 
-
-def round_bf16(x) -> np.ndarray:
-    """Round fp64 values to bfloat16 (8 significant bits, ties to even).
-
-    bfloat16 keeps the fp32 exponent range and 1 + 7 mantissa bits.  Written
-    as: x = m * 2**e with 0.5 <= |m| < 1, keep round(m * 2**8) (numpy's rint
-    rounds half to even).  Valid for normal numbers, which is all the step
-    produces; bf16 subnormals (|x| < 2**-126) are not modelled.
-    """
-    x = np.asarray(x, dtype=np.float64)
-    m, e = np.frexp(x)
-    return np.ldexp(np.rint(m * 256.0), e - 8)
-
-
 def round_to(x, dtype: str) -> np.ndarray:
     """Round fp64 values to the storage dtype ("f32" or "bf16")."""
-    if dtype == "bf16":
-        return round_bf16(x)
-    if dtype == "f32":
-        return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
-    raise ValueError(dtype)
+    code = {"f32": F32, "bf16": BF16}[dtype]
+    x = _f64(x)
+    out = np.empty_like(x)
+    lib().orc_round(x.size, _ptr(x), code, _ptr(out))
+    return out
+
+
+def round_bf16(x) -> np.ndarray:
+    """Round fp64 values to bfloat16 (8 significant bits, ties to even)."""
+    return round_to(x, "bf16")
 
 
 # ------------------------------------------------------------------ masks
 
-
 def training_mask(L: int, D: int) -> np.ndarray:
-    """M_full over the concatenation [x_t ; x_0] of length 2L (v2 digest,
-    "Attention Mask Design"): [[M_BD, M_OBC], [0, M_BC]].
-
-    M_BD: noised i sees noised j iff same block.  M_OBC: noised i sees clean j
-    iff j's block is strictly before i's.  M_BC: clean i sees clean j iff j's
-    block is the same or earlier.  Clean never sees noised (zero quadrant).
-    """
-    blk = np.arange(L) // D
-    same = blk[:, None] == blk[None, :]
-    before = blk[None, :] < blk[:, None]
-    same_or_before = blk[None, :] <= blk[:, None]
-    top = np.concatenate([same, before], axis=1)
-    bottom = np.concatenate([np.zeros((L, L), dtype=bool), same_or_before], axis=1)
-    return np.concatenate([top, bottom], axis=0)
+    """M_full over [x_t ; x_0] (v2 digest, "Attention Mask Design"), [2L, 2L]."""
+    out = np.empty((2 * L, 2 * L), dtype=np.uint8)
+    lib().orc_training_mask(L, D, _ptr(out))
+    return out.astype(bool)
 
 
-def block_ids(pos: np.ndarray, prompt_len: int, D: int) -> np.ndarray:
-    """Block index of absolute positions: the prompt is block 0, then the
-    generated answer is cut into blocks of D (v2 digest, Level 1)."""
-    pos = np.asarray(pos)
-    return np.where(pos < prompt_len, 0, 1 + (pos - prompt_len) // D)
+def block_ids(pos, prompt_len: int, D: int) -> np.ndarray:
+    """Block index of absolute positions (prompt = block 0)."""
+    pos = _i64(pos)
+    out = np.empty_like(pos)
+    lib().orc_block_ids(pos.size, _ptr(pos), int(prompt_len), int(D), _ptr(out))
+    return out
 
 
-def inference_visibility(q_pos, k_pos, prompt_len: int, D: int,
-                         full: bool) -> np.ndarray:
-    """Which keys each query of the active block may attend to.
-
-    Block-causal (v2, Figure 7b): a query sees every key in its own block
-    (bidirectional) and every key in an earlier block (causal across blocks).
-    ``full``: v1 DualCache over a full-attention dLLM, where every position of
-    the sequence (prefix, block, masked suffix) is visible (technical review,
-    section 3).
-    """
-    q_pos = np.asarray(q_pos)
-    k_pos = np.asarray(k_pos)
-    if full:
-        return np.ones((q_pos.size, k_pos.size), dtype=bool)
-    qb = block_ids(q_pos, prompt_len, D)
-    kb = block_ids(k_pos, prompt_len, D)
-    return kb[None, :] <= qb[:, None]
+def inference_visibility(q_pos, k_pos, prompt_len: int, D: int, full: bool) -> np.ndarray:
+    """Block-causal (or, with ``full``, full) visibility of keys by queries."""
+    q_pos, k_pos = _i64(q_pos).ravel(), _i64(k_pos).ravel()
+    out = np.empty((q_pos.size, k_pos.size), dtype=np.uint8)
+    lib().orc_inference_visibility(q_pos.size, _ptr(q_pos), k_pos.size, _ptr(k_pos),
+                                   int(prompt_len), int(D), int(bool(full)), _ptr(out))
+    return out.astype(bool)
 
 
 # -------------------------------------------------------------- attention
 
-
 def masked_attention(q, k, v, visible) -> np.ndarray:
-    """softmax(q k^T / sqrt(d)) v, blocked pairs at -inf before the softmax
-    (technical review eq. (3); v2 digest "Attention Mask Design")."""
-    q = np.asarray(q, dtype=np.float64)
-    k = np.asarray(k, dtype=np.float64)
-    v = np.asarray(v, dtype=np.float64)
-    s = q @ k.T / np.sqrt(q.shape[-1])
-    s = np.where(visible, s, -np.inf)
-    s = s - s.max(axis=1, keepdims=True)
-    p = np.exp(s)
-    p = p / p.sum(axis=1, keepdims=True)
-    return p @ v
-
-
-def attention_step(q, k_pre, v_pre, len_pre, prompt_len, k_blk, v_blk, q_off,
-                   k_suf=None, v_suf=None, len_suf=None) -> np.ndarray:
-    """Attention output of the active unit's queries, fp64, [B, q_len, Hq, d].
-
-    Keys of sequence b = prefix cache rows [0, len_pre[b]) followed by the D
-    block rows (and, for DualCache, the suffix cache rows [0, len_suf[b])).
-    Absolute positions: prefix 0..Lp-1, block Lp..Lp+D-1, suffix after it.
-    Query r of the unit sits at position Lp + q_off + r.  With a suffix the
-    mask is full attention, otherwise block-causal.
-    """
-    B, q_len, Hq, d = q.shape
-    Hkv = k_pre.shape[1]
-    D = k_blk.shape[2]
-    group = Hq // Hkv
-    dual = k_suf is not None
-    out = np.empty((B, q_len, Hq, d), dtype=np.float64)
-    for b in range(B):
-        Lp = int(len_pre[b])
-        Ls = int(len_suf[b]) if dual else 0
-        k_pos = np.arange(Lp + D + Ls)
-        q_pos = Lp + q_off + np.arange(q_len)
-        vis = inference_visibility(q_pos, k_pos, int(prompt_len[b]), D, full=dual)
-        for h in range(Hq):
-            kvh = h // group
-            parts_k = [k_pre[b, kvh, :Lp], k_blk[b, kvh]]
-            parts_v = [v_pre[b, kvh, :Lp], v_blk[b, kvh]]
-            if dual:
-                parts_k.append(k_suf[b, kvh, :Ls])
-                parts_v.append(v_suf[b, kvh, :Ls])
-            K = np.concatenate(parts_k, axis=0)
-            Vv = np.concatenate(parts_v, axis=0)
-            out[b, :, h, :] = masked_attention(q[b, :, h, :], K, Vv, vis)
+    """softmax(q k^T / sqrt(d)) v over an explicit visibility mask."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    vis = np.ascontiguousarray(np.broadcast_to(np.asarray(visible, dtype=bool),
+                                               (q.shape[0], k.shape[0]))).astype(np.uint8)
+    out = np.empty((q.shape[0], q.shape[1]), dtype=np.float64)
+    lib().orc_masked_attention(q.shape[0], k.shape[0], q.shape[1], _ptr(q), _ptr(k),
+                               _ptr(v), _ptr(vis), _ptr(out))
     return out
 
 
-def prefixcache_attention(q, k_pre, v_pre, len_pre, k_fresh, v_fresh) -> np.ndarray:
-    """PrefixCache attention of v1 (technical review, section 3 and
-    Algorithm 1, the PrefixCache branch), fp64, [B, n, Hq, d].
+def attention_step(q, k_pre, v_pre, len_pre, prompt_len, k_blk, v_blk, q_off,
+                   k_suf=None, v_suf=None, len_suf=None, threads: int = 0) -> np.ndarray:
+    """Attention of the active unit's queries, fp64, [B, q_len, Hq, d]."""
+    (q, k_pre, v_pre, k_blk, v_blk, k_suf, v_suf), code = _same_stored(
+        q, k_pre, v_pre, k_blk, v_blk, k_suf, v_suf)
+    B, q_len, Hq, d = q.shape
+    Hkv, cap_pre, D = k_pre.shape[1], k_pre.shape[2], k_blk.shape[2]
+    cap_suf = 0 if k_suf is None else k_suf.shape[2]
+    lp, pl = _i64(len_pre), _i64(prompt_len)
+    ls = None if len_suf is None else _i64(len_suf)
+    out = np.empty((B, q_len, Hq, d), dtype=np.float64)
+    lib().orc_attention_step(B, q_len, Hq, Hkv, d, D, cap_pre, cap_suf, int(q_off), code,
+                             _ptr(q), _ptr(k_pre), _ptr(v_pre), _ptr(lp), _ptr(pl),
+                             _ptr(k_blk), _ptr(v_blk), _ptr(k_suf), _ptr(v_suf), _ptr(ls),
+                             _ptr(out), threads)
+    return out
 
-    Only the prompt and the finished answer prefix are cached; the active
-    block and the still-masked suffix after it (n positions in all) are
-    recomputed every step.  Their queries attend, with full (bidirectional)
-    attention, to the cached prefix rows [0, len_pre[b]) followed by the n
-    recomputed rows' own fresh K/V.
-    """
+
+def prefixcache_attention(q, k_pre, v_pre, len_pre, k_fresh, v_fresh,
+                          threads: int = 0) -> np.ndarray:
+    """PrefixCache attention (technical review, section 3), fp64, [B, n, Hq, d]."""
+    (q, k_pre, v_pre, k_fresh, v_fresh), code = _same_stored(q, k_pre, v_pre, k_fresh,
+                                                              v_fresh)
     B, n, Hq, d = q.shape
-    Hkv = k_pre.shape[1]
-    group = Hq // Hkv
+    Hkv, cap_pre = k_pre.shape[1], k_pre.shape[2]
+    lp = _i64(len_pre)
     out = np.empty((B, n, Hq, d), dtype=np.float64)
-    for b in range(B):
-        Lp = int(len_pre[b])
-        vis = np.ones((n, Lp + n), dtype=bool)
-        for h in range(Hq):
-            kvh = h // group
-            K = np.concatenate([k_pre[b, kvh, :Lp], k_fresh[b, kvh]], axis=0)
-            Vv = np.concatenate([v_pre[b, kvh, :Lp], v_fresh[b, kvh]], axis=0)
-            out[b, :, h, :] = masked_attention(q[b, :, h, :], K, Vv, vis)
+    lib().orc_prefixcache_attention(B, n, Hq, Hkv, d, cap_pre, code, _ptr(q), _ptr(k_pre),
+                                    _ptr(v_pre), _ptr(lp), _ptr(k_fresh), _ptr(v_fresh),
+                                    _ptr(out), threads)
     return out
 
 
 # ------------------------------------------------------- LM head + commit
 
-
 def shifted_rows(src, h_prev, shift: int) -> np.ndarray:
-    """LM-head input row for each unit position (v2 digest, section 3.4
-    Step 5): position q_off + i is predicted from the hidden state at the
-    position before it.  ``src`` is [B, q_len, H]; with shift the first row
-    comes from ``h_prev`` [B, H]."""
-    src = np.asarray(src)
-    if not shift:
-        return src.copy()
-    rows = np.empty_like(src)
-    rows[:, 0] = h_prev
-    rows[:, 1:] = src[:, :-1]
-    return rows
+    """LM-head input rows with the token shift (v2 digest, Step 5)."""
+    src = _f64(src)
+    B, q_len, H = src.shape
+    hp = _f64(h_prev) if shift else None
+    out = np.empty_like(src)
+    lib().orc_shifted_rows(B, q_len, H, int(shift), _ptr(src), _ptr(hp), _ptr(out))
+    return out
 
 
-def lmhead_confidence(rows, w, chunk: int = 8192):
-    """Greedy prediction and its confidence for each row (v2 digest, Level 2;
-    technical review, section 4, Algorithm 2).
+def lmhead_confidence(rows, w, threads: int = 0):
+    """(argmax token, confidence, top-1 minus top-2 logit gap) of each row
+    over the full vocabulary; ``w`` [V, H] as stored."""
+    rows = _f64(rows)
+    R, H = rows.shape
+    w_arr, w_code = _stored(w)
+    V = w_arr.shape[0]
+    tok = np.empty(R, dtype=np.int64)
+    conf = np.empty(R, dtype=np.float64)
+    gap = np.empty(R, dtype=np.float64)
+    lib().orc_lmhead_confidence(R, V, H, _ptr(rows), _ptr(w_arr), w_code, _ptr(tok),
+                                _ptr(conf), _ptr(gap), threads)
+    return tok, conf, gap
 
-    logits l = W h over the full vocabulary; token = argmax l (lowest index
-    on a tie, numpy's argmax); confidence = the probability softmax(l) gives
-    that token = 1 / sum_v exp(l_v - l_max).  Also returns the top-1 minus
-    top-2 logit gap (a decision margin for the tests).
-    """
-    rows = np.asarray(rows, dtype=np.float64)
-    R = rows.shape[0]
-    V = w.shape[0]
-    logits = np.empty((R, V), dtype=np.float64)
-    for c0 in range(0, V, chunk):
-        c1 = min(V, c0 + chunk)
-        logits[:, c0:c1] = rows @ np.asarray(w[c0:c1], dtype=np.float64).T
-    tok = logits.argmax(axis=1)
-    lmax = logits[np.arange(R), tok]
-    conf = 1.0 / np.exp(logits - lmax[:, None]).sum(axis=1)
-    second = np.partition(logits, V - 2, axis=1)[:, V - 2] if V > 1 else lmax
-    return tok.astype(np.int64), conf, lmax - second
+
+def _select(rule: int, param: float, masked_positions, conf_of):
+    M = [int(p) for p in masked_positions]
+    if not M:
+        return []
+    conf = np.zeros(max(M) + 1, dtype=np.float64)
+    for p in M:
+        conf[p] = float(conf_of(p))
+    m = np.asarray(M, dtype=np.int32)
+    out = np.empty(len(M), dtype=np.int32)
+    n = lib().orc_select(rule, float(param), len(M), _ptr(m), _ptr(conf), _ptr(out))
+    return out[:n].tolist()
 
 
 def threshold_select(masked_positions, conf_of, tau: float):
-    """Technical review Algorithm 2: S = {i in M : c_i >= tau}; if S is empty
-    (and M is not), S = {the position with maximum c_i}.  Ties in the
-    fallback go to the lowest position."""
-    M = list(masked_positions)
-    S = [p for p in M if conf_of(p) >= tau]
-    if not S and M:
-        best = M[0]
-        for p in M[1:]:
-            if conf_of(p) > conf_of(best):
-                best = p
-        S = [best]
-    return S
+    """Technical review Algorithm 2 over a list of masked positions."""
+    return _select(RULE_THRESHOLD, tau, masked_positions, conf_of)
 
 
-def threshold_commit(block_tokens, conf, tok, q_off: int, q_len: int,
-                     mask_id: int, tau: float):
-    """Commit step over the active unit [q_off, q_off + q_len) of each block.
+def factor_select(masked_positions, conf_of, f: float):
+    """Technical review eq. (13) with Algorithm 3."""
+    return _select(RULE_FACTOR, f, masked_positions, conf_of)
 
-    Candidates are the unit's positions still holding the mask token (v2
-    digest Level 1: undecoded positions hold the mask token).  The sub-block is the
-    thresholding unit (v2 digest, "Sub-block size as a decoding granularity
-    knob").  conf / tok are [B, q_len], indexed by unit position.
-    Returns new block tokens, the committed bitmap over the whole block,
-    the commit count and the masked count left in the unit.
-    """
-    bt = np.array(block_tokens, dtype=np.int64)
-    B, D = bt.shape
-    new = bt.copy()
-    committed = np.zeros((B, D), dtype=np.uint8)
-    n_comm = np.zeros(B, dtype=np.int64)
-    n_left = np.zeros(B, dtype=np.int64)
-    for b in range(B):
-        M = [p for p in range(q_off, q_off + q_len) if bt[b, p] == mask_id]
-        S = threshold_select(M, lambda p: conf[b, p - q_off], tau)
-        for p in S:
-            new[b, p] = tok[b, p - q_off]
-            committed[b, p] = 1
-        n_comm[b] = len(S)
-        n_left[b] = sum(1 for p in range(q_off, q_off + q_len) if new[b, p] == mask_id)
-    return new, committed, n_comm, n_left
+
+def budget_select(masked_positions, conf_of):
+    """Selection by the heterogeneous error budget of eq. (9)."""
+    return _select(RULE_BUDGET, 0.0, masked_positions, conf_of)
+
+
+def budget_ok(eps) -> bool:
+    """Eq. (9): sum_j eps_j + max_j eps_j < 1."""
+    e = _f64(eps).ravel()
+    return bool(lib().orc_budget_ok(e.size, _ptr(e)))
 
 
 def select_commit(block_tokens, conf, tok, q_off: int, q_len: int, mask_id: int,
-                  select):
-    """Commit step with any selection rule ``select(masked, conf_of)`` over
-    the unit's still-masked positions (technical review, Algorithms 2 and 3;
-    eq. 9).  Same outputs as ``threshold_commit``."""
-    bt = np.array(block_tokens, dtype=np.int64)
+                  rule: int = RULE_THRESHOLD, param: float = 0.0):
+    """Commit over the active unit of every block with a selection rule
+    (RULE_THRESHOLD with tau, RULE_FACTOR with f, RULE_BUDGET).  Returns the new
+    block tokens, the committed bitmap, the commit counts and the masked counts
+    left in the unit."""
+    bt = _i64(block_tokens)
     B, D = bt.shape
-    new = bt.copy()
-    committed = np.zeros((B, D), dtype=np.uint8)
-    n_comm = np.zeros(B, dtype=np.int64)
-    n_left = np.zeros(B, dtype=np.int64)
-    for b in range(B):
-        M = [p for p in range(q_off, q_off + q_len) if bt[b, p] == mask_id]
-        S = select(M, lambda p: conf[b, p - q_off]) if M else []
-        for p in S:
-            new[b, p] = tok[b, p - q_off]
-            committed[b, p] = 1
-        n_comm[b] = len(S)
-        n_left[b] = sum(1 for p in range(q_off, q_off + q_len) if new[b, p] == mask_id)
+    c, t = _f64(conf), _i64(tok)
+    new = np.empty_like(bt)
+    committed = np.empty((B, D), dtype=np.uint8)
+    n_comm = np.empty(B, dtype=np.int64)
+    n_left = np.empty(B, dtype=np.int64)
+    lib().orc_commit(B, D, int(q_off), int(q_len), int(mask_id), int(rule), float(param),
+                     _ptr(bt), _ptr(c), _ptr(t), _ptr(new), _ptr(committed), _ptr(n_comm),
+                     _ptr(n_left))
     return new, committed, n_comm, n_left
 
 
-def lmhead_stage(rows, w, active, tau=None):
+def threshold_commit(block_tokens, conf, tok, q_off: int, q_len: int, mask_id: int,
+                     tau: float):
+    """Technical review Algorithm 2 over the active unit of every block."""
+    return select_commit(block_tokens, conf, tok, q_off, q_len, mask_id,
+                         RULE_THRESHOLD, tau)
+
+
+def lmhead_stage(rows, w, active):
     """LM-head stage outputs as the library reports them: rows whose target
     position is not masked get conf = -1 and tok = -1."""
+    rows = _f64(rows)
     B, q_len, H = rows.shape
     tok, conf, gap = lmhead_confidence(rows.reshape(B * q_len, H), w)
-    tok = tok.reshape(B, q_len)
-    conf = conf.reshape(B, q_len)
-    gap = gap.reshape(B, q_len)
     active = np.asarray(active, dtype=bool)
-    return (np.where(active, conf, -1.0), np.where(active, tok, -1), gap)
+    return (np.where(active, conf.reshape(B, q_len), -1.0),
+            np.where(active, tok.reshape(B, q_len), -1), gap.reshape(B, q_len))
 
 
 def denoise_step(c: dict, q, k_pre, v_pre, len_pre, prompt_len, k_blk, v_blk,
                  hidden, h_prev, w_lm, block_tokens, k_suf=None, v_suf=None,
-                 len_suf=None) -> dict:
-    """One denoising step of the active unit, written from its definition.
+                 len_suf=None, threads: int = 0, previous: dict = None,
+                 redo_q=None, redo_lm=None) -> dict:
+    """One denoising step of the active unit (``orc_denoise_step``).
 
-    1. attention of the unit's queries over prefix (+ suffix) cache and block;
-    2. that output rounded to the storage dtype;
-    3. LM-head rows: ``hidden`` if given, else the attention output (the
-       single-layer chaining), then the token shift;
-    4. full-vocabulary argmax and confidence;
-    5. the threshold commit (tau as float32).
-    Also returns the decision margins the parity tests rely on.
+    Tensors may be numpy arrays or CPU torch tensors, as stored.  With
+    ``previous`` (an earlier result on the same case) and the [B, q_len] flags
+    ``redo_q`` / ``redo_lm``, only the flagged attention query rows and LM-head
+    rows are recomputed; the result equals a full call (every row is
+    independent of the others).
     """
-    dtype = c["dtype"]
-    q_off, q_len, mask_id = int(c["q_off"]), int(c["q_len"]), int(c["mask_id"])
-    tau = float(np.float32(c["tau"]))
-    attn = attention_step(q, k_pre, v_pre, len_pre, prompt_len, k_blk, v_blk,
-                          q_off, k_suf, v_suf, len_suf)
-    attn_r = round_to(attn, dtype)
-    B = attn.shape[0]
-    src = attn_r.reshape(B, q_len, -1) if hidden is None else np.asarray(hidden, np.float64)
-    rows = shifted_rows(src, None if h_prev is None else np.asarray(h_prev, np.float64),
-                        int(c["shift"]))
-    bt = np.asarray(block_tokens)
-    active = bt[:, q_off:q_off + q_len] == mask_id
-    conf, tok, gap = lmhead_stage(rows, w_lm, active)
-    new, committed, n_comm, n_left = threshold_commit(bt, conf, tok, q_off, q_len,
-                                                      mask_id, tau)
-    # Decision margins: logit gap and |conf - tau| per active row; the
-    # relative confidence gap between the two best candidates where the
-    # fallback fires.
-    cand_gap = np.full(B, np.inf)
-    for b in range(B):
-        cs = sorted(conf[b][active[b]], reverse=True)
-        if len(cs) >= 2 and cs[0] < tau:
-            cand_gap[b] = (cs[0] - cs[1]) / cs[0]
-    return dict(attn=attn, attn_rounded=attn_r, rows=rows, active=active,
-                conf=conf, tok=tok, logit_gap=gap, block_tokens=new,
-                committed=committed, n_committed=n_comm, n_masked_left=n_left,
-                tau=tau, cand_gap=cand_gap)
+    (q, k_pre, v_pre, k_blk, v_blk, k_suf, v_suf, hidden, h_prev), code = _same_stored(
+        q, k_pre, v_pre, k_blk, v_blk, k_suf, v_suf, hidden, h_prev)
+    w_arr, w_code = _stored(w_lm)
+    B, q_len, Hq, d = q.shape
+    Hkv, cap_pre, D = k_pre.shape[1], k_pre.shape[2], k_blk.shape[2]
+    cap_suf = 0 if k_suf is None else k_suf.shape[2]
+    V, H = w_arr.shape
+    cfg = StepCfg(B=B, q_len=q_len, Hq=Hq, Hkv=Hkv, d=d, D=D, q_off=int(c["q_off"]),
+                  cap_pre=cap_pre, cap_suf=cap_suf, H=H, V=V, mask_id=int(c["mask_id"]),
+                  shift=int(c["shift"]), stored=code, w_stored=w_code, threads=threads,
+                  tau=float(c["tau"]))
+    lp, pl, bt = _i64(len_pre), _i64(prompt_len), _i64(block_tokens)
+    ls = None if len_suf is None else _i64(len_suf)
+    if previous is not None:
+        attn = np.array(previous["attn"], dtype=np.float64, order="C")
+        conf = np.array(previous["conf"], dtype=np.float64, order="C")
+        tok = np.array(previous["tok"], dtype=np.int64, order="C")
+        gap = np.array(previous["logit_gap"], dtype=np.float64, order="C")
+        rq = np.ascontiguousarray(np.asarray(redo_q, dtype=np.uint8).reshape(B, q_len))
+        rl = np.ascontiguousarray(np.asarray(redo_lm, dtype=np.uint8).reshape(B, q_len))
+    else:
+        attn = np.empty((B, q_len, Hq, d), dtype=np.float64)
+        conf = np.empty((B, q_len), dtype=np.float64)
+        tok = np.empty((B, q_len), dtype=np.int64)
+        gap = np.empty((B, q_len), dtype=np.float64)
+        rq = rl = None
+    attn_r = np.empty_like(attn)
+    rows = np.empty((B, q_len, H), dtype=np.float64)
+    active = np.empty((B, q_len), dtype=np.uint8)
+    new = np.empty_like(bt)
+    committed = np.empty((B, D), dtype=np.uint8)
+    n_comm = np.empty(B, dtype=np.int64)
+    n_left = np.empty(B, dtype=np.int64)
+    cand_gap = np.empty(B, dtype=np.float64)
+    rc = lib().orc_denoise_step(
+        ctypes.byref(cfg), _ptr(q), _ptr(k_pre), _ptr(v_pre), _ptr(lp), _ptr(pl),
+        _ptr(k_blk), _ptr(v_blk), _ptr(k_suf), _ptr(v_suf), _ptr(ls), _ptr(hidden),
+        _ptr(h_prev), _ptr(w_arr), _ptr(bt), _ptr(rq), _ptr(rl), _ptr(attn), _ptr(attn_r),
+        _ptr(rows), _ptr(active), _ptr(conf), _ptr(tok), _ptr(gap), _ptr(new),
+        _ptr(committed), _ptr(n_comm), _ptr(n_left), _ptr(cand_gap))
+    if rc != 0:
+        raise ValueError("oracle rejected the step's shapes")
+    return dict(attn=attn, attn_rounded=attn_r, rows=rows, active=active.astype(bool),
+                conf=conf, tok=tok, logit_gap=gap, block_tokens=new, committed=committed,
+                n_committed=n_comm, n_masked_left=n_left, tau=float(np.float32(c["tau"])),
+                cand_gap=cand_gap)
+
+
+def library_path() -> str:
+    return os.path.abspath(lib()._name)

@@ -7,6 +7,12 @@ Parallel Tokens" (technical review): section 4 eq. (4) and the product of
 marginals; section 5 eqs. (5)-(8) (the (n+1)eps <= 1 agreement condition) and
 the eta counterexample family; section 5.1 eq. (9) (heterogeneous budget);
 section 6 eq. (13) and Algorithm 3 (factor selection).
+
+The joint-distribution mathematics (marginals, total variation, joint and
+product maximisers, the eta family) is written here in numpy: it pins the
+theorem the selection rules rest on and feeds no GPU comparison.  The
+selection rules themselves (eq. 9, eq. 13 / Algorithm 3) are evaluated by the
+C++ oracle in ``step.cc``.
 """
 from __future__ import annotations
 
@@ -14,6 +20,8 @@ import itertools
 import math
 
 import numpy as np
+
+from . import step
 
 
 def marginals(joint: np.ndarray):
@@ -76,38 +84,25 @@ def eta_family(n: int, eta: float) -> np.ndarray:
 
 
 def heterogeneous_budget_ok(eps) -> bool:
-    """Eq. (9): sum_j eps_j + max_j eps_j < 1."""
-    eps = [float(e) for e in eps]
-    return sum(eps) + max(eps) < 1.0
+    """Eq. (9): sum_j eps_j + max_j eps_j < 1 (evaluated by the C++ oracle)."""
+    return step.budget_ok(eps)
 
 
 def factor_select(masked_positions, conf_of, f: float):
     """Algorithm 3 with eq. (13): sort the masked positions by decreasing
     confidence (ties: lower position first); keep the largest n with
-    (n + 1) (1 - c_(n)) < f; if no n qualifies, the first position alone."""
-    order = sorted(masked_positions, key=lambda p: (-conf_of(p), p))
-    best = 0
-    for n in range(1, len(order) + 1):
-        if (n + 1) * (1.0 - conf_of(order[n - 1])) < f:
-            best = n
-    if best == 0:
-        return order[:1]
-    return order[:best]
+    (n + 1) (1 - c_(n)) < f; if no n qualifies, the first position alone.
+    Evaluated by the C++ oracle."""
+    return step.factor_select(masked_positions, conf_of, f)
 
 
 def budget_select(masked_positions, conf_of):
     """Selection by the heterogeneous error budget of eq. (9): sort the masked
     positions by decreasing confidence (ties: lower position first), with
     eps_j = 1 - c_j; keep the largest n whose first n positions satisfy
-    sum eps + max eps < 1; if no n qualifies, the first position alone."""
-    order = sorted(masked_positions, key=lambda p: (-conf_of(p), p))
-    best = 0
-    for n in range(1, len(order) + 1):
-        if heterogeneous_budget_ok([1.0 - conf_of(q) for q in order[:n]]):
-            best = n
-    if best == 0:
-        return order[:1]
-    return order[:best]
+    sum eps + max eps < 1; if no n qualifies, the first position alone.
+    Evaluated by the C++ oracle."""
+    return step.budget_select(masked_positions, conf_of)
 
 
 def all_assignments(n: int, k: int):

@@ -321,10 +321,8 @@ def test_select_commit_factor_and_budget(policy, f):
     n_l = torch.empty(B, dtype=torch.int32, device="cuda")
     fdl.select_commit(cfg, policy, f, torch.from_numpy(conf).cuda(), torch.from_numpy(tok).cuda(),
                       d_bt, comm, n_c, n_l)
-    from oracle import theory
-    sel = ((lambda M, c: theory.factor_select(M, c, f)) if policy == fdl.SELECT_FACTOR
-           else theory.budget_select)
-    want = step.select_commit(bt, conf.astype(np.float64), tok, q_off, q_len, mask, sel)
+    rule = step.RULE_FACTOR if policy == fdl.SELECT_FACTOR else step.RULE_BUDGET
+    want = step.select_commit(bt, conf.astype(np.float64), tok, q_off, q_len, mask, rule, f)
     assert np.array_equal(d_bt.cpu().numpy(), want[0])
     assert np.array_equal(comm.cpu().numpy(), want[1])
     assert np.array_equal(n_c.cpu().numpy(), want[2])

@@ -235,7 +235,7 @@ def test_token_shift_rows():
 def test_confidence_is_exp_of_max_minus_logsumexp():
     rows = RNG.standard_normal((5, 32))
     w = RNG.standard_normal((1000, 32)) * 0.7
-    tok, conf, gap = step.lmhead_confidence(rows, w, chunk=128)
+    tok, conf, gap = step.lmhead_confidence(rows, w)
     logits = rows @ w.T
     np.testing.assert_array_equal(tok, logits.argmax(1))
     want = np.exp(logits.max(1) - scipy.special.logsumexp(logits, axis=1))
@@ -468,7 +468,6 @@ def test_select_commit_matches_threshold_commit_for_algorithm_2():
         tok = rng.integers(0, 100, (3, 8))
         bt = np.where(rng.random((3, 16)) < 0.5, 99, rng.integers(0, 99, (3, 16)))
         a = step.threshold_commit(bt, conf, tok, 4, 8, 99, 0.7)
-        b = step.select_commit(bt, conf, tok, 4, 8, 99,
-                               lambda M, cf: step.threshold_select(M, cf, 0.7))
+        b = step.select_commit(bt, conf, tok, 4, 8, 99, step.RULE_THRESHOLD, 0.7)
         for x, y in zip(a, b):
             assert np.array_equal(x, y)
