@@ -144,6 +144,29 @@ def oracle_baseline(case, min_seconds: float = 10.0, max_steps: int = 50) -> dic
                               "sample": "one whole oracle step on one thread"}}
 
 
+# ------------------------------------------------------------ timing helpers
+
+def rounds_us(timed, fn, k: int, reps: int, world: int) -> list:
+    """Per-launch microseconds of ``reps`` timed regions of ``k`` launches
+    each (every region the max over ranks)."""
+    return [max_over_ranks(timed(fn, k), world) / k * 1e6 for _ in range(reps)]
+
+
+def spread(us: list) -> dict:
+    """Median and range of repeated timings."""
+    return {"median": statistics.median(us), "min": min(us), "max": max(us),
+            "rounds": len(us)}
+
+
+def kv_copies_for(torch, bytes_per_copy: int, lo: int = 2, hi: int = 64) -> int:
+    """How many copies of a KV input to rotate over so that the bytes read in
+    one pass over all copies exceed twice the L2 (the reads then come from
+    HBM)."""
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    need = -(-2 * l2 // max(1, bytes_per_copy))
+    return int(min(hi, max(lo, need)))
+
+
 # ------------------------------------------------------------------- main
 
 def parse():
@@ -155,6 +178,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=1002)
     ap.add_argument("--kv-copies", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the sweep, the other workloads and the block-decode grid")
     return ap.parse_args()
 
 
@@ -320,7 +345,10 @@ def main():
 
     with ClockSampler(_gpu_id(torch)) as clocks:
         t_step = timed(lambda i: step(sets[i % n_copies]), args.steps)
-    t_step = max_over_ranks(t_step, world)
+        t_step = max_over_ranks(t_step, world)
+        # two more rounds of the same K steps, for the spread
+        step_rounds = [t_step / args.steps * 1e6] + rounds_us(
+            timed, lambda i: step(sets[i % n_copies]), args.steps, 2, world)
     ms_per_step = t_step / args.steps * 1e3
     pos = world * B * q_len * args.steps
     value = pos / t_step
@@ -332,14 +360,16 @@ def main():
                                          ws, stream)
     for i in range(3):
         lm(i)
-    t_lm = max_over_ranks(timed(lm, args.steps), world) / args.steps
+    lm_rounds = rounds_us(timed, lm, args.steps, 3, world)
+    t_lm = statistics.median(lm_rounds) * 1e-6
     attn = lambda i: fdl.block_attn(cfg, sets[i % n_copies]["q"], sets[i % n_copies]["k_pre"],
                                     sets[i % n_copies]["v_pre"], sets[i % n_copies]["len_pre"],
                                     sets[i % n_copies]["k_blk"], sets[i % n_copies]["v_blk"],
                                     out["attn"], ws, stream)
     for i in range(3):
         attn(i)
-    t_attn = max_over_ranks(timed(attn, args.steps), world) / args.steps
+    attn_rounds = rounds_us(timed, attn, args.steps, 3, world)
+    t_attn = statistics.median(attn_rounds) * 1e-6
     pc = prefixcache_leg(torch, fdl, stream, timed, world, args.steps, peaks)
     try:
         blk = block_decode_leg(torch, fdl, c_run, sets[0], w, stream, world)
@@ -352,6 +382,13 @@ def main():
         blk["positions_per_s_graph"] = c["batch"] * c["block_size"] / (
             blk["graph_us_per_block"] * 1e-6)
     lm_big = large_batch_lm_leg(torch, fdl, synth, stream, timed, world, args.steps, peaks)
+    sweep = others = grid = None
+    if not args.no_sweep:
+        sweep = sweep_leg(torch, fdl, synth, stream, timed, world, args.steps, peaks, w,
+                          rank_seed(args.seed, rank))
+        others = configs_leg(torch, fdl, synth, stream, timed, world, args.steps, peaks,
+                             rank_seed(args.seed, rank))
+        grid = block_decode_grid(torch, fdl, c_run, sets[0], w, stream, world)
 
     # End to end through the public API: per step, pinned host inputs copied
     # in, the step, and its results copied out and read on the host.
@@ -461,14 +498,20 @@ def main():
                      "frac": lm_gbs / peaks["hbm_gbs"],
                      "peak_source": f"{peaks['source']} hbm_gbs (burst copy)",
                      "traffic": traffic, "bytes_per_launch": lm_bytes,
-                     "us_per_launch": t_lm * 1e6},
+                     "us_per_launch": t_lm * 1e6, "us_rounds": spread(lm_rounds)},
+        "step_us_rounds": spread(step_rounds),
         "attention": {"us_per_launch": t_attn * 1e6, "bytes_per_launch": attn_bytes,
-                      "achieved_gbs": attn_bytes / t_attn / 1e9},
+                      "achieved_gbs": attn_bytes / t_attn / 1e9,
+                      "frac_hbm": attn_bytes / t_attn / 1e9 / peaks["hbm_gbs"],
+                      "us_rounds": spread(attn_rounds)},
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": step_bytes / (t_step / args.steps) / 1e9,
                           "frac": step_bytes / (t_step / args.steps) / 1e9 / peaks["hbm_gbs"]},
         "prefixcache": pc,
         "block_decode": blk,
         "lmhead_large_batch": lm_big,
+        "sweep": sweep,
+        "other_workloads": others,
+        "block_decode_grid": grid,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e / args.steps * 1e3,
                 "upload": "double-buffered: step i+1's inputs copied on a second stream "
@@ -606,6 +649,36 @@ def block_decode_leg(torch, fdl, c, x, w, stream, world, blocks: int = 5) -> dic
             "positions_per_s_graph": B * D / (t_graph * 1e-3)}
 
 
+def block_decode_grid(torch, fdl, c, x, w8, stream, world, blocks: int = 3) -> list:
+    """The block decode at tau {0.7, 0.9, 1.0} x logit scale {4, 8, 12}:
+    steps per block, committed tokens per step per sequence (D / steps, the
+    pages' tokens-per-step figure) and the block time from the graph and from
+    the host loop.  tau = 1.0 disables parallel decoding (one token per
+    step unless an fp32 confidence rounds up to exactly 1)."""
+    out = []
+    D = c["block_size"]
+    for sc in SWEEP_SCALE:
+        w = _scaled_weight(torch, w8, sc)
+        for tau in (0.7, 0.9, 1.0):
+            try:
+                r = block_decode_leg(torch, fdl, dict(c, tau=tau), x, w, stream, world,
+                                     blocks=blocks)
+            except Exception as e:  # reported; every rank still reduces below
+                r = {"error": f"{type(e).__name__}: {e}"}
+            for k in ("graph_us_per_block", "host_loop_us_per_block"):
+                r[k] = max_over_ranks(float(r.get(k, float("nan"))), world)
+            n = r.get("steps_per_block", 0)
+            out.append({"tau": tau, "scale": sc, "steps_per_block": n,
+                        "steps_per_sub_block": r.get("steps_per_sub_block"),
+                        "tokens_per_step_per_sequence": D / n if n else None,
+                        "graph_us_per_block": r["graph_us_per_block"],
+                        "host_loop_us_per_block": r["host_loop_us_per_block"],
+                        "block_decoded": r.get("block_decoded"),
+                        **({"error": r["error"]} if "error" in r else {})})
+        del w
+    return out
+
+
 PREFIXCACHE = dict(batch=1, n_q_heads=32, n_kv_heads=32, head_dim=128, prefix=768, rows=768)
 
 
@@ -674,6 +747,250 @@ def large_batch_lm_leg(torch, fdl, synth, stream, timed, world, steps, peaks) ->
     return {"workload": "Qwen2.5-7B vocabulary, 512 rows (64 x 8), 2 passes",
             "us_per_launch": t * 1e6, "flops": flops, "bound": "tensor",
             "tflops": flops / t / 1e12, "frac_tensor": flops / t / 1e12 / peaks["bf16_tflops"]}
+
+
+SWEEP_BATCH = (1, 4, 16)
+SWEEP_PREFIX = (2048, 8192)
+SWEEP_SCALE = (4.0, 8.0, 12.0)
+
+
+def _scaled_weight(torch, w8, scale: float):
+    """The Qwen2.5-7B LM-head weight at another logit scale: the scale-8
+    draw times scale / 8, rounded to bf16 (layout-independent, so it applies
+    to the tiled copy as is)."""
+    if scale == 8.0:
+        return w8
+    out = torch.empty_like(w8)
+    step_rows = 8192
+    for r0 in range(0, w8.shape[0], step_rows):
+        out[r0:r0 + step_rows] = (w8[r0:r0 + step_rows].float() * (scale / 8.0)).to(w8.dtype)
+    return out
+
+
+def _attn_bytes(c, len_pre, len_suf=None) -> int:
+    """Algorithmic bytes of the attention: K and V of every visible key once
+    (prefix + block + suffix, per KV head), Q in and O out."""
+    B, q_len, D = c["batch"], c["q_len"], c["block_size"]
+    keys = int(len_pre.sum()) + B * D + (0 if len_suf is None else int(len_suf.sum()))
+    return (keys * c["n_kv_heads"] * 2 * c["head_dim"] * 2
+            + 2 * B * q_len * c["n_q_heads"] * c["head_dim"] * 2)
+
+
+def _lm_bytes_flops(c) -> tuple:
+    R, H, V = c["batch"] * c["q_len"], c["hidden"], c["vocab"]
+    return V * H * 2 + R * H * 2 + R * 8, 2.0 * V * H * R
+
+
+def _device_inputs(torch, case, stream, copies: int):
+    """The case's step inputs on the device, with ``copies`` distinct copies
+    of the KV caches (the attention reads rotate over them)."""
+    dev = lambda t: None if t is None else t.cuda().contiguous()
+    with torch.cuda.stream(stream):
+        base = dict(q=dev(case.q), len_pre=dev(case.len_pre), k_blk=dev(case.k_blk),
+                    v_blk=dev(case.v_blk), hidden=dev(case.hidden), h_prev=dev(case.h_prev),
+                    len_suf=dev(case.len_suf), bt0=dev(case.block_tokens))
+        kv = []
+        first = dict(k_pre=dev(case.k_pre), v_pre=dev(case.v_pre), k_suf=dev(case.k_suf),
+                     v_suf=dev(case.v_suf))
+        for i in range(copies):
+            kv.append(first if i == 0 else
+                      {k: None if v is None else v.clone() for k, v in first.items()})
+        base["bt"] = base["bt0"].clone()
+    return base, kv
+
+
+def _step_outputs(torch, c):
+    B, q_len, D = c["batch"], c["q_len"], c["block_size"]
+    return dict(conf=torch.empty((B, q_len), dtype=torch.float32, device="cuda"),
+                tok=torch.empty((B, q_len), dtype=torch.int32, device="cuda"),
+                comm=torch.empty((B, D), dtype=torch.uint8, device="cuda"),
+                n_c=torch.empty(B, dtype=torch.int32, device="cuda"),
+                n_l=torch.empty(B, dtype=torch.int32, device="cuda"))
+
+
+def sweep_leg(torch, fdl, synth, stream, timed, world, steps, peaks, w8, seed,
+              reps: int = 3) -> dict:
+    """Long-context sweep at Qwen2.5-7B shapes: batch {1, 4, 16} x prefix
+    {2048, 8192} x logit scale {4, 8, 12}.  Per (batch, prefix): the
+    attention entry point alone (algorithmic bytes, GB/s, fraction of the
+    measured HBM bandwidth); per batch: the LM head alone against its roofline
+    (the slower of its weight bytes at HBM bandwidth and its FLOPs at the
+    tensor peak); per point: the fused step and the tokens one step commits
+    from the case's block state.  KV caches rotate over enough copies to
+    exceed twice the L2; every timing is ``reps`` rounds of ``steps``
+    launches (median and range)."""
+    hbm = peaks["hbm_gbs"] * 1e9
+    tens = peaks["bf16_tflops"] * 1e12
+    weights = {sc: _scaled_weight(torch, w8, sc) for sc in SWEEP_SCALE}
+    lm_by_batch, points = {}, []
+    for B in SWEEP_BATCH:
+        for P in SWEEP_PREFIX:
+            case = synth.make_case("sweep", seed, cfg=synth.sweep_config(B, P, 8.0),
+                                   draw_w=False)
+            c = dict(case.cfg, w_layout=fdl.W_PACKED)
+            cfg = fdl.make_cfg(c)
+            Hkv, d = c["n_kv_heads"], c["head_dim"]
+            n_kv = kv_copies_for(torch, B * Hkv * P * d * 2 * 2)
+            x, kv = _device_inputs(torch, case, stream, n_kv)
+            o = _step_outputs(torch, c)
+            with torch.cuda.stream(stream):
+                attn_out = torch.empty_like(x["q"])
+                ws = fdl.workspace(cfg)
+            stream.synchronize()
+
+            def attn(i):
+                y = kv[i % n_kv]
+                fdl.block_attn(cfg, x["q"], y["k_pre"], y["v_pre"], x["len_pre"], x["k_blk"],
+                               x["v_blk"], attn_out, ws, stream)
+            for i in range(3):
+                attn(i)
+            a_us = rounds_us(timed, attn, steps, reps, world)
+            a_bytes = _attn_bytes(c, case.len_pre)
+            lm_bytes, lm_flops = _lm_bytes_flops(c)
+            if B not in lm_by_batch:
+                rows = x["hidden"].view(B * c["q_len"], c["hidden"])
+                lm = lambda i: fdl.lmhead_confidence(cfg, rows, w8, None, o["conf"], o["tok"],
+                                                     ws, stream)
+                for i in range(3):
+                    lm(i)
+                l_us = rounds_us(timed, lm, steps, reps, world)
+                t_roof = roofline_seconds(lm_bytes, lm_flops, hbm, tens)
+                lm_by_batch[B] = {"rows": B * c["q_len"], "us": spread(l_us),
+                                  "roofline_us": t_roof * 1e6,
+                                  "frac": t_roof * 1e6 / statistics.median(l_us),
+                                  "bound": "hbm" if lm_bytes / hbm >= lm_flops / tens
+                                  else "tensor"}
+            for sc in SWEEP_SCALE:
+                w = weights[sc]
+
+                def step(i):
+                    y = kv[i % n_kv]
+                    fdl.denoise_step(cfg, x["q"], y["k_pre"], y["v_pre"], x["len_pre"],
+                                     x["k_blk"], x["v_blk"], None, None, None, x["hidden"],
+                                     x["h_prev"], w, x["bt"], None, o["conf"], o["tok"],
+                                     o["comm"], o["n_c"], o["n_l"], ws, stream)
+                # tokens one step commits from the case's block state
+                with torch.cuda.stream(stream):
+                    x["bt"].copy_(x["bt0"])
+                step(0)
+                stream.synchronize()
+                n_c = o["n_c"].cpu()
+                masked = int((case.block_tokens[:, c["q_off"]:c["q_off"] + c["q_len"]]
+                              == c["mask_id"]).sum())
+                for i in range(3):
+                    step(i)
+                s_us = rounds_us(timed, step, steps, reps, world)
+                s_bytes = a_bytes + lm_bytes + (2 * B * c["q_len"] * c["hidden"] * 2)
+                points.append({
+                    "batch": B, "prefix": P, "scale": sc,
+                    "attention": {"us": spread(a_us), "bytes": a_bytes,
+                                  "gbs": a_bytes / statistics.median(a_us) / 1e3,
+                                  "frac_hbm": a_bytes / statistics.median(a_us) / 1e3
+                                  / peaks["hbm_gbs"]},
+                    "lm_head_frac": lm_by_batch[B]["frac"],
+                    "step": {"us": spread(s_us),
+                             "positions_per_s": B * c["q_len"] / statistics.median(s_us) * 1e6,
+                             "frac_hbm": s_bytes / statistics.median(s_us) / 1e3
+                             / peaks["hbm_gbs"]},
+                    "masked_in_unit": masked,
+                    "committed_per_step": int(n_c.sum()),
+                    "committed_per_sequence": (n_c.float().mean().item()),
+                    "kv_copies": n_kv})
+            assert fdl.get_status(ws, stream) == 0
+            del kv, x, o, attn_out, ws
+            torch.cuda.empty_cache()
+    del weights
+    return {"workload": "Qwen2.5-7B shapes (28/4 heads, d 128, H 3584, V 152064), "
+                        "block 32 / sub-block 8, tau 0.9, tiled LM-head weight",
+            "peak_hbm_gbs": peaks["hbm_gbs"], "peak_tflops": peaks["bf16_tflops"],
+            "lm_head": {str(b): v for b, v in lm_by_batch.items()},
+            "points": points}
+
+
+def configs_leg(torch, fdl, synth, stream, timed, world, steps, peaks, seed,
+                reps: int = 3) -> dict:
+    """The other single-GPU workloads: Qwen2.5-1.5B shapes (batch 1, prefix
+    512) and LLaDA-8B-like DualCache (prefix 768 + block 32 + suffix 736,
+    all 32 block positions queried): the fused step, the LM head and the
+    attention entry point alone, each against the measured HBM bandwidth."""
+    hbm = peaks["hbm_gbs"] * 1e9
+    tens = peaks["bf16_tflops"] * 1e12
+    res = {}
+    for name in ("qwen1.5b", "llada"):
+        case = synth.make_case(name, seed)
+        c = dict(case.cfg, w_layout=fdl.W_PACKED)
+        cfg = fdl.make_cfg(c)
+        B, Hkv, d = c["batch"], c["n_kv_heads"], c["head_dim"]
+        per_copy = B * Hkv * (c["cap_prefix"] + c["cap_suffix"]) * d * 2 * 2
+        n_kv = kv_copies_for(torch, per_copy)
+        x, kv = _device_inputs(torch, case, stream, n_kv)
+        o = _step_outputs(torch, c)
+        with torch.cuda.stream(stream):
+            w_rm = case.w_lm.cuda()
+            w = torch.empty_like(w_rm)
+            fdl.lmhead_pack_weight(cfg, w_rm, w, stream)
+            del w_rm
+            attn_out = torch.empty_like(x["q"])
+            ws = fdl.workspace(cfg)
+        stream.synchronize()
+        dual = case.k_suf is not None
+
+        def step(i):
+            y = kv[i % n_kv]
+            fdl.denoise_step(cfg, x["q"], y["k_pre"], y["v_pre"], x["len_pre"], x["k_blk"],
+                             x["v_blk"], y["k_suf"], y["v_suf"], x["len_suf"], x["hidden"],
+                             x["h_prev"], w, x["bt"], None, o["conf"], o["tok"], o["comm"],
+                             o["n_c"], o["n_l"], ws, stream)
+
+        def attn(i):
+            y = kv[i % n_kv]
+            if dual:
+                fdl.dualcache_attn(cfg, x["q"], y["k_pre"], y["v_pre"], x["len_pre"],
+                                   x["k_blk"], x["v_blk"], y["k_suf"], y["v_suf"],
+                                   x["len_suf"], attn_out, ws, stream)
+            else:
+                fdl.block_attn(cfg, x["q"], y["k_pre"], y["v_pre"], x["len_pre"], x["k_blk"],
+                               x["v_blk"], attn_out, ws, stream)
+        rows = x["hidden"].view(B * c["q_len"], c["hidden"])
+        lm = lambda i: fdl.lmhead_confidence(cfg, rows, w, None, o["conf"], o["tok"], ws,
+                                             stream)
+        out = {}
+        for key, fn in (("step", step), ("lm_head", lm), ("attention", attn)):
+            for i in range(3):
+                fn(i)
+            out[key] = rounds_us(timed, fn, steps, reps, world)
+        with torch.cuda.stream(stream):
+            x["bt"].copy_(x["bt0"])
+        step(0)
+        stream.synchronize()
+        committed = int(o["n_c"].sum().item())
+        assert fdl.get_status(ws, stream) == 0
+        a_bytes = _attn_bytes(c, case.len_pre, case.len_suf)
+        lm_bytes, lm_flops = _lm_bytes_flops(c)
+        shift_bytes = 2 * B * c["q_len"] * c["hidden"] * 2 if c["shift"] else 0
+        s_bytes = a_bytes + lm_bytes + shift_bytes
+        t_step = statistics.median(out["step"])
+        t_lm = statistics.median(out["lm_head"])
+        t_attn = statistics.median(out["attention"])
+        lm_roof = roofline_seconds(lm_bytes, lm_flops, hbm, tens) * 1e6
+        res[name] = {
+            "workload": ("Qwen2.5-1.5B shapes: batch 1, 12/2 heads, d 128, H 1536, "
+                         "V 151936, prefix 512, block 32 / sub-block 8, tau 0.9"
+                         if name == "qwen1.5b" else
+                         "LLaDA-8B-like DualCache: batch 1, 32/32 heads, d 128, H 4096, "
+                         "V 126464, prefix 768 + block 32 + suffix 736, tau 0.9"),
+            "step": {"us": spread(out["step"]), "bytes": s_bytes,
+                     "positions_per_s": B * c["q_len"] / t_step * 1e6,
+                     "frac_hbm": s_bytes / t_step / 1e3 / peaks["hbm_gbs"]},
+            "lm_head": {"us": spread(out["lm_head"]), "bytes": lm_bytes,
+                        "roofline_us": lm_roof, "frac": lm_roof / t_lm},
+            "attention": {"us": spread(out["attention"]), "bytes": a_bytes,
+                          "gbs": a_bytes / t_attn / 1e3,
+                          "frac_hbm": a_bytes / t_attn / 1e3 / peaks["hbm_gbs"]},
+            "committed_first_step": committed, "kv_copies": n_kv}
+        del kv, x, o, w, attn_out, ws
+        torch.cuda.empty_cache()
+    return res
 
 
 def _gpu_id(torch) -> str:

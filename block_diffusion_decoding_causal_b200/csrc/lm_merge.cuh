@@ -24,11 +24,17 @@ __device__ __forceinline__ bool last_cta_arrives(unsigned int* ticket,
 // is the fused step, commit (technical review, section 4, Algorithm 2).
 // conf = 1 / sum_v exp(l_v - l_max) is the max softmax probability; the
 // token is the argmax with the lowest vocabulary index on a tie.
+// If a CTA's bounded wait ran out (FDL_DEV_TIMEOUT in the status word, set
+// before its ticket), its partials are stale: every row then reports
+// conf = -1 and tok = -1 and the commit selects nothing (block tokens kept,
+// counts written), until the caller reads and clears the status word.
 __device__ __forceinline__ void lm_final_merge(const LmArgs& a) {
   __shared__ float s_conf[kMaxRows];
   __shared__ int s_tok[kMaxRows];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = blockDim.x >> 5;
+  const bool timed_out =
+      (*reinterpret_cast<volatile unsigned int*>(&a.ctrl->status) & FDL_DEV_TIMEOUT) != 0u;
   for (int r = warp; r < a.R; r += nw) {
     MSI st = msi_empty();
     for (int c = lane; c < a.n_cta; c += 32) {
@@ -43,6 +49,7 @@ __device__ __forceinline__ void lm_final_merge(const LmArgs& a) {
         const int b = r / a.q_len, i = r % a.q_len;
         act = a.block_tokens_in[(size_t)b * a.D + a.q_off + i] == a.mask_id;
       }
+      act = act && !timed_out;
       const float c = act ? 1.0f / st.s : -1.0f;
       const int t = act ? st.i : -1;
       a.conf[r] = c;
@@ -55,6 +62,12 @@ __device__ __forceinline__ void lm_final_merge(const LmArgs& a) {
   __syncthreads();
   for (int b = warp; b < a.B; b += nw) {
     const int base = b * a.q_len;
+    if (timed_out) {
+      apply_selection_warp(b, lane, a.D, a.q_off, a.q_len, a.mask_id, 0u,
+                           [&](int i) { return s_tok[base + i]; }, a.block_tokens,
+                           a.committed, a.n_committed, a.n_masked_left);
+      continue;
+    }
     commit_sequence_warp(
         b, lane, a.D, a.q_off, a.q_len, a.mask_id, a.tau,
         [&](int i) { return s_conf[base + i]; },

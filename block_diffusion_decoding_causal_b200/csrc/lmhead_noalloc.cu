@@ -17,11 +17,15 @@
 namespace fdl {
 namespace {
 
-constexpr int kStaticMaxRows = 128;           // B * q_len
-constexpr int kStaticMaxCtas = 2 * kPlanCTAs;  // CUDA-core plan uses up to 296
+constexpr int kStaticMaxRows = FDL_NOALLOC_MAX_ROWS;  // B * q_len
+constexpr int kStaticMaxCtas = 2 * kPlanCTAs;         // CUDA-core plan uses up to 296
 constexpr size_t kStaticControl = 256;
 constexpr size_t kStaticBytes =
-    kStaticControl + sizeof(Partial) * (size_t)kStaticMaxCtas * kStaticMaxRows;  // 606,464 B
+    kStaticControl + sizeof(Partial) * (size_t)kStaticMaxCtas * kStaticMaxRows;
+// The header states both limits as numbers; keep them tied to the code.
+static_assert(kStaticBytes == FDL_NOALLOC_SCRATCH_BYTES,
+              "FDL_NOALLOC_SCRATCH_BYTES in fdl.h must match the static scratch");
+static_assert(sizeof(Control) <= kStaticControl, "control words exceed their slot");
 
 // The scratch itself.  In host code this name is only a stand-in for the
 // symbol, never a device address: the address is looked up per device below.
@@ -31,9 +35,10 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch[kMaxDevices] = {};
 
-// Device address of the scratch on the current device; the first call on a
-// device looks it up and zeroes the control words (synchronously).
-cudaError_t static_scratch(void** out) {
+// Device address of the scratch on the current device.  The first call on a
+// device looks it up and queues the zeroing of the control words on `stream`,
+// ahead of whatever the caller launches next on that stream.
+cudaError_t static_scratch(cudaStream_t stream, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -43,7 +48,7 @@ cudaError_t static_scratch(void** out) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_lm_scratch);
     if (e != cudaSuccess) return e;
-    e = cudaMemset(p, 0, kStaticControl);
+    e = cudaMemsetAsync(p, 0, kStaticControl, stream);
     if (e != cudaSuccess) return e;
     g_scratch[dev] = p;
   }
@@ -52,6 +57,8 @@ cudaError_t static_scratch(void** out) {
 }
 
 }  // namespace
+
+constexpr size_t kStaticControlSize = kStaticControl;
 
 // Sizes the static scratch can serve; fills `why` otherwise.
 int lmhead_static_check(const Plan& p, const fdl_step_cfg& c, std::string* why) {
@@ -68,9 +75,9 @@ int lmhead_static_check(const Plan& p, const fdl_step_cfg& c, std::string* why) 
   return FDL_OK;
 }
 
-cudaError_t lmhead_static_workspace(Control** ctrl, Partial** part) {
+cudaError_t lmhead_static_workspace(cudaStream_t stream, Control** ctrl, Partial** part) {
   void* p = nullptr;
-  cudaError_t e = static_scratch(&p);
+  cudaError_t e = static_scratch(stream, &p);
   if (e != cudaSuccess) return e;
   *ctrl = static_cast<Control*>(p);
   *part = reinterpret_cast<Partial*>(static_cast<unsigned char*>(p) + kStaticControl);
@@ -82,6 +89,7 @@ cudaError_t lmhead_static_workspace(Control** ctrl, Partial** part) {
 namespace fdl {
 int record_error(int code, const std::string& msg);
 int record_ok();
+int launch_wait_timeout(unsigned int* status, long long limit_cycles, cudaStream_t stream);
 }  // namespace fdl
 
 extern "C" int fdl_lmhead_confidence_noalloc(const fdl_step_cfg* cfg, const void* rows,
@@ -106,7 +114,7 @@ extern "C" int fdl_lmhead_confidence_noalloc(const fdl_step_cfg* cfg, const void
   if (rc != FDL_OK) return record_error(rc, why);
   LmArgs a;
   memset(&a, 0, sizeof(a));
-  cudaError_t e = lmhead_static_workspace(&a.ctrl, &a.part);
+  cudaError_t e = lmhead_static_workspace((cudaStream_t)stream, &a.ctrl, &a.part);
   if (e != cudaSuccess)
     return record_error(FDL_ERR_CUDA, std::string("static scratch: ") + cudaGetErrorString(e));
   const bool tc = cfg->dtype == FDL_BF16;
@@ -132,4 +140,56 @@ extern "C" int fdl_lmhead_confidence_noalloc(const fdl_step_cfg* cfg, const void
   if (e != cudaSuccess)
     return record_error(FDL_ERR_CUDA, std::string("lm-head launch: ") + cudaGetErrorString(e));
   return record_ok();
+}
+
+// Status of the allocation-free LM head: synchronise `stream`, read the static
+// scratch's status word into *status and clear it.
+extern "C" int fdl_lmhead_noalloc_status(void* stream, uint32_t* status) {
+  using namespace fdl;
+  if (status == nullptr) return record_error(FDL_ERR_INVALID_ARG, "status is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  Control* ctrl = nullptr;
+  Partial* part = nullptr;
+  uint32_t host = 0;
+  cudaError_t e = lmhead_static_workspace(s, &ctrl, &part);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(&host, &ctrl->status, sizeof(host), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(&ctrl->status, 0, sizeof(uint32_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess)
+    return record_error(FDL_ERR_CUDA, std::string("static status word: ") + cudaGetErrorString(e));
+  *status = host;
+  if (host != 0)
+    return record_error(FDL_ERR_DEVICE_STATUS, "device status " + std::to_string(host));
+  return record_ok();
+}
+
+// Zero every control word of the static scratch (status and counters), on
+// `stream`.
+extern "C" int fdl_lmhead_noalloc_reset(void* stream) {
+  using namespace fdl;
+  cudaStream_t s = (cudaStream_t)stream;
+  Control* ctrl = nullptr;
+  Partial* part = nullptr;
+  cudaError_t e = lmhead_static_workspace(s, &ctrl, &part);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctrl, 0, fdl::kStaticControlSize, s);
+  if (e != cudaSuccess)
+    return record_error(FDL_ERR_CUDA, std::string("static scratch reset: ") + cudaGetErrorString(e));
+  return record_ok();
+}
+
+// The failure self-check of fdl_check_wait_timeout, aimed at the static
+// scratch's status word.
+extern "C" int fdl_lmhead_noalloc_check_wait_timeout(long long limit_cycles, void* stream) {
+  using namespace fdl;
+  if (limit_cycles < 1000 || limit_cycles > 2000000000LL)
+    return record_error(FDL_ERR_INVALID_ARG, "limit_cycles must be in [1e3, 2e9]");
+  cudaStream_t s = (cudaStream_t)stream;
+  Control* ctrl = nullptr;
+  Partial* part = nullptr;
+  cudaError_t e = lmhead_static_workspace(s, &ctrl, &part);
+  if (e != cudaSuccess)
+    return record_error(FDL_ERR_CUDA, std::string("static scratch: ") + cudaGetErrorString(e));
+  return launch_wait_timeout(&ctrl->status, limit_cycles, s);
 }

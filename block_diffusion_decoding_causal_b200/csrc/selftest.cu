@@ -26,6 +26,17 @@ __global__ void wait_timeout_kernel(unsigned int* status, long long limit_cycles
 int record_error(int code, const std::string& msg);
 int record_ok();
 
+// The self-check kernel against any status word (the workspace's, or the
+// allocation-free LM head's static one).
+int launch_wait_timeout(unsigned int* status, long long limit_cycles, cudaStream_t stream) {
+  if (limit_cycles < 1000 || limit_cycles > 2000000000LL)
+    return record_error(FDL_ERR_INVALID_ARG, "limit_cycles must be in [1e3, 2e9]");
+  wait_timeout_kernel<<<1, 32, 0, stream>>>(status, limit_cycles);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return record_error(FDL_ERR_CUDA, cudaGetErrorString(e));
+  return record_ok();
+}
+
 }  // namespace fdl
 
 extern "C" int fdl_check_wait_timeout(void* ws, size_t ws_bytes, long long limit_cycles,
@@ -33,11 +44,6 @@ extern "C" int fdl_check_wait_timeout(void* ws, size_t ws_bytes, long long limit
   using namespace fdl;
   if (ws == nullptr || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
     return record_error(FDL_ERR_WORKSPACE, "workspace must be at least 256 aligned bytes");
-  if (limit_cycles < 1000 || limit_cycles > 2000000000LL)
-    return record_error(FDL_ERR_INVALID_ARG, "limit_cycles must be in [1e3, 2e9]");
-  wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(
-      &static_cast<Control*>(ws)->status, limit_cycles);
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return record_error(FDL_ERR_CUDA, cudaGetErrorString(e));
-  return record_ok();
+  return launch_wait_timeout(&static_cast<Control*>(ws)->status, limit_cycles,
+                             (cudaStream_t)stream);
 }

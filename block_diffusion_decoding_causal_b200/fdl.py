@@ -29,7 +29,10 @@ SYMBOLS = ["fdl_version", "fdl_last_error", "fdl_workspace_size",
            "fdl_lmhead_confidence", "fdl_threshold_commit", "fdl_denoise_step",
            "fdl_get_status", "fdl_lmhead_confidence_noalloc", "fdl_select_commit",
            "fdl_unit_status", "fdl_append_block", "fdl_prefixcache_attn",
-           "fdl_check_wait_timeout", "fdl_lmhead_pack_weight"]
+           "fdl_check_wait_timeout", "fdl_lmhead_pack_weight",
+           "fdl_lmhead_noalloc_status", "fdl_lmhead_noalloc_reset",
+           "fdl_lmhead_noalloc_check_wait_timeout"]
+NOALLOC_MAX_ROWS = 128
 
 
 class StepCfg(ctypes.Structure):
@@ -86,12 +89,17 @@ def lib() -> ctypes.CDLL:
         L.fdl_check_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_longlong, _P]
         L.fdl_lmhead_pack_weight.argtypes = [ctypes.POINTER(StepCfg), _P, _P, _P]
         L.fdl_append_block.argtypes = [ctypes.POINTER(StepCfg)] + [_P] * 5 + [_P, ctypes.c_size_t, _P]
+        L.fdl_lmhead_noalloc_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
+        L.fdl_lmhead_noalloc_reset.argtypes = [_P]
+        L.fdl_lmhead_noalloc_check_wait_timeout.argtypes = [ctypes.c_longlong, _P]
         for name in ["fdl_reset_workspace", "fdl_block_attn", "fdl_dualcache_attn",
                      "fdl_lmhead_confidence", "fdl_threshold_commit",
                      "fdl_denoise_step", "fdl_get_status",
                      "fdl_lmhead_confidence_noalloc", "fdl_select_commit",
                      "fdl_unit_status", "fdl_append_block", "fdl_prefixcache_attn",
-                     "fdl_check_wait_timeout", "fdl_lmhead_pack_weight"]:
+                     "fdl_check_wait_timeout", "fdl_lmhead_pack_weight",
+                     "fdl_lmhead_noalloc_status", "fdl_lmhead_noalloc_reset",
+                     "fdl_lmhead_noalloc_check_wait_timeout"]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -172,8 +180,9 @@ def lmhead_confidence(cfg, rows, w_lm, row_active, conf, tok, ws, stream=None):
 
 def lmhead_confidence_noalloc(cfg, rows, w_lm, row_active, conf, tok, stream=None):
     """fdl_lmhead_confidence with the library's built-in scratch instead of a
-    caller workspace (at most 128 rows; calls on one device must not overlap
-    on the GPU; make the first call on a device before any stream capture)."""
+    caller workspace (at most NOALLOC_MAX_ROWS rows; calls on one device must
+    not overlap on the GPU; make the first call on a device before any stream
+    capture; device failures are read with ``lmhead_noalloc_status``)."""
     _check(lib().fdl_lmhead_confidence_noalloc(ctypes.byref(cfg), ptr(rows), ptr(w_lm),
                                                ptr(row_active), ptr(conf), ptr(tok),
                                                stream_ptr(stream)))
@@ -234,3 +243,21 @@ def get_status(ws, stream=None) -> int:
     if rc not in (OK, ERR_DEVICE_STATUS):
         raise FdlError(rc, last_error())
     return int(st.value)
+
+
+def lmhead_noalloc_status(stream=None) -> int:
+    """Synchronise, read and clear the allocation-free LM head's own status
+    word (FDL_DEV_* bits)."""
+    st = ctypes.c_uint32(0)
+    rc = lib().fdl_lmhead_noalloc_status(stream_ptr(stream), ctypes.byref(st))
+    if rc not in (OK, ERR_DEVICE_STATUS):
+        raise FdlError(rc, last_error())
+    return int(st.value)
+
+
+def lmhead_noalloc_reset(stream=None):
+    _check(lib().fdl_lmhead_noalloc_reset(stream_ptr(stream)))
+
+
+def lmhead_noalloc_check_wait_timeout(limit_cycles=1_000_000, stream=None):
+    _check(lib().fdl_lmhead_noalloc_check_wait_timeout(int(limit_cycles), stream_ptr(stream)))

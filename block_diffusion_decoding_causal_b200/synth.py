@@ -86,7 +86,7 @@ class Case:
     len_suf: Optional[torch.Tensor]
     hidden: Optional[torch.Tensor]  # [B, q_len, H] LM-head input rows, or None
     h_prev: Optional[torch.Tensor]  # [B, H] hidden state before the unit
-    w_lm: torch.Tensor             # [V, H]
+    w_lm: Optional[torch.Tensor]   # [V, H] (None when not drawn)
     block_tokens: torch.Tensor     # [B, D] int32
 
 
@@ -125,13 +125,15 @@ def torch_dtype(dtype: str) -> torch.dtype:
 
 
 def make_case(name: str, seed: int, cfg: Optional[dict] = None,
-              attn_as_hidden: bool = False, **overrides) -> Case:
+              attn_as_hidden: bool = False, draw_w: bool = True, **overrides) -> Case:
     """Draw one step input.
 
     ``name`` picks a row of ``CONFIGS`` (or pass ``cfg`` explicitly); keyword
     overrides replace config entries (e.g. ``tau=0.7``, ``batch=2``).  With
     ``attn_as_hidden`` the LM-head rows are the attention output itself (no
-    separate hidden input), the literal single-layer chaining.
+    separate hidden input), the literal single-layer chaining.  With
+    ``draw_w=False`` the LM-head weight is not drawn (``w_lm`` is None), for
+    callers that already hold the case's weight.
     """
     c = dict(CONFIGS[name] if cfg is None else cfg)
     c.update(overrides)
@@ -167,7 +169,8 @@ def make_case(name: str, seed: int, cfg: Optional[dict] = None,
         len_suf = torch.full((B,), int(c["suffix"]), dtype=torch.int32)
     hidden = None if attn_as_hidden else _normal(seed, "hidden", (B, q_len, H), dt)
     h_prev = _normal(seed, "h_prev", (B, H), dt) if c["shift"] else None
-    w_lm = _normal(seed, "w_lm", (V, H), dt, scale=c["w_scale"] / H ** 0.5)
+    w_lm = (_normal(seed, "w_lm", (V, H), dt, scale=c["w_scale"] / H ** 0.5)
+            if draw_w else None)
 
     # Block tokens: finished positions hold random non-mask tokens; inside the
     # unit a seeded subset is masked; later sub-blocks are still all masked.

@@ -286,20 +286,44 @@ int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
  * For callers that cannot allocate device memory: a plugin inside another
  * engine that owns every allocation, a loop where allocation is forbidden
  * after start-up, or code that cannot reach the host framework's allocator.
- * The scratch is a fixed array inside libfdl (606,464 bytes, held by every
- * GPU that loads the library until the process exits), so:
- *  - batch * q_len must be at most 128 (else FDL_ERR_UNSUPPORTED);
- *  - the first call on a device looks the array up and zeroes its control
- *    words, synchronously, with that device current: make that first call
- *    before any stream capture;
+ * The scratch is a fixed array inside libfdl (FDL_NOALLOC_SCRATCH_BYTES,
+ * held by every GPU that loads the library until the process exits), so:
+ *  - batch * q_len must be at most FDL_NOALLOC_MAX_ROWS (else
+ *    FDL_ERR_UNSUPPORTED, before any launch);
+ *  - the first call on a device (of this function or of the three
+ *    fdl_lmhead_noalloc_* calls below) looks the array up, with that device
+ *    current, and queues the zeroing of its control words on `stream`, ahead
+ *    of its kernel: make that first call before any stream capture;
  *  - every call on a device shares the array and leaves its counters at zero;
  *    calls whose kernels overlap on the GPU (other streams, other threads)
- *    race on it and must be serialised by the caller.
+ *    race on it and must be serialised by the caller;
+ *  - device-detected failures (a bounded wait that ran out) set bits in the
+ *    array's own status word, which fdl_get_status cannot see: read them with
+ *    fdl_lmhead_noalloc_status.  While FDL_DEV_TIMEOUT is set every row
+ *    reports conf = -1, tok = -1.
  * It calls no cudaMalloc, cudaFree or other allocating routine.
  */
+#define FDL_NOALLOC_MAX_ROWS 128
+#define FDL_NOALLOC_SCRATCH_BYTES 606464 /* 256 control bytes + 296 x 128 partials of 16 B */
 int fdl_lmhead_confidence_noalloc(const fdl_step_cfg* cfg, const void* rows,
                                   const void* w_lm, const uint8_t* row_active,
                                   float* conf, int32_t* tok, void* stream);
+
+/* The allocation-free LM head's status word: synchronise `stream`, read it
+ * into *status (bits FDL_DEV_*) and clear it.  Returns FDL_ERR_DEVICE_STATUS
+ * if any bit was set, FDL_OK otherwise.  Allocates nothing. */
+int fdl_lmhead_noalloc_status(void* stream, uint32_t* status);
+
+/* Zero all control words of the allocation-free LM head's array (status and
+ * counters), on `stream`; for use after a device-detected failure.  Allocates
+ * nothing. */
+int fdl_lmhead_noalloc_reset(void* stream);
+
+/* fdl_check_wait_timeout aimed at the allocation-free LM head's status word:
+ * one CTA's bounded wait runs out after limit_cycles (1e3 .. 2e9) and sets
+ * FDL_DEV_TIMEOUT there, which fdl_lmhead_noalloc_status then reports.
+ * A diagnostic of this library (no counterpart on the pages). */
+int fdl_lmhead_noalloc_check_wait_timeout(long long limit_cycles, void* stream);
 
 /*
  * Loop control of the block decode (technical review Algorithm 1: repeat

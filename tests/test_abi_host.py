@@ -215,6 +215,35 @@ def test_wait_timeout_check_rejects_bad_arguments(L):
     assert rc == fdl.ERR_INVALID_ARG and "limit_cycles" in fdl.last_error()
 
 
+def test_noalloc_helpers_reject_bad_arguments(L):
+    assert L.fdl_lmhead_noalloc_status(None, None) == fdl.ERR_INVALID_ARG
+    rc = L.fdl_lmhead_noalloc_check_wait_timeout(10, None)
+    assert rc == fdl.ERR_INVALID_ARG and "limit_cycles" in fdl.last_error()
+
+
+def test_noalloc_limits_in_header_match_binding(tmp_path):
+    """FDL_NOALLOC_MAX_ROWS and FDL_NOALLOC_SCRATCH_BYTES as the C compiler
+    reads them from include/fdl.h (the library static_asserts the latter
+    against its own array); the binding's row limit agrees."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "limits.c"
+    src.write_text("#include <stdio.h>\n#include \"fdl.h\"\n"
+                   "int main(void) { printf(\"%d %d\\n\", FDL_NOALLOC_MAX_ROWS, "
+                   "FDL_NOALLOC_SCRATCH_BYTES); return 0; }\n")
+    exe = tmp_path / "limits"
+    include = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                           "include")
+    subprocess.run([cc, "-I", include, str(src), "-o", str(exe)], check=True)
+    rows, nbytes = map(int, subprocess.run([str(exe)], check=True, capture_output=True,
+                                           text=True).stdout.split())
+    assert rows == fdl.NOALLOC_MAX_ROWS
+    assert nbytes == 256 + 16 * 296 * rows
+
+
 def test_weight_layout_rules(L):
     bad = _cfg()
     bad.w_layout = 2

@@ -191,6 +191,51 @@ def test_sweep_full_size(batch, prefix):
     gh.compare_step(case, gpu, ref, check_attn=True)
 
 
+def _assert_regime(ref, regime):
+    """The commit regime a case claims to exercise, read from the oracle.
+    "fallback": no candidate reaches tau, so each unit with candidates
+    commits exactly its single most confident position (Algorithm 2's
+    fallback); "parallel": at least one unit commits several positions in
+    this one step."""
+    act, tau = ref["active"], ref["tau"]
+    has_cand = act.any(axis=1)
+    if regime == "fallback":
+        assert (ref["conf"][act] < tau).all()
+        assert (ref["n_committed"][has_cand] == 1).all()
+    elif regime == "parallel":
+        assert ref["n_committed"].max() > 1
+    else:
+        raise ValueError(regime)
+
+
+@pytest.mark.parametrize("batch,prefix,scale,tau,regime", [
+    (4, 2048, 4.0, 0.9, "fallback"),      # mostly below tau: the fallback decides
+    (1, 2048, 4.0, 0.9, "fallback"),
+    (4, 8192, 12.0, 0.9, "parallel"),     # mostly above tau: several commit at once
+    (16, 2048, 12.0, 0.9, "parallel"),
+    (4, 2048, 8.0, 0.7, "parallel"),      # the 7B workload's lower threshold
+    (16, 8192, 4.0, 0.9, None),
+])
+def test_sweep_points_and_their_commit_regimes(batch, prefix, scale, tau, regime):
+    """Long-context sweep points at full size over batch, prefix and logit
+    scale (the confidence regime), each checked against the oracle and for
+    the regime it is meant to exercise."""
+    cfg = synth.sweep_config(batch, prefix, scale)
+    cfg["tau"] = tau
+    case, ref, _ = cases.parity_case("sweep", 0, cfg=cfg)
+    if regime is not None:
+        _assert_regime(ref, regime)
+    gh.compare_step(case, gh.run_denoise_step(case), ref, check_attn=True)
+
+
+@pytest.mark.parametrize("seed,regime", [(1, None), (2, "parallel")])
+def test_llada_dualcache_step_more_seeds(seed, regime):
+    case, ref, _ = cases.parity_case("llada", seed)
+    if regime is not None:
+        _assert_regime(ref, regime)
+    gh.compare_step(case, gh.run_denoise_step(case), ref)
+
+
 # ---------------------------------------------- LM head shapes and tails
 
 @pytest.mark.parametrize("R,V,H", [(1, 5000, 64), (32, 5000, 448), (33, 33000, 128),
