@@ -393,73 +393,108 @@ def main():
     # End to end through the public API: per step, pinned host inputs copied
     # in, the step, and its results copied out and read on the host.
     host_in = sets[0]["_buf"].cpu().pin_memory()       # one packed upload per step
-    host_out = torch.empty_like(out_buf, device="cpu").pin_memory()
-    host_bt = torch.empty_like(sets[0]["bt"], device="cpu").pin_memory()
-    host_n_l = _views(torch, host_out, out_buf, out)["n_l"]
-    host_n_l_np = host_n_l.numpy()
-    h2d = host_in.numel()
-    d2h = host_out.numel() + host_bt.numel() * host_bt.element_size()
-
-    # As a serving loop runs it: the step and the copy of its results to the
-    # host are replayed from one CUDA graph per input set (captured from the
-    # same fdl_denoise_step call), and the upload is double-buffered: step
-    # i+1's inputs cross PCIe on a copy stream while step i runs (each input
-    # set has its own device buffer; a set is refilled only after the step
-    # that last read it finished).  Every step still uploads its inputs, and
-    # the host still reads every step's result before the next step starts.
-    copy_stream = torch.cuda.Stream()
     n_sets = n_copies
+    e2e_out = [_pack(torch, dict(
+        conf=torch.empty((B, q_len), dtype=torch.float32),
+        tok=torch.empty((B, q_len), dtype=torch.int32),
+        committed=torch.empty((B, c["block_size"]), dtype=torch.uint8),
+        n_c=torch.empty(B, dtype=torch.int32),
+        n_l=torch.empty(B, dtype=torch.int32)), "cuda") for _ in range(n_sets)]
+    host_outs = [torch.empty_like(ob, device="cpu").pin_memory() for ob, _ in e2e_out]
+    host_bts = [torch.empty_like(sets[0]["bt"], device="cpu").pin_memory()
+                for _ in range(n_sets)]
+    host_n_l_np = [_views(torch, h, e2e_out[0][0], e2e_out[0][1])["n_l"].numpy()
+                   for h in host_outs]
+    h2d = host_in.numel()
+    d2h = host_outs[0].numel() + host_bts[0].numel() * host_bts[0].element_size()
+
+    # As a serving loop runs it.  Each input set has its own device inputs
+    # and outputs and pinned host outputs.  The step is replayed from one CUDA
+    # graph per set (captured from the same fdl_denoise_step call).  Step
+    # i+1's inputs cross PCIe on a copy stream while step i runs (a set is
+    # refilled only after its previous step and result copy finished), and
+    # step i's results go back to the host on a third stream while step i+1
+    # computes.  Every step uploads its inputs and the host reads every
+    # step's result.  Pipelined (the headline): the host reads step i-1's
+    # result while step i runs.  Serial (reported beside it): the host reads
+    # step i's result before step i+1 is launched.
+    copy_stream = torch.cuda.Stream()
+    d2h_stream = torch.cuda.Stream()
     copied = [torch.cuda.Event() for _ in range(n_sets)]
-    freed = [torch.cuda.Event() for _ in range(n_sets)]
+    computed = [torch.cuda.Event() for _ in range(n_sets)]
+    done = [torch.cuda.Event() for _ in range(n_sets)]
+
+    def step_into(x, o):
+        fdl.denoise_step(cfg, x["q"], x["k_pre"], x["v_pre"], x["len_pre"], x["k_blk"],
+                         x["v_blk"], None, None, None, x["hidden"], x["h_prev"], w,
+                         x["bt"], None, o["conf"], o["tok"], o["committed"],
+                         o["n_c"], o["n_l"], ws, stream)
 
     graphs = []
     for j in range(n_sets):
         gph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gph, stream=stream):
-            step(sets[j])
-            host_out.copy_(out_buf, non_blocking=True)
-            host_bt.copy_(sets[j]["bt"], non_blocking=True)
+            step_into(sets[j], e2e_out[j][1])
         graphs.append(gph)
     stream.synchronize()
 
     def upload(i):
         j = i % n_sets
-        copy_stream.wait_event(freed[j])
+        copy_stream.wait_event(done[j])
         with torch.cuda.stream(copy_stream):
             sets[j]["_buf"].copy_(host_in, non_blocking=True)
         copied[j].record(copy_stream)
 
-    def e2e_run(k, start):
+    def e2e_run(k, start, pipelined):
         for j in range(n_sets):
-            freed[j].record(stream)
+            done[j].record(stream)
         copy_stream.wait_event(start)        # the first upload is inside the timing
         upload(0)
+        seen = 0
         for i in range(k):
             j = i % n_sets
             stream.wait_event(copied[j])
             with torch.cuda.stream(stream):
-                graphs[j].replay()           # the step, then its results to the host
-            freed[j].record(stream)
+                graphs[j].replay()           # the step
+            computed[j].record(stream)
+            d2h_stream.wait_event(computed[j])
+            with torch.cuda.stream(d2h_stream):  # its results to the host
+                host_outs[j].copy_(e2e_out[j][0], non_blocking=True)
+                host_bts[j].copy_(sets[j]["bt"], non_blocking=True)
+            done[j].record(d2h_stream)
             if i + 1 < k and n_sets > 1:
                 upload(i + 1)                # crosses PCIe while step i runs
-            stream.synchronize()
-            _ = int(host_n_l_np.sum())       # the host reads the result
-            if n_sets == 1 and i + 1 < k:
-                upload(i + 1)
+            if pipelined:
+                if i >= 1:
+                    jp = (i - 1) % n_sets
+                    done[jp].synchronize()   # step i-1's results are on the host
+                    seen += int(host_n_l_np[jp].sum())
+            else:
+                done[j].synchronize()
+                seen += int(host_n_l_np[j].sum())   # the host reads the result
+                if n_sets == 1 and i + 1 < k:
+                    upload(i + 1)
+        jl = (k - 1) % n_sets
+        if pipelined:
+            done[jl].synchronize()
+            seen += int(host_n_l_np[jl].sum())
+        stream.wait_event(done[jl])          # the timing ends after the last read-back
+        return seen
 
-    def timed_e2e(k):
+    def timed_e2e(k, pipelined):
         ev0 = torch.cuda.Event(enable_timing=True)
         ev1 = torch.cuda.Event(enable_timing=True)
         barrier(world)
         torch.cuda.synchronize()
         ev0.record(stream)
-        e2e_run(k, ev0)
+        e2e_run(k, ev0, pipelined)
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
         return ev0.elapsed_time(ev1) / 1e3
-    timed_e2e(3)                              # warm-up
-    t_e2e = max_over_ranks(timed_e2e(args.steps), world)
+    timed_e2e(3, True)                        # warm-up
+    t_e2e = max_over_ranks(timed_e2e(args.steps, True), world)
+    t_e2e_serial = max_over_ranks(timed_e2e(args.steps, False), world)
     e2e_value = pos / t_e2e
     assert fdl.get_status(ws, stream) == 0
     del graphs
@@ -515,10 +550,16 @@ def main():
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e / args.steps * 1e3,
                 "upload": "double-buffered: step i+1's inputs copied on a second stream "
-                          "during step i; step i's results read on the host before "
-                          "step i+1 is launched",
+                          "during step i",
+                "readback": "every step's results copied to pinned host memory on a third "
+                            "stream and read on the host; the host reads step i-1's while "
+                            "step i runs",
                 "launch": "the step and its result copies replayed from one CUDA graph "
-                          "per input set, captured from fdl_denoise_step"},
+                          "per input set, captured from fdl_denoise_step",
+                "serial": {"value": pos / t_e2e_serial,
+                           "ms_per_step": t_e2e_serial / args.steps * 1e3,
+                           "readback": "step i's results read on the host before step "
+                                       "i+1 is launched"}},
         "gpu_launches": _launches_per_step(c) * args.steps,
         "committed_per_step": committed,
         "clocks": clk,

@@ -31,6 +31,8 @@
 // No thread waits on another CTA.
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "fdl_common.cuh"
 #include "sm100.cuh"
 
@@ -76,6 +78,7 @@ struct TcArgs {
   float* part_o;          // [2 * n_cta][128][128]
   float2* part_ml;        // [2 * n_cta][128]
   int inline_merge;       // the last CTA to finish a row of an item merges it
+  int coop_merge;         // grid barrier, then every CTA merges split rows
   int q_region;           // bytes between the two d-halves of the Q buffer
 };
 
@@ -245,6 +248,102 @@ __device__ __noinline__ void merge_row_inline(const TcArgs& a, int r, int cta_lo
       o.w = pack_bf16(acc[8 * t + 6] * inv, acc[8 * t + 7] * inv);
       *reinterpret_cast<uint4*>(orow + cc * 32 + 8 * t) = o;
     }
+  }
+}
+
+// Grid-wide barrier of a cooperative launch (every CTA is resident, so
+// every CTA arrives).  The last CTA to arrive rearms the count and bumps the
+// generation the others watch.  The watch is bounded: on expiry it returns
+// false and the caller flags a timeout.
+__device__ __noinline__ bool grid_barrier(Control* ctrl, unsigned int n) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bool ok = true;
+    volatile unsigned int* gen = &ctrl->grid_gen;
+    const unsigned int g = *gen;
+    __threadfence();
+    if (atomicAdd(&ctrl->grid_bar, 1u) == n - 1u) {
+      ctrl->grid_bar = 0u;
+      __threadfence();
+      atomicAdd(&ctrl->grid_gen, 1u);
+    } else {
+      const long long t0 = clock64();
+      while (*gen == g) {
+        if (clock64() - t0 > kWaitCycles) {
+          ok = false;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+    s_ok = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+// After the grid barrier: every split row of every item, one warp per
+// (item, row), tasks strided over all warps of the grid.  The row's partials
+// (CTAs cta_lo .. cta_hi) are combined with the usual (max, sum) rescaling,
+// eight reads in flight at a time; lanes hold four of the 128 columns.
+__device__ __noinline__ void merge_split_rows(const TcArgs& a, const int* cb, const int* nc, long long T,
+                                 int n) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per_seq = a.Hkv * a.n_rt;
+  const int rows_full = a.qpt * a.group;
+  const long long n_tasks = (long long)a.B * per_seq * rows_full;
+  const int warps = kThreads / 32;
+  for (long long task = (long long)blockIdx.x * warps + warp; task < n_tasks;
+       task += (long long)n * warps) {
+    const int x = (int)(task / rows_full), r = (int)(task % rows_full);
+    const int b = x / per_seq, it = x % per_seq;
+    const long long x_start = cb[b] + (long long)it * nc[b];
+    const long long x_end = x_start + nc[b];
+    if (x_end <= x_start) continue;
+    const int cta_lo = cta_of(x_start, T, n), cta_hi = cta_of(x_end - 1, T, n);
+    if (cta_lo == cta_hi) continue;  // written directly by its only CTA
+    const int kvh = it / a.n_rt, rt = it % a.n_rt;
+    const int qpt_eff = min(a.qpt, a.q_len - rt * a.qpt);
+    if (r >= qpt_eff * a.group) continue;
+    float M = kEmptyMax, L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = cta_lo; j0 <= cta_hi; j0 += 8) {
+      float2 ml[8];
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u;
+        if (j <= cta_hi && cta_nonempty(j, T, n)) {
+          const int sl = partial_slot(j, cta_lo, x_start, T, n);
+          ml[u] = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
+          v[u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128) +
+                        lane);
+        } else {
+          ml[u] = make_float2(kEmptyMax, 0.f);
+          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float m_new = fmaxf(M, ml[u].x);
+        const float f_old = exp2f(M - m_new), w = exp2f(ml[u].x - m_new);
+        L = L * f_old + ml[u].y * w;
+        acc.x = acc.x * f_old + v[u].x * w;
+        acc.y = acc.y * f_old + v[u].y * w;
+        acc.z = acc.z * f_old + v[u].z * w;
+        acc.w = acc.w * f_old + v[u].w * w;
+        M = m_new;
+      }
+    }
+    const float inv = 1.f / L;
+    const int pq = r / a.group, jq = r % a.group;
+    bf16* dst = a.out + (((size_t)b * a.q_len + rt * a.qpt + pq) * a.Hq + kvh * a.group + jq) * 128;
+    uint2 packed;
+    packed.x = pack_bf16(acc.x * inv, acc.y * inv);
+    packed.y = pack_bf16(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(dst)[lane] = packed;
   }
 }
 
@@ -666,6 +765,14 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
     tmem_dealloc(tmem, kTmemCols);
   }
   if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
+  if (a.coop_merge) {
+    // Cooperative launch: once every CTA has written its partials, all of
+    // them merge the split rows (no second kernel).
+    if (grid_barrier(a.ctrl, (unsigned int)n))
+      merge_split_rows(a, cb, nc, T, n);
+    else if (threadIdx.x == 0)
+      atomicOr(&a.ctrl->status, kDevTimeout);
+  }
   // This CTA is done: the merge kernel may be scheduled once every CTA got
   // here (it still waits for the whole grid before reading anything).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -944,9 +1051,50 @@ size_t attn_tc_smem_for(int q_len, int group, int B, bool beside) {
 }
 
 
+// Per-device host state of the attention launches: the dynamic shared memory
+// each kernel variant was last opened up to, and how many of its CTAs fit on
+// the device at once for that size (the condition of a cooperative launch).
+// Both are driver queries worth skipping on every call.
+constexpr int kMaxDev = 64;
+struct KernState {
+  size_t smem_set = 0;
+  size_t resident_for = 0;
+  long resident = 0;
+};
+static KernState g_kern_state[kMaxDev][kMaxStages + 1];
+static std::mutex g_kern_mu;
+
+static cudaError_t prepare_kernel(const void* kern, int stages, size_t smem, long* resident) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_kern_mu);
+  KernState& st = g_kern_state[dev][stages];
+  if (st.smem_set < smem) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    st.smem_set = smem;
+  }
+  if (st.resident_for != smem) {
+    int sms = 0, per_sm = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    st.resident = (long)per_sm * sms;
+    st.resident_for = smem;
+  }
+  *resident = st.resident;
+  return cudaSuccess;
+}
+
 cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
                            unsigned int* tickets, int n_cta, cudaStream_t s,
-                           bool beside_prior) {
+                           bool beside_prior, bool coop_merge) {
   const int qpt = attn_tc_qpt(a.q_len, a.group);
   if (a.d != 128 || qpt == 0 || a.B > kMaxSeq) return cudaErrorInvalidValue;
   Maps maps;
@@ -1000,6 +1148,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   t.part_o = part_o;
   t.part_ml = part_ml;
   t.inline_merge = beside_prior ? 1 : 0;
+  t.coop_merge = 0;
   t.q_region = q_region_for(qpt * a.group);
   // Beside the LM head: one K/V stage, so the SM's remaining shared memory
   // goes to that kernel's weight ring.
@@ -1007,30 +1156,32 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   const size_t smem = attn_tc_smem_bytes(stages, t.q_region, a.B);
   auto kern = stages == 1 ? attn_tc_kernel<1> : (stages == 2 ? attn_tc_kernel<2>
                                                              : attn_tc_kernel<3>);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  long resident = 0;
+  cudaError_t e = prepare_kernel(reinterpret_cast<const void*>(kern), stages, smem, &resident);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared);
-  if (e != cudaSuccess) return e;
+  // One sequence and one CTA per item: all its items have the same chunks,
+  // so each CTA's range is exactly one item and there is nothing to merge.
+  const bool nothing_split = a.B == 1 && n_cta == n_items_all;
+  if (coop_merge && !beside_prior && !nothing_split && resident >= n_cta) t.coop_merge = 1;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   {
+    cudaLaunchAttribute coop[1];
+    coop[0].id = cudaLaunchAttributeCooperative;
+    coop[0].val.cooperative = 1;
     cudaLaunchConfig_t mc = {};
     mc.gridDim = dim3(n_cta, 1, 1);
     mc.blockDim = dim3(kThreads, 1, 1);
     mc.dynamicSmemBytes = smem;
     mc.stream = s;
-    mc.attrs = attr;
-    mc.numAttrs = beside_prior ? 1 : 0;
+    mc.attrs = t.coop_merge ? coop : attr;
+    mc.numAttrs = (beside_prior || t.coop_merge) ? 1 : 0;
     e = cudaLaunchKernelEx(&mc, kern, maps, t);
     if (e != cudaSuccess) return e;
   }
   if (beside_prior) return cudaSuccess;  // merged inside the kernel
-  // One sequence and one CTA per item: all its items have the same chunks,
-  // so each CTA's range is exactly one item and there is nothing to merge.
-  if (a.B == 1 && n_cta == n_items_all) return cudaGetLastError();
+  if (t.coop_merge || nothing_split) return cudaGetLastError();
   cudaLaunchConfig_t lc = {};
   const int n_items = a.B * a.Hkv * t.n_rt;
   // Partials per split item are about n_cta / n_items + 1: few, and a CTA
