@@ -152,6 +152,31 @@ def rounds_us(timed, fn, k: int, reps: int, world: int) -> list:
     return [max_over_ranks(timed(fn, k), world) / k * 1e6 for _ in range(reps)]
 
 
+def graph_rounds_us(torch, stream, fn, k: int, reps: int, world: int) -> list:
+    """Per-launch microseconds of ``reps`` replays of one CUDA graph that holds
+    ``k`` launches of ``fn`` (captured on ``stream``): the device time of
+    back-to-back launches without the host's per-call work between them, as
+    a serving loop that captures its step sees it."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(k):
+            fn(i)
+    out = []
+    with torch.cuda.stream(stream):
+        g.replay()
+        stream.synchronize()
+        for _ in range(reps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            stream.synchronize()
+            out.append(max_over_ranks(e0.elapsed_time(e1) * 1e3 / k, world))
+    del g
+    return out
+
+
 def spread(us: list) -> dict:
     """Median and range of repeated timings."""
     return {"median": statistics.median(us), "min": min(us), "max": max(us),
@@ -370,6 +395,7 @@ def main():
         attn(i)
     attn_rounds = rounds_us(timed, attn, args.steps, 3, world)
     t_attn = statistics.median(attn_rounds) * 1e-6
+    attn_graph = graph_rounds_us(torch, stream, attn, args.steps, 3, world)
     pc = prefixcache_leg(torch, fdl, stream, timed, world, args.steps, peaks)
     try:
         blk = block_decode_leg(torch, fdl, c_run, sets[0], w, stream, world)
@@ -538,7 +564,10 @@ def main():
         "attention": {"us_per_launch": t_attn * 1e6, "bytes_per_launch": attn_bytes,
                       "achieved_gbs": attn_bytes / t_attn / 1e9,
                       "frac_hbm": attn_bytes / t_attn / 1e9 / peaks["hbm_gbs"],
-                      "us_rounds": spread(attn_rounds)},
+                      "us_rounds": spread(attn_rounds),
+                      "graph": {"us": spread(attn_graph),
+                                "frac_hbm": attn_bytes / statistics.median(attn_graph) / 1e3
+                                / peaks["hbm_gbs"]}},
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": step_bytes / (t_step / args.steps) / 1e9,
                           "frac": step_bytes / (t_step / args.steps) / 1e9 / peaks["hbm_gbs"]},
         "prefixcache": pc,
@@ -751,6 +780,7 @@ def prefixcache_leg(torch, fdl, stream, timed, world, steps, peaks) -> dict:
     for i in range(3):
         run(i)
     t = max_over_ranks(timed(run, steps), world) / steps
+    t_graph = statistics.median(graph_rounds_us(torch, stream, run, steps, 3, world)) * 1e-6
     flops = 4.0 * B * Hq * n * (Lp + n) * d
     bytes_ = B * Hkv * (Lp + n) * d * 2 * 2 + 2 * B * n * Hq * d * 2
     bound = "tensor" if flops / (peaks["bf16_tflops"] * 1e12) > bytes_ / (peaks["hbm_gbs"] * 1e9) \
@@ -758,7 +788,9 @@ def prefixcache_leg(torch, fdl, stream, timed, world, steps, peaks) -> dict:
     return {"workload": "LLaDA-8B shapes, 32/32 heads, d 128, 768 cached + 768 recomputed rows",
             "us_per_launch": t * 1e6, "flops": flops, "bytes": bytes_, "bound": bound,
             "tflops": flops / t / 1e12, "frac_tensor": flops / t / 1e12 / peaks["bf16_tflops"],
-            "gbs": bytes_ / t / 1e9, "frac_hbm": bytes_ / t / 1e9 / peaks["hbm_gbs"]}
+            "gbs": bytes_ / t / 1e9, "frac_hbm": bytes_ / t / 1e9 / peaks["hbm_gbs"],
+            "graph": {"us_per_launch": t_graph * 1e6,
+                      "frac_tensor": flops / t_graph / 1e12 / peaks["bf16_tflops"]}}
 
 
 def large_batch_lm_leg(torch, fdl, synth, stream, timed, world, steps, peaks) -> dict:
@@ -886,6 +918,7 @@ def sweep_leg(torch, fdl, synth, stream, timed, world, steps, peaks, w8, seed,
             for i in range(3):
                 attn(i)
             a_us = rounds_us(timed, attn, steps, reps, world)
+            a_graph = graph_rounds_us(torch, stream, attn, steps, reps, world)
             a_bytes = _attn_bytes(c, case.len_pre)
             lm_bytes, lm_flops = _lm_bytes_flops(c)
             if B not in lm_by_batch:
@@ -927,7 +960,10 @@ def sweep_leg(torch, fdl, synth, stream, timed, world, steps, peaks, w8, seed,
                     "attention": {"us": spread(a_us), "bytes": a_bytes,
                                   "gbs": a_bytes / statistics.median(a_us) / 1e3,
                                   "frac_hbm": a_bytes / statistics.median(a_us) / 1e3
-                                  / peaks["hbm_gbs"]},
+                                  / peaks["hbm_gbs"],
+                                  "graph": {"us": spread(a_graph),
+                                            "frac_hbm": a_bytes / statistics.median(a_graph)
+                                            / 1e3 / peaks["hbm_gbs"]}},
                     "lm_head_frac": lm_by_batch[B]["frac"],
                     "step": {"us": spread(s_us),
                              "positions_per_s": B * c["q_len"] / statistics.median(s_us) * 1e6,
@@ -1000,6 +1036,7 @@ def configs_leg(torch, fdl, synth, stream, timed, world, steps, peaks, seed,
             for i in range(3):
                 fn(i)
             out[key] = rounds_us(timed, fn, steps, reps, world)
+        attn_graph = graph_rounds_us(torch, stream, attn, steps, reps, world)
         with torch.cuda.stream(stream):
             x["bt"].copy_(x["bt0"])
         step(0)
@@ -1027,7 +1064,10 @@ def configs_leg(torch, fdl, synth, stream, timed, world, steps, peaks, seed,
                         "roofline_us": lm_roof, "frac": lm_roof / t_lm},
             "attention": {"us": spread(out["attention"]), "bytes": a_bytes,
                           "gbs": a_bytes / t_attn / 1e3,
-                          "frac_hbm": a_bytes / t_attn / 1e3 / peaks["hbm_gbs"]},
+                          "frac_hbm": a_bytes / t_attn / 1e3 / peaks["hbm_gbs"],
+                          "graph": {"us": spread(attn_graph),
+                                    "frac_hbm": a_bytes / statistics.median(attn_graph) / 1e3
+                                    / peaks["hbm_gbs"]}},
             "committed_first_step": committed, "kv_copies": n_kv}
         del kv, x, o, w, attn_out, ws
         torch.cuda.empty_cache()

@@ -34,6 +34,7 @@
 #include <mutex>
 
 #include "fdl_common.cuh"
+#include "fdl_plan.h"
 #include "sm100.cuh"
 
 namespace fdl {
@@ -65,7 +66,6 @@ constexpr int kThreads = 192;
 constexpr float kRescale = 8.0f;         // log2-domain growth forcing a rescale
 constexpr unsigned kDevTimeout = FDL_DEV_TIMEOUT;
 constexpr int kMaxSeq = 256;
-constexpr int kMaxMergeParts = 512;      // >= CTAs of any attention grid
 
 struct TcArgs {
   int B, Hq, Hkv, q_len, D, cap_p, cap_s, group, qpt, n_rt, n_cta, dual;
@@ -78,7 +78,6 @@ struct TcArgs {
   float* part_o;          // [2 * n_cta][128][128]
   float2* part_ml;        // [2 * n_cta][128]
   int inline_merge;       // the last CTA to finish a row of an item merges it
-  int coop_merge;         // grid barrier, then every CTA merges split rows
   int q_region;           // bytes between the two d-halves of the Q buffer
 };
 
@@ -251,52 +250,24 @@ __device__ __noinline__ void merge_row_inline(const TcArgs& a, int r, int cta_lo
   }
 }
 
-// Grid-wide barrier of a cooperative launch (every CTA is resident, so
-// every CTA arrives).  The last CTA to arrive rearms the count and bumps the
-// generation the others watch.  The watch is bounded: on expiry it returns
-// false and the caller flags a timeout.
-__device__ __noinline__ bool grid_barrier(Control* ctrl, unsigned int n) {
-  __shared__ int s_ok;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    bool ok = true;
-    volatile unsigned int* gen = &ctrl->grid_gen;
-    const unsigned int g = *gen;
-    __threadfence();
-    if (atomicAdd(&ctrl->grid_bar, 1u) == n - 1u) {
-      ctrl->grid_bar = 0u;
-      __threadfence();
-      atomicAdd(&ctrl->grid_gen, 1u);
-    } else {
-      const long long t0 = clock64();
-      while (*gen == g) {
-        if (clock64() - t0 > kWaitCycles) {
-          ok = false;
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    __threadfence();
-    s_ok = ok ? 1 : 0;
-  }
-  __syncthreads();
-  return s_ok != 0;
-}
+// Every split row of every item, one warp per (item, row), the tasks
+// strided over `n_warps` warps of which this one is `first`.  The row's
+// partials (CTAs cta_lo .. cta_hi of the attention grid of n CTAs over T
+// chunks) are combined with the usual (max, sum) rescaling.  The lanes first
+// work out which of 32 CTAs hold a partial of the item and where (one CTA
+// each, in parallel: the split arithmetic is 64-bit), then the warp reads
+// them sixteen at a time with every read in flight; lanes hold four of the
+// 128 columns.
+constexpr int kMergeBatch = 8;
 
-// After the grid barrier: every split row of every item, one warp per
-// (item, row), tasks strided over all warps of the grid.  The row's partials
-// (CTAs cta_lo .. cta_hi) are combined with the usual (max, sum) rescaling,
-// eight reads in flight at a time; lanes hold four of the 128 columns.
-__device__ __noinline__ void merge_split_rows(const TcArgs& a, const int* cb, const int* nc, long long T,
-                                 int n) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ __forceinline__ void merge_split_rows(const TcArgs& a, const int* cb, const int* nc,
+                                                 long long T, int n, long long first,
+                                                 long long n_warps) {
+  const int lane = threadIdx.x & 31;
   const int per_seq = a.Hkv * a.n_rt;
   const int rows_full = a.qpt * a.group;
   const long long n_tasks = (long long)a.B * per_seq * rows_full;
-  const int warps = kThreads / 32;
-  for (long long task = (long long)blockIdx.x * warps + warp; task < n_tasks;
-       task += (long long)n * warps) {
+  for (long long task = first; task < n_tasks; task += n_warps) {
     const int x = (int)(task / rows_full), r = (int)(task % rows_full);
     const int b = x / per_seq, it = x % per_seq;
     const long long x_start = cb[b] + (long long)it * nc[b];
@@ -309,32 +280,51 @@ __device__ __noinline__ void merge_split_rows(const TcArgs& a, const int* cb, co
     if (r >= qpt_eff * a.group) continue;
     float M = kEmptyMax, L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = cta_lo; j0 <= cta_hi; j0 += 8) {
-      float2 ml[8];
-      float4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = j0 + u;
-        if (j <= cta_hi && cta_nonempty(j, T, n)) {
-          const int sl = partial_slot(j, cta_lo, x_start, T, n);
-          ml[u] = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
-          v[u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128) +
-                        lane);
-        } else {
-          ml[u] = make_float2(kEmptyMax, 0.f);
-          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+    // CTA starts T i / n in 32-bit arithmetic when T n fits (always, at the
+    // sizes the library takes; 64-bit otherwise).
+    const bool narrow = T * n < (1ll << 32);
+    const uint32_t T32 = (uint32_t)T, n32 = (uint32_t)n;
+    for (int j0 = cta_lo; j0 <= cta_hi; j0 += 32) {
+      const int j = j0 + lane;
+      long long s0, s1;
+      if (narrow) {
+        s0 = (long long)(T32 * (uint32_t)j / n32);
+        s1 = (long long)(T32 * (uint32_t)(j + 1) / n32);
+      } else {
+        s0 = cta_start(j, T, n);
+        s1 = cta_start(j + 1, T, n);
       }
+      const bool have = j <= cta_hi && s0 < s1;
+      const int my_slot = 2 * j + ((j == cta_lo && s0 != x_start) ? 1 : 0);
+      unsigned mask = __ballot_sync(0xffffffffu, have);
+      while (mask != 0u) {
+        const int cnt = min(kMergeBatch, __popc(mask));  // uniform across the warp
+        float2 ml[kMergeBatch];
+        float4 v[kMergeBatch];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float m_new = fmaxf(M, ml[u].x);
-        const float f_old = exp2f(M - m_new), w = exp2f(ml[u].x - m_new);
-        L = L * f_old + ml[u].y * w;
-        acc.x = acc.x * f_old + v[u].x * w;
-        acc.y = acc.y * f_old + v[u].y * w;
-        acc.z = acc.z * f_old + v[u].z * w;
-        acc.w = acc.w * f_old + v[u].w * w;
-        M = m_new;
+        for (int u = 0; u < kMergeBatch; ++u) {
+          if (u < cnt) {
+            const int src = __ffs(mask) - 1;
+            mask &= mask - 1u;
+            const int sl = __shfl_sync(0xffffffffu, my_slot, src);
+            ml[u] = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
+            v[u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128) +
+                          lane);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kMergeBatch; ++u) {
+          if (u < cnt) {
+            const float m_new = fmaxf(M, ml[u].x);
+            const float f_old = ex2_fast(M - m_new), w = ex2_fast(ml[u].x - m_new);
+            L = L * f_old + ml[u].y * w;
+            acc.x = acc.x * f_old + v[u].x * w;
+            acc.y = acc.y * f_old + v[u].y * w;
+            acc.z = acc.z * f_old + v[u].z * w;
+            acc.w = acc.w * f_old + v[u].w * w;
+            M = m_new;
+          }
+        }
       }
     }
     const float inv = 1.f / L;
@@ -765,14 +755,6 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
     tmem_dealloc(tmem, kTmemCols);
   }
   if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
-  if (a.coop_merge) {
-    // Cooperative launch: once every CTA has written its partials, all of
-    // them merge the split rows (no second kernel).
-    if (grid_barrier(a.ctrl, (unsigned int)n))
-      merge_split_rows(a, cb, nc, T, n);
-    else if (threadIdx.x == 0)
-      atomicOr(&a.ctrl->status, kDevTimeout);
-  }
   // This CTA is done: the merge kernel may be scheduled once every CTA got
   // here (it still waits for the whole grid before reading anything).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -782,204 +764,54 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// Merge of the partials of every item the split spread over several CTAs.
-// A CTA holds 8 / WPR rows of one item, WPR warps per row (WPR follows the
-// expected number of partials per item): warp w of a row combines partials
-// cta_lo + w, + WPR, ... with the usual (max, sum) rescaling, each lane
-// holding four of the 128 columns (one coalesced 512-byte read per partial
-// and warp); the row's warps then combine through shared memory.  Launched
-// as a programmatic dependent of the attention grid: scheduled as its CTAs
-// retire, it waits for the whole grid before reading anything.
-// Warp-collective: the partial slots of item (b, it), in CTA order, into
-// slot[] (at most kMaxMergeParts) and their count into *n_out (lane 0); the
-// split recomputed exactly as the attention kernel did.
-__device__ __noinline__ void item_partial_slots(const TcArgs& a, int b, int it, int* slot,
-                                                int* n_out) {
-  const int lane = threadIdx.x & 31;
+// Merge of the partials of every item the split spread over several CTAs,
+// launched as a programmatic dependent of the attention grid: its CTAs are
+// scheduled as the attention's retire and wait for the whole grid before
+// reading anything.  At most three CTAs per SM, eight warps each, every warp a
+// (item, row) task at a time (few fat CTAs: the launch of one small CTA per
+// (item, row block) cost more than the merge itself; three per SM keep about
+// one task per warp in flight at batch 16).  Warp 0 first rebuilds
+// the attention's sequence table from the device-resident lengths.
+__global__ void __launch_bounds__(256, 3)
+attn_merge_rows_kernel(const TcArgs a) {
+  __shared__ int cb[kMaxSeq + 1];
+  __shared__ int nc[kMaxSeq];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_seq = a.Hkv * a.n_rt;
-  long long T = 0, cb = 0;
-  int ncb = 0;
-  for (int b0 = 0; b0 < a.B; b0 += 32) {
-    const int s2 = b0 + lane;
-    int nc = 0;
-    if (s2 < a.B) {
-      int Lp = a.len_pre[s2];
-      if (Lp < 0 || Lp > a.cap_p) Lp = 0;
-      int Ls = 0;
-      if (a.dual) {
-        Ls = a.len_suf[s2];
-        if (Ls < 0 || Ls > a.cap_s) Ls = 0;
+  if (warp == 0) {
+    int run = 0;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+      const int b = b0 + lane;
+      int n_ch = 0;
+      if (b < a.B) {
+        int Lp = a.len_pre[b];
+        if (Lp < 0 || Lp > a.cap_p) Lp = 0;
+        int Ls = 0;
+        if (a.dual) {
+          Ls = a.len_suf[b];
+          if (Ls < 0 || Ls > a.cap_s) Ls = 0;
+        }
+        n_ch = item_chunks(Lp, Ls, a.D);
       }
-      nc = item_chunks(Lp, Ls, a.D);
-    }
-    int incl = nc * per_seq;
+      int incl = n_ch * per_seq;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (b < a.B) {
+        nc[b] = n_ch;
+        cb[b] = run + incl - n_ch * per_seq;
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (b >= b0 && b < b0 + 32) {
-      cb = T + __shfl_sync(0xffffffffu, incl - nc * per_seq, b - b0);
-      ncb = __shfl_sync(0xffffffffu, nc, b - b0);
-    }
-    T += __shfl_sync(0xffffffffu, incl, 31);
+    if (lane == 0) cb[a.B] = run;
   }
-  const int n = a.n_cta;
-  const long long x_start = cb + (long long)it * ncb, x_end = x_start + ncb;
-  const int cta_lo = cta_of(x_start, T, n), cta_hi = cta_of(x_end - 1, T, n);
-  // Lanes take CTAs cta_lo + lane, + 32, ...; the nonempty ones keep their
-  // order through a ballot prefix count.  One CTA alone: no partials.
-  int count = 0;
-  if (cta_lo != cta_hi) {
-    for (int j0 = cta_lo; j0 <= cta_hi; j0 += 32) {
-      const int j = j0 + lane;
-      const bool have = j <= cta_hi && cta_nonempty(j, T, n);
-      const unsigned m = __ballot_sync(0xffffffffu, have);
-      const int pos = count + __popc(m & ((1u << lane) - 1u));
-      if (have && pos < kMaxMergeParts) slot[pos] = partial_slot(j, cta_lo, x_start, T, n);
-      count += __popc(m);
-    }
-  }
-  if (lane == 0) *n_out = count < kMaxMergeParts ? count : kMaxMergeParts;
-}
-
-template <int WPR>
-__global__ void __launch_bounds__(256)
-attn_merge_kernel(const TcArgs a) {
-  constexpr int RPC = 8 / WPR;  // rows per CTA
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ float s_m[RPC][WPR], s_l[RPC][WPR];
-  __shared__ float4 s_acc[RPC][WPR][32];
-  __shared__ int s_slot[kMaxMergeParts];  // partial slots of the item, in order
-  __shared__ int s_n;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = warp / WPR, wq = warp % WPR;
-  const int per_seq = a.Hkv * a.n_rt;
-  const int x = blockIdx.x, r = blockIdx.y * RPC + half;
-  const int b = x / per_seq, it = x % per_seq;
-  const int kvh = it / a.n_rt, rt = it % a.n_rt;
-  const int qpt_eff = min(a.qpt, a.q_len - rt * a.qpt);
-  const bool row_ok = r < qpt_eff * a.group;
-  if (warp == 0) item_partial_slots(a, b, it, s_slot, &s_n);
   __syncthreads();
-  const int n_parts = s_n;
-  if (n_parts == 0) return;  // written directly by its only CTA (uniform in the CTA)
-  float M = kEmptyMax, L = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (row_ok) {
-#pragma unroll 4
-    for (int q = wq; q < n_parts; q += WPR) {
-      const int sl = s_slot[q];
-      const float2 ml = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
-      const float4 v =
-          __ldcg(reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128) + lane);
-      const float m_new = fmaxf(M, ml.x);
-      const float f_old = exp2f(M - m_new), w = exp2f(ml.x - m_new);
-      L = L * f_old + ml.y * w;
-      acc.x = acc.x * f_old + v.x * w;
-      acc.y = acc.y * f_old + v.y * w;
-      acc.z = acc.z * f_old + v.z * w;
-      acc.w = acc.w * f_old + v.w * w;
-      M = m_new;
-    }
-  }
-  if (lane == 0) {
-    s_m[half][wq] = M;
-    s_l[half][wq] = L;
-  }
-  s_acc[half][wq][lane] = acc;
-  __syncthreads();
-  if (wq != 0 || !row_ok) return;
-  float Mall = s_m[half][0];
-#pragma unroll
-  for (int w = 1; w < WPR; ++w) Mall = fmaxf(Mall, s_m[half][w]);
-  float Lall = 0.f;
-  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int w = 0; w < WPR; ++w) {
-    const float f = exp2f(s_m[half][w] - Mall);
-    const float4 v = s_acc[half][w][lane];
-    Lall += s_l[half][w] * f;
-    o.x += v.x * f;
-    o.y += v.y * f;
-    o.z += v.z * f;
-    o.w += v.w * f;
-  }
-  const float inv = 1.f / Lall;
-  const int pq = r / a.group, jq = r % a.group;
-  bf16* dst = a.out + (((size_t)b * a.q_len + rt * a.qpt + pq) * a.Hq + kvh * a.group + jq) * 128;
-  uint2 packed;
-  packed.x = pack_bf16(o.x * inv, o.y * inv);
-  packed.y = pack_bf16(o.z * inv, o.w * inv);
-  reinterpret_cast<uint2*>(dst)[lane] = packed;
-}
-
-// Merge for items with few partials (about two each, the usual case when
-// there are more items than CTAs): a CTA holds 32 rows of one item, each warp
-// four rows whose partial reads are all in flight together; lanes hold four
-// of the 128 columns.
-__global__ void __launch_bounds__(256)
-attn_merge_few_kernel(const TcArgs a) {
-  constexpr int RW = 4;  // rows per warp
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ int s_slot[kMaxMergeParts];
-  __shared__ int s_n;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per_seq = a.Hkv * a.n_rt;
-  const int x = blockIdx.x;
-  const int b = x / per_seq, it = x % per_seq;
-  const int kvh = it / a.n_rt, rt = it % a.n_rt;
-  const int qpt_eff = min(a.qpt, a.q_len - rt * a.qpt);
-  const int rows = qpt_eff * a.group;
-  if (warp == 0) item_partial_slots(a, b, it, s_slot, &s_n);
-  __syncthreads();
-  const int n_parts = s_n;
-  const int r0 = blockIdx.y * 32 + warp * RW;
-  if (n_parts == 0 || r0 >= rows) return;
-  float M[RW], L[RW];
-  float4 acc[RW];
-#pragma unroll
-  for (int k = 0; k < RW; ++k) {
-    M[k] = kEmptyMax;
-    L[k] = 0.f;
-    acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int q = 0; q < n_parts; ++q) {
-    const int sl = s_slot[q];
-    float2 ml[RW];
-    float4 v[RW];
-#pragma unroll
-    for (int k = 0; k < RW; ++k) {  // rows past the item read a valid slot row, unused
-      const int r = min(r0 + k, 127);
-      ml[k] = __ldcg(&a.part_ml[(size_t)sl * 128 + r]);
-      v[k] = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * 128 + r) * 128) +
-                    lane);
-    }
-#pragma unroll
-    for (int k = 0; k < RW; ++k) {
-      const float m_new = fmaxf(M[k], ml[k].x);
-      const float f_old = exp2f(M[k] - m_new), w = exp2f(ml[k].x - m_new);
-      L[k] = L[k] * f_old + ml[k].y * w;
-      acc[k].x = acc[k].x * f_old + v[k].x * w;
-      acc[k].y = acc[k].y * f_old + v[k].y * w;
-      acc[k].z = acc[k].z * f_old + v[k].z * w;
-      acc[k].w = acc[k].w * f_old + v[k].w * w;
-      M[k] = m_new;
-    }
-  }
-#pragma unroll
-  for (int k = 0; k < RW; ++k) {
-    const int r = r0 + k;
-    if (r >= rows) break;
-    const float inv = 1.f / L[k];
-    const int pq = r / a.group, jq = r % a.group;
-    bf16* dst =
-        a.out + (((size_t)b * a.q_len + rt * a.qpt + pq) * a.Hq + kvh * a.group + jq) * 128;
-    uint2 packed;
-    packed.x = pack_bf16(acc[k].x * inv, acc[k].y * inv);
-    packed.y = pack_bf16(acc[k].z * inv, acc[k].w * inv);
-    reinterpret_cast<uint2*>(dst)[lane] = packed;
-  }
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  merge_split_rows(a, cb, nc, cb[a.B], a.n_cta, (long long)blockIdx.x * (blockDim.x >> 5) + warp,
+                   warps);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -1052,49 +884,32 @@ size_t attn_tc_smem_for(int q_len, int group, int B, bool beside) {
 
 
 // Per-device host state of the attention launches: the dynamic shared memory
-// each kernel variant was last opened up to, and how many of its CTAs fit on
-// the device at once for that size (the condition of a cooperative launch).
-// Both are driver queries worth skipping on every call.
+// each kernel variant was last opened up to (a driver call worth skipping on
+// every launch).
 constexpr int kMaxDev = 64;
-struct KernState {
-  size_t smem_set = 0;
-  size_t resident_for = 0;
-  long resident = 0;
-};
-static KernState g_kern_state[kMaxDev][kMaxStages + 1];
+static size_t g_smem_set[kMaxDev][kMaxStages + 1];
 static std::mutex g_kern_mu;
 
-static cudaError_t prepare_kernel(const void* kern, int stages, size_t smem, long* resident) {
+static cudaError_t prepare_kernel(const void* kern, int stages, size_t smem) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_kern_mu);
-  KernState& st = g_kern_state[dev][stages];
-  if (st.smem_set < smem) {
+  if (g_smem_set[dev][stages] < smem) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    st.smem_set = smem;
+    g_smem_set[dev][stages] = smem;
   }
-  if (st.resident_for != smem) {
-    int sms = 0, per_sm = 0;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
-    if (e != cudaSuccess) return e;
-    st.resident = (long)per_sm * sms;
-    st.resident_for = smem;
-  }
-  *resident = st.resident;
   return cudaSuccess;
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
                            unsigned int* tickets, int n_cta, cudaStream_t s,
-                           bool beside_prior, bool coop_merge) {
+                           bool beside_prior) {
   const int qpt = attn_tc_qpt(a.q_len, a.group);
   if (a.d != 128 || qpt == 0 || a.B > kMaxSeq) return cudaErrorInvalidValue;
   Maps maps;
@@ -1148,7 +963,6 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   t.part_o = part_o;
   t.part_ml = part_ml;
   t.inline_merge = beside_prior ? 1 : 0;
-  t.coop_merge = 0;
   t.q_region = q_region_for(qpt * a.group);
   // Beside the LM head: one K/V stage, so the SM's remaining shared memory
   // goes to that kernel's weight ring.
@@ -1156,48 +970,39 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   const size_t smem = attn_tc_smem_bytes(stages, t.q_region, a.B);
   auto kern = stages == 1 ? attn_tc_kernel<1> : (stages == 2 ? attn_tc_kernel<2>
                                                              : attn_tc_kernel<3>);
-  long resident = 0;
-  cudaError_t e = prepare_kernel(reinterpret_cast<const void*>(kern), stages, smem, &resident);
+  cudaError_t e = prepare_kernel(reinterpret_cast<const void*>(kern), stages, smem);
   if (e != cudaSuccess) return e;
-  // One sequence and one CTA per item: all its items have the same chunks,
-  // so each CTA's range is exactly one item and there is nothing to merge.
-  const bool nothing_split = a.B == 1 && n_cta == n_items_all;
-  if (coop_merge && !beside_prior && !nothing_split && resident >= n_cta) t.coop_merge = 1;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   {
-    cudaLaunchAttribute coop[1];
-    coop[0].id = cudaLaunchAttributeCooperative;
-    coop[0].val.cooperative = 1;
     cudaLaunchConfig_t mc = {};
     mc.gridDim = dim3(n_cta, 1, 1);
     mc.blockDim = dim3(kThreads, 1, 1);
     mc.dynamicSmemBytes = smem;
     mc.stream = s;
-    mc.attrs = t.coop_merge ? coop : attr;
-    mc.numAttrs = (beside_prior || t.coop_merge) ? 1 : 0;
+    mc.attrs = attr;
+    mc.numAttrs = beside_prior ? 1 : 0;
     e = cudaLaunchKernelEx(&mc, kern, maps, t);
     if (e != cudaSuccess) return e;
   }
   if (beside_prior) return cudaSuccess;  // merged inside the kernel
-  if (t.coop_merge || nothing_split) return cudaGetLastError();
+  // One sequence and one CTA per item: all its items have the same chunks,
+  // so each CTA's range is exactly one item and there is nothing to merge.
+  if (a.B == 1 && n_cta == n_items_all) return cudaGetLastError();
+  // The merge: up to three CTAs per SM, eight warps each, one (item, row)
+  // task per warp at a time.
+  const long long tasks = (long long)n_items_all * qpt * a.group;
+  const long long want = (tasks + 7) / 8;
+  const long long cap = 3LL * kPlanCTAs;
   cudaLaunchConfig_t lc = {};
-  const int n_items = a.B * a.Hkv * t.n_rt;
-  // Partials per split item are about n_cta / n_items + 1: few, and a CTA
-  // takes 32 rows (4 per warp); more, and 1, 2 or 4 warps share a row.
-  const int est = n_cta / n_items + 1;
-  const int wpr = est <= 3 ? 0 : (est <= 6 ? 2 : 4);
-  const int rows_per_cta = wpr == 0 ? 32 : 8 / wpr;
-  lc.gridDim = dim3(n_items, (qpt * a.group + rows_per_cta - 1) / rows_per_cta, 1);
+  lc.gridDim = dim3((unsigned)(want < cap ? (want < 1 ? 1 : want) : cap), 1, 1);
   lc.blockDim = dim3(256, 1, 1);
   lc.dynamicSmemBytes = 0;
   lc.stream = s;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  e = wpr == 0 ? cudaLaunchKernelEx(&lc, attn_merge_few_kernel, t)
-               : (wpr == 2 ? cudaLaunchKernelEx(&lc, attn_merge_kernel<2>, t)
-                           : cudaLaunchKernelEx(&lc, attn_merge_kernel<4>, t));
+  e = cudaLaunchKernelEx(&lc, attn_merge_rows_kernel, t);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -140,21 +140,9 @@ int run_attention(const fdl_step_cfg& c, const Plan& p, bool dual, const void* q
                   const void* k_pre, const void* v_pre, const int32_t* len_pre,
                   const void* k_blk, const void* v_blk, const void* k_suf,
                   const void* v_suf, const int32_t* len_suf, void* out, void* ws,
-                  cudaStream_t s, bool beside_lmhead = false, bool coop_merge = false,
-                  bool prefixcache = false) {
+                  cudaStream_t s, bool beside_lmhead = false) {
   AttnArgs a = attn_args(c, p, dual, q, k_pre, v_pre, len_pre, k_blk, v_blk,
                          k_suf, v_suf, len_suf, out, ws);
-  // PrefixCache with items of more than 64 query rows: the compute-bound
-  // regime, served by the paired-tile kernel.
-  if (prefixcache && p.attn_tc && !dual) {
-    const int group = c.n_q_heads / c.n_kv_heads;
-    const int qpt = 128 / group < c.q_len ? 128 / group : c.q_len;
-    if (qpt * group > 64) {
-      cudaError_t e = launch_attn_pc(a, kPlanSMs, s);
-      if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-      return FDL_OK;
-    }
-  }
   // bf16 with d = 128: tensor-core kernel (two CTAs per SM; beside the LM
   // head, at most one per SM and only as many as keep about 32 chunks each,
   // so that few partials need merging); otherwise the CUDA-core kernel.
@@ -163,7 +151,7 @@ int run_attention(const fdl_step_cfg& c, const Plan& p, bool dual, const void* q
                                        at<float2>(ws, p.off_tc_part_ml),
                                        at<unsigned int>(ws, p.off_tc_tickets),
                                        beside_lmhead ? attn_ctas_beside(c, dual) : kAttnTcCTAs,
-                                       s, beside_lmhead, coop_merge)
+                                       s, beside_lmhead)
                       : launch_attn_simt(a, (fdl_dtype)c.dtype, kAttnRowTile, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return FDL_OK;
@@ -262,7 +250,7 @@ static int attn_common(const fdl_step_cfg* cfg, bool dual, const void* q,
                        const void* k_pre, const void* v_pre, const int32_t* len_pre,
                        const void* k_blk, const void* v_blk, const void* k_suf,
                        const void* v_suf, const int32_t* len_suf, void* out,
-                       void* ws, size_t ws_bytes, void* stream, bool prefixcache = false) {
+                       void* ws, size_t ws_bytes, void* stream) {
   Plan p;
   std::string why;
   if (!make_plan(cfg, &p, &why, false)) return fail(FDL_ERR_INVALID_ARG, "%s", why.c_str());
@@ -284,9 +272,8 @@ static int attn_common(const fdl_step_cfg* cfg, bool dual, const void* q,
   }
   int rc = check_ws(p, ws, ws_bytes);
   if (rc != FDL_OK) return rc;
-  // The standalone entry points merge split rows inside a cooperative grid.
   rc = run_attention(*cfg, p, dual, q, k_pre, v_pre, len_pre, k_blk, v_blk, k_suf,
-                     v_suf, len_suf, out, ws, (cudaStream_t)stream, false, true, prefixcache);
+                     v_suf, len_suf, out, ws, (cudaStream_t)stream);
   return rc != FDL_OK ? rc : ok();
 }
 
@@ -321,7 +308,7 @@ int fdl_prefixcache_attn(const fdl_step_cfg* cfg, const void* q, const void* k_p
   // The recomputed rows take the block's place: every key of
   // [prefix | recomputed rows] is visible to every query.
   return attn_common(cfg, false, q, k_pre, v_pre, len_pre, k_fresh, v_fresh, nullptr, nullptr,
-                     nullptr, out, ws, ws_bytes, stream, true);
+                     nullptr, out, ws, ws_bytes, stream);
 }
 
 int fdl_lmhead_confidence(const fdl_step_cfg* cfg, const void* rows,

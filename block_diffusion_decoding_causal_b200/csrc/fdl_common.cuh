@@ -70,8 +70,6 @@ struct alignas(16) Partial {
 struct Control {
   unsigned int status;     // FDL_DEV_* bits
   unsigned int lm_ticket;  // LM-head last-CTA ticket
-  unsigned int grid_bar;   // attention grid barrier: arrivals (left at zero)
-  unsigned int grid_gen;   // attention grid barrier: generation (counts up)
 };
 
 // ----------------------------------------------------------------- attention
@@ -267,15 +265,9 @@ cudaError_t launch_attn_simt(const AttnArgs& a, fdl_dtype dt, int row_tile,
 // beside_prior: launched as a programmatic dependent of the kernel before it
 // (the step's LM head), so its CTAs start beside that kernel's; it reads
 // nothing that kernel writes and, before it completes, waits for it.
-// coop_merge: when the split leaves partials, launch the grid cooperatively
-// and merge them inside it after a grid barrier instead of in a second
-// kernel (only where every CTA fits on the GPU at once; never beside_prior).
 cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
                            unsigned int* tickets, int n_cta, cudaStream_t s,
-                           bool beside_prior = false, bool coop_merge = false);
-// PrefixCache shape (items of more than 64 query rows, no suffix): pairs of
-// 128-row query tiles per CTA sharing every K/V stage, at most n_sm CTAs.
-cudaError_t launch_attn_pc(const AttnArgs& a, int n_sm, cudaStream_t s);
+                           bool beside_prior = false);
 cudaError_t launch_lmhead_simt(const LmArgs& a, fdl_dtype dt, cudaStream_t s);
 // beside_smem > 0: the shared form, leaving room on every SM for one
 // attention CTA of that many bytes of shared memory (see lmhead_tc.cu).

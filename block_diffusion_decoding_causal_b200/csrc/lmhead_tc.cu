@@ -370,6 +370,255 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
   if (threadIdx.x == 0) a.ctrl->lm_ticket = 0u;
 }
 
+// The LM head over CTA pairs (from 129 rows on, full form).  The two CTAs of
+// a cluster keep their own vocabulary ranges and tiles, and each stages its
+// own weight tile, but they share every X chunk: CTA r stages rows
+// [r N/2, (r+1) N/2) of it, and the even CTA issues tcgen05.mma.cta_group::2
+// (M = 256: its tile over the odd CTA's tile), whose result lands in each
+// CTA's own TMEM.  Per SM that halves the X bytes, which past 64 rows are
+// what the shared-memory stream carries besides the weight.  Weight tiles
+// are always loaded as full 128-row boxes (rows past a range are masked in
+// the epilogue, rows past the tensor read zeros), so the two CTAs expect the
+// same bytes at every step.  Barriers:
+//   full_a / full_b   on the even CTA only: the even CTA arms them for both
+//                     CTAs' bytes, both CTAs' loads complete on them;
+//   empty_a / empty_b in each CTA: the MMA commits to both;
+//   acc_full          in each CTA: the MMA commits to both;
+//   acc_empty         on the even CTA: both CTAs' epilogue threads arrive.
+template <int NCH, int KSUB>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
+                  const __grid_constant__ CUtensorMap tm_x, const LmArgs a, const TcParams tp) {
+  constexpr int NPAD = NCH * 32;
+  constexpr int NH = NPAD / 2;                    // X rows this CTA stages
+  constexpr int SA_BYTES = kStageA * KSUB;        // one A stage: 128 rows x 64*KSUB
+  constexpr int SB_BYTES = NH * 128 * KSUB;       // one B stage: NH rows x 64*KSUB
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int SA = tp.stages_a, SB = tp.stages_b;
+  uint8_t* sa = smem;
+  uint8_t* sb = sa + SA * SA_BYTES;
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(sb + SB * SB_BYTES);
+  uint64_t* empty_a = full_a + SA;
+  uint64_t* full_b = empty_a + SA;
+  uint64_t* empty_b = full_b + SB;
+  uint64_t* acc_full = empty_b + SB;   // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint64_t* drain = acc_empty + 2;     // [1]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  MSI* s_red = reinterpret_cast<MSI*>(tmem_holder + 4);  // [4][NPAD]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int v0 = blockIdx.x * a.rows_per_cta;
+  const int v1 = min(a.V, v0 + a.rows_per_cta);
+  // The pair steps through the same number of tiles: the larger range's.
+  const int pair0 = (blockIdx.x & ~1) * a.rows_per_cta;
+  const int pair_rows = max(0, min(a.V, pair0 + a.rows_per_cta) - pair0);
+  const int n_tiles = (pair_rows + kTileM - 1) / kTileM;
+  const int G = tp.group;
+  const int n_groups = (n_tiles + G - 1) / G;
+  const int KC = a.H / (kKChunk * KSUB);
+  const int KCT = a.H / kKChunk;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < SA; ++i) {
+      mbar_init(&full_a[i], 1);
+      mbar_init(&empty_a[i], 1);
+    }
+    for (int i = 0; i < SB; ++i) {
+      mbar_init(&full_b[i], 1);
+      mbar_init(&empty_b[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 256);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_holder, tp.tmem_cols);
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers exist before either signals the other
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  bool failed = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&tm_w_full);
+      tma_prefetch_desc(&tm_x);
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      // The rows may come from the kernel launched just before this one (the
+      // token-shift gather, programmatic launch); without one this returns.
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      int ia = 0, ib = 0;
+      for (int g = 0; g < n_groups && !failed; ++g) {
+        const int t0 = g * G, t1 = min(n_tiles, t0 + G);
+        for (int kc = 0; kc < KC && !failed; ++kc) {
+          {
+            const int slot_b = ib % SB;
+            if (!mbar_wait(&empty_b[slot_b], ((ib / SB) & 1) ^ 1)) { failed = true; break; }
+            if (leader) mbar_arrive_expect_tx(&full_b[slot_b], 2 * SB_BYTES);
+            const uint32_t bar = mapa_shared(smem_u32(&full_b[slot_b]), 0u);
+#pragma unroll
+            for (int u = 0; u < KSUB; ++u)
+              tma_load_2d_pair(sb + slot_b * SB_BYTES + u * NH * 128, &tm_x,
+                               (kc * KSUB + u) * kKChunk, (int)rank * NH, bar, pol_x);
+            ++ib;
+          }
+          for (int t = t0; t < t1; ++t) {
+            const int slot_a = ia % SA;
+            if (!mbar_wait(&empty_a[slot_a], ((ia / SA) & 1) ^ 1)) { failed = true; break; }
+            if (leader) mbar_arrive_expect_tx(&full_a[slot_a], 2 * SA_BYTES);
+            const uint32_t bar = mapa_shared(smem_u32(&full_a[slot_a]), 0u);
+            const int row0 = v0 + t * kTileM;
+            const int rt = max(0, min(kTileM, v1 - row0));  // rows of the tile (packed layout)
+            uint8_t* dst = sa + slot_a * SA_BYTES;
+#pragma unroll
+            for (int u = 0; u < KSUB; ++u) {
+              const int kk = kc * KSUB + u;
+              if (a.w_packed)
+                tma_load_2d_pair(dst + u * kStageA, &tm_w_full, 0, row0 * KCT + kk * rt, bar,
+                                 pol_w);
+              else
+                tma_load_2d_pair(dst + u * kStageA, &tm_w_full, kk * kKChunk, row0, bar, pol_w);
+            }
+            ++ia;
+          }
+        }
+      }
+      // Drain: every load of this CTA has landed before it can exit (the
+      // even CTA's full barriers count both CTAs' bytes; the odd CTA waits
+      // on its empty barriers, which the MMA releases only after the loads
+      // they followed).
+      if (leader) {
+        for (int n = max(0, ia - SA); n < ia; ++n)
+          if (!mbar_wait(&full_a[n % SA], (n / SA) & 1)) failed = true;
+        for (int n = max(0, ib - SB); n < ib; ++n)
+          if (!mbar_wait(&full_b[n % SB], (n / SB) & 1)) failed = true;
+      } else {
+        for (int n = max(0, ia - SA); n < ia; ++n)
+          if (!mbar_wait(&empty_a[n % SA], (n / SA) & 1)) failed = true;
+        for (int n = max(0, ib - SB); n < ib; ++n)
+          if (!mbar_wait(&empty_b[n % SB], (n / SB) & 1)) failed = true;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------- MMA issuer (even CTA)
+    if (leader && lane == 0 && n_tiles > 0) {
+      const uint32_t idesc = idesc_bf16_f32(2 * kTileM, NPAD);
+      int ia = 0, ib = 0;
+      for (int g = 0; g < n_groups && !failed; ++g) {
+        const int buf = tp.nbuf == 2 ? (g & 1) : 0;
+        const uint32_t ph = tp.nbuf == 2 ? ((g >> 1) & 1) : (g & 1);
+        if (!mbar_wait(&acc_empty[buf], ph ^ 1)) { failed = true; break; }
+        tc_fence_after();
+        const int t0 = g * G, t1 = min(n_tiles, t0 + G);
+        for (int kc = 0; kc < KC && !failed; ++kc) {
+          const int slot_b = ib % SB;
+          if (!mbar_wait(&full_b[slot_b], (ib / SB) & 1)) { failed = true; break; }
+          tc_fence_after();
+          const uint32_t b_base = smem_u32(sb + slot_b * SB_BYTES);
+          for (int t = t0; t < t1; ++t) {
+            const int slot_a = ia % SA;
+            if (!mbar_wait(&full_a[slot_a], (ia / SA) & 1)) { failed = true; break; }
+            tc_fence_after();
+            const uint32_t a_base = smem_u32(sa + slot_a * SA_BYTES);
+            const uint32_t d = tmem + (uint32_t)((buf * G + (t - t0)) * NPAD);
+#pragma unroll
+            for (int u = 0; u < KSUB; ++u)
+#pragma unroll
+              for (int k = 0; k < kKChunk / 16; ++k)
+                mma_bf16_pair(d, desc_k_sw128(a_base + u * kStageA + k * 32),
+                              desc_k_sw128(b_base + u * NH * 128 + k * 32), idesc,
+                              (kc | u | k) != 0 ? 1u : 0u);
+            mma_commit_pair(&empty_a[slot_a]);
+            ++ia;
+          }
+          mma_commit_pair(&empty_b[slot_b]);
+          ++ib;
+        }
+        mma_commit_pair(&acc_full[buf]);
+      }
+      mma_commit_pair_local(drain);
+      if (!mbar_wait(drain, 0)) failed = true;
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    float* tr = reinterpret_cast<float*>(s_red) + (warp - 2) * (32 * kTrStride);
+    const uint32_t acc_empty_lead0 = mapa_shared(smem_u32(&acc_empty[0]), 0u);
+    const uint32_t acc_empty_lead1 = mapa_shared(smem_u32(&acc_empty[1]), 0u);
+    MSI st[NCH];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) st[c] = msi_empty();
+    for (int g = 0; g < n_groups; ++g) {
+      const int buf = tp.nbuf == 2 ? (g & 1) : 0;
+      const uint32_t ph = tp.nbuf == 2 ? ((g >> 1) & 1) : (g & 1);
+      if (!mbar_wait(&acc_full[buf], ph)) { failed = true; break; }
+      tc_fence_after();
+      const int t0 = g * G, t1 = min(n_tiles, t0 + G);
+      for (int t = t0; t < t1; ++t) {
+        const int vbase = v0 + t * kTileM + q * 32;
+        const int n_valid = min(32, v1 - vbase);  // same for the whole warp; may be <= 0
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) +
+                                 (uint32_t)((buf * G + (t - t0)) * NPAD + c * 32),
+                             r);
+          tmem_ld_wait();
+          // Lane = vocabulary row in r; after the transpose lane j reads
+          // column j, rows in increasing vocabulary order.
+#pragma unroll
+          for (int j = 0; j < 32; ++j) tr[lane * kTrStride + j] = __uint_as_float(r[j]);
+          __syncwarp();
+          MSI m = st[c];
+          for (int k = 0; k < n_valid; ++k) msi_push(m, tr[k * kTrStride + lane], vbase + k);
+          st[c] = m;
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(buf == 0 ? acc_empty_lead0 : acc_empty_lead1);
+    }
+    named_barrier_epilogue();
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) s_red[q * NPAD + c * 32 + lane] = st[c];
+    named_barrier_epilogue();
+    for (int col = threadIdx.x - 64; col < NPAD; col += 128) {
+      MSI m = s_red[col];
+#pragma unroll
+      for (int j = 1; j < 4; ++j) m = msi_merge(m, s_red[j * NPAD + col]);
+      if (col < a.R) {
+        Partial p;
+        p.m = m.m;
+        p.s = m.s;
+        p.i = m.i;
+        p.pad = 0;
+        a.part[(size_t)blockIdx.x * a.R + col] = p;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the pair's MMAs or arrivals may touch it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, tp.tmem_cols);
+  }
+  if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
+  if (!last_cta_arrives(&a.ctrl->lm_ticket, a.n_cta)) return;
+  lm_final_merge(a);
+  if (threadIdx.x == 0) a.ctrl->lm_ticket = 0u;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -457,6 +706,60 @@ cudaError_t launch_nch(const CUtensorMap& wf, const CUtensorMap& wp, const CUten
   lc.attrs = attr;
   lc.numAttrs = after_producer ? 1 : 0;
   return cudaLaunchKernelEx(&lc, k, wf, wp, x, a, tp);
+}
+
+template <int NCH, int KSUB>
+cudaError_t launch_pair(const CUtensorMap& wf, const CUtensorMap& x, const LmArgs& a,
+                        const TcParams& tp, size_t smem, cudaStream_t s, bool after_producer) {
+  auto k = lmhead_tc2_kernel<NCH, KSUB>;
+  static std::mutex mu;
+  static size_t smem_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (smem_set[dev] < smem) {
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      smem_set[dev] = smem;
+    }
+  }
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(a.n_cta, 1, 1);  // even: whole pairs
+  lc.blockDim = dim3(kThreads, 1, 1);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = after_producer ? 1 : 0;
+  return cudaLaunchKernelEx(&lc, k, wf, x, a, tp);
+}
+
+// Ring shapes of the CTA-pair form (256 padded rows, full form): two-box K
+// stages (32 KB weight stages; X stages of half the rows), one tile per TMEM
+// buffer, two buffers, about 192 KB of rings.  (Other shapes measured at 256
+// rows: 3 + 3 stages 327 us; 4 weight + 2 X stages 350 us; two tiles per
+// buffer sharing each X chunk 334 us; a single X stage 490-560 us.)
+bool lmhead_tc2_params(int npad, int H, TcParams* tp, size_t* smem) {
+  if (npad != 256) return false;
+  if ((H / kKChunk) % 2 != 0) return false;
+  tp->npad = npad;
+  tp->ksub = 2;
+  tp->nbuf = 2;
+  tp->group = npad == 128 ? 2 : 1;
+  tp->tmem_cols = 512;
+  const size_t a_stage = (size_t)kStageA * 2;
+  const size_t b_stage = (size_t)(npad / 2) * 128 * 2;
+  tp->stages_b = npad == 128 ? 4 : 3;
+  tp->stages_a = npad == 128 ? 4 : 3;
+  const size_t bars = 8 * (size_t)(2 * tp->stages_a + 2 * tp->stages_b + 5) + 16;
+  *smem = 1024 + (size_t)tp->stages_a * a_stage + (size_t)tp->stages_b * b_stage + bars +
+          red_bytes(npad);
+  return *smem <= 227 * 1024;
 }
 
 }  // namespace
@@ -584,6 +887,22 @@ cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem
                              bool after_producer) {
   TcParams tp;
   size_t smem = 0;
+  // From 129 rows on (full form): CTA pairs sharing each X chunk.  At 256
+  // rows (7B vocabulary) 327 us a pass against 348 us for one CTA; at 128
+  // rows the pair measured no faster (232 against 228 us) and the one-CTA
+  // form stays.
+  if (beside_smem == 0 && a.R > 128 && a.R <= 256 &&
+      lmhead_tc2_params(256, a.H, &tp, &smem)) {
+    CUtensorMap wf, x;
+    const uint64_t w_inner = a.w_packed ? kKChunk : a.H;
+    const uint64_t w_outer = a.w_packed ? (uint64_t)a.V * (a.H / kKChunk) : a.V;
+    if (!make_map(&wf, a.w, w_inner, w_outer, kKChunk, kTileM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+        !make_map(&x, a.rows, a.H, a.R, kKChunk, tp.npad / 2, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+      return cudaErrorInvalidValue;
+    LmArgs ap = a;
+    ap.n_cta = (a.n_cta + 1) & ~1;  // whole pairs; a spare CTA reports an empty range
+    return launch_pair<8, 2>(wf, x, ap, tp, smem, s, after_producer);
+  }
   if (!lmhead_tc_params(a.R, a.H, a.rows_per_cta, beside_smem, &tp, &smem))
     return cudaErrorInvalidValue;
   CUtensorMap wf, wp, x;
