@@ -772,8 +772,9 @@ bool lmhead_tc2_params(int npad, int H, TcParams* tp, size_t* smem) {
 // kernels stream HBM side by side.  Its shared memory is what is left of
 // the SM's 228 KB after that CTA and the two per-CTA reservations, and must
 // exceed half the SM (so two LM-head CTAs never share one); TMEM stays within
-// 256 columns and registers within 168 per thread (R <= 64).  The widest K
-// stage (4, 2 or 1 boxes of 64) that still fits two weight stages is taken.
+// 256 columns (R <= 128: one tile per buffer from 65 rows on) and registers
+// within 168 per thread.  The widest K stage (4, 2 or 1 boxes of 64) that
+// still fits two weight stages is taken.
 bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcParams* tp,
                       size_t* smem);
 
@@ -787,7 +788,7 @@ bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcPara
   const bool shared = beside_smem > 0;
   int nch = 1;
   while (nch * 32 < R) nch *= 2;
-  if (nch > (shared ? 2 : 8)) return false;
+  if (nch > (shared ? 4 : 8)) return false;
   tp->npad = nch * 32;
   // Tiles per TMEM buffer: about half a CTA's range, so each X chunk serves
   // several weight tiles and the epilogue of one group hides under the next
