@@ -1085,12 +1085,12 @@ def _gpu_id(torch) -> str:
 
 def _launches_per_step(c) -> int:
     """Kernels one fdl_denoise_step launches at these shapes.  bf16, head
-    dim 128, hidden rows given and at most 128 LM-head rows: the token-shift
+    dim 128, hidden rows given and at most 64 LM-head rows: the token-shift
     gather (if shifting), the fused LM head + commit, and the attention beside
     it; otherwise attention, its partial merge, the gather (if shifting) and
     the LM head."""
     beside = (c["dtype"] == "bf16" and c["head_dim"] == 128
-              and c["batch"] * c["q_len"] <= 128)
+              and c["batch"] * c["q_len"] <= 64)
     return (2 if beside else 3) + (1 if c["shift"] else 0)
 
 

@@ -757,7 +757,10 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   }
   if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
   // This CTA is done: the merge kernel may be scheduled once every CTA got
-  // here (it still waits for the whole grid before reading anything).
+  // here (it still waits for the whole grid before reading a partial).
+  // Triggered at entry instead, the merge's CTAs took the room of retiring
+  // attention CTAs early and the pair ran slower (batch 1, prefix 8192: 34.5
+  // against 18 us).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // When launched beside the step's LM head, finish only after it did, so
   // that this grid's completion (which the merge waits for) covers both.
@@ -860,8 +863,8 @@ __device__ __forceinline__ void merge_split_rows_wide(const TcArgs& a, const int
 
 // Merge of the partials of every item the split spread over several CTAs,
 // launched as a programmatic dependent of the attention grid: its CTAs are
-// scheduled as the attention's retire and wait for the whole grid before
-// reading anything.  At most three CTAs per SM, eight warps each, every warp a
+// scheduled as the attention's retire, rebuild the sequence table from the
+// lengths, and wait for the whole grid before reading a partial.  At most three CTAs per SM, eight warps each, every warp a
 // (item, row) task at a time (few fat CTAs: the launch of one small CTA per
 // (item, row block) cost more than the merge itself; three per SM keep about
 // one task per warp in flight at batch 16).  Warp 0 first rebuilds
@@ -870,7 +873,6 @@ __global__ void __launch_bounds__(256, 3)
 attn_merge_rows_kernel(const TcArgs a) {
   __shared__ int cb[kMaxSeq + 1];
   __shared__ int nc[kMaxSeq];
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_seq = a.Hkv * a.n_rt;
   if (warp == 0) {
@@ -903,6 +905,9 @@ attn_merge_rows_kernel(const TcArgs a) {
     if (lane == 0) cb[a.B] = run;
   }
   __syncthreads();
+  // The lengths are inputs of the attention grid (complete before it began),
+  // the partials its outputs: only these wait for the grid to finish.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   const long long first = (long long)blockIdx.x * (blockDim.x >> 5) + warp;
   if (a.merge_wide)

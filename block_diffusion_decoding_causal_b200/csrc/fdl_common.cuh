@@ -67,9 +67,12 @@ struct alignas(16) Partial {
 };
 
 // Workspace control words (first 256 bytes of the workspace).
+constexpr int kLmTeam = 16;      // LM-head CTAs per first-level merge
+constexpr int kLmMaxTeams = 16;  // teams the control words count for
 struct Control {
-  unsigned int status;     // FDL_DEV_* bits
-  unsigned int lm_ticket;  // LM-head last-CTA ticket
+  unsigned int status;                // FDL_DEV_* bits
+  unsigned int lm_ticket;             // LM-head last-CTA (or last-team) ticket
+  unsigned int lm_team[kLmMaxTeams];  // LM-head per-team tickets
 };
 
 // ----------------------------------------------------------------- attention

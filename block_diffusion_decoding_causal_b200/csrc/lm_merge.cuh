@@ -20,43 +20,90 @@ __device__ __forceinline__ bool last_cta_arrives(unsigned int* ticket,
   return s_last != 0;
 }
 
-// Merge the n_cta partials of each row into (conf, tok); then, when the call
-// is the fused step, commit (technical review, section 4, Algorithm 2).
+// Row r's merge of n partials part[(first + j * stride) * R + r], j < n, in
+// increasing j: one thread per row, sixteen reads in flight at a time (the
+// partials of one source are consecutive rows, so a warp's reads coalesce).
+__device__ __forceinline__ MSI lm_merge_sources(const Partial* part, int R, int r, int first,
+                                                int stride, int n) {
+  MSI st = msi_empty();
+  for (int j0 = 0; j0 < n; j0 += 16) {
+    float4 p[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      if (j0 + u < n)
+        p[u] = __ldcg(reinterpret_cast<const float4*>(
+            part + (size_t)(first + (j0 + u) * stride) * R + r));
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      if (j0 + u < n) st = msi_merge(st, MSI{p[u].x, p[u].y, __float_as_int(p[u].z)});
+  }
+  return st;
+}
+
+// Two-level arrival of the tensor-core LM head's CTAs, after each wrote its
+// partials.  CTAs come in teams of kLmTeam (by index); the last of a team to
+// arrive merges the team's partials row by row, in CTA order, into the slot
+// of the team's first CTA, and then arrives on the grid-wide ticket over the
+// teams.  Returns true in exactly one CTA, the last team's merger, with every
+// team's merged partial visible: it finishes with lm_final_merge(a, kLmTeam).
+// The merges run one thread per row with all of a team's reads in flight, so
+// the tail after the last CTA is two short merges instead of one over every
+// CTA.  Each merger rearms its ticket.  No thread waits on another CTA.
+__device__ __forceinline__ bool lm_team_arrives(const LmArgs& a) {
+  const int team = blockIdx.x / kLmTeam;
+  const int first = team * kLmTeam;
+  const int size = min(kLmTeam, a.n_cta - first);
+  const int n_teams = (a.n_cta + kLmTeam - 1) / kLmTeam;
+  if (!last_cta_arrives(&a.ctrl->lm_team[team], (unsigned int)size)) return false;
+  if (threadIdx.x == 0) a.ctrl->lm_team[team] = 0u;
+  for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
+    const MSI st = lm_merge_sources(a.part, a.R, r, first, 1, size);
+    Partial p;
+    p.m = st.m;
+    p.s = st.s;
+    p.i = st.i;
+    p.pad = 0;
+    a.part[(size_t)first * a.R + r] = p;  // read above by this thread only
+  }
+  if (!last_cta_arrives(&a.ctrl->lm_ticket, (unsigned int)n_teams)) return false;
+  if (threadIdx.x == 0) a.ctrl->lm_ticket = 0u;
+  return true;
+}
+
+// Merge the partials of each row into (conf, tok); then, when the call is
+// the fused step, commit (technical review, section 4, Algorithm 2).  The
+// sources are part[(j * stride) * R + r] for the n_src = ceil(n_cta / stride)
+// values of j: every CTA's own partials (stride 1), or the teams' merged
+// ones (stride kLmTeam, after lm_team_arrives).
 // conf = 1 / sum_v exp(l_v - l_max) is the max softmax probability; the
 // token is the argmax with the lowest vocabulary index on a tie.
 // If a CTA's bounded wait ran out (FDL_DEV_TIMEOUT in the status word, set
 // before its ticket), its partials are stale: every row then reports
 // conf = -1 and tok = -1 and the commit selects nothing (block tokens kept,
 // counts written), until the caller reads and clears the status word.
-__device__ __forceinline__ void lm_final_merge(const LmArgs& a) {
+__device__ __forceinline__ void lm_final_merge(const LmArgs& a, int stride = 1) {
   __shared__ float s_conf[kMaxRows];
   __shared__ int s_tok[kMaxRows];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = blockDim.x >> 5;
+  const int n_src = (a.n_cta + stride - 1) / stride;
   const bool timed_out =
       (*reinterpret_cast<volatile unsigned int*>(&a.ctrl->status) & FDL_DEV_TIMEOUT) != 0u;
-  for (int r = warp; r < a.R; r += nw) {
-    MSI st = msi_empty();
-    for (int c = lane; c < a.n_cta; c += 32) {
-      const float4 p = __ldcg(reinterpret_cast<const float4*>(a.part + (size_t)c * a.R + r));
-      st = msi_merge(st, MSI{p.x, p.y, __float_as_int(p.z)});
+  for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
+    const MSI st = lm_merge_sources(a.part, a.R, r, 0, stride, n_src);
+    bool act = true;
+    if (a.row_active != nullptr) act = a.row_active[r] != 0;
+    if (a.block_tokens_in != nullptr) {
+      const int b = r / a.q_len, i = r % a.q_len;
+      act = a.block_tokens_in[(size_t)b * a.D + a.q_off + i] == a.mask_id;
     }
-    st = msi_warp_allmerge(st);
-    if (lane == 0) {
-      bool act = true;
-      if (a.row_active != nullptr) act = a.row_active[r] != 0;
-      if (a.block_tokens_in != nullptr) {
-        const int b = r / a.q_len, i = r % a.q_len;
-        act = a.block_tokens_in[(size_t)b * a.D + a.q_off + i] == a.mask_id;
-      }
-      act = act && !timed_out;
-      const float c = act ? 1.0f / st.s : -1.0f;
-      const int t = act ? st.i : -1;
-      a.conf[r] = c;
-      a.tok[r] = t;
-      s_conf[r] = c;
-      s_tok[r] = t;
-    }
+    act = act && !timed_out;
+    const float c = act ? 1.0f / st.s : -1.0f;
+    const int t = act ? st.i : -1;
+    a.conf[r] = c;
+    a.tok[r] = t;
+    s_conf[r] = c;
+    s_tok[r] = t;
   }
   if (!a.commit) return;
   __syncthreads();

@@ -25,8 +25,9 @@
 //            bounds the kernel, the 32 x 32 block is transposed through
 //            shared memory instead and lane j folds column j's 32 logits into
 //            its running state one at a time (one exponential per logit).
-// The per-CTA triples go to the workspace; the last CTA to arrive merges them
-// (and, in the fused step, commits).  No thread waits on another CTA.
+// The per-CTA triples go to the workspace; the last CTA of each team of 16
+// merges its team's, the last team's merger merges the teams' (and, in the
+// fused step, commits).  No thread waits on another CTA.
 #include "lm_merge.cuh"
 #include "sm100.cuh"
 
@@ -365,9 +366,8 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
     tmem_dealloc(tmem, tp.tmem_cols);
   }
   if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
-  if (!last_cta_arrives(&a.ctrl->lm_ticket, a.n_cta)) return;
-  lm_final_merge(a);
-  if (threadIdx.x == 0) a.ctrl->lm_ticket = 0u;
+  if (!lm_team_arrives(a)) return;
+  lm_final_merge(a, kLmTeam);
 }
 
 // The LM head over CTA pairs (from 129 rows on, full form).  The two CTAs of
@@ -614,9 +614,8 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
     tmem_dealloc_pair(tmem, tp.tmem_cols);
   }
   if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
-  if (!last_cta_arrives(&a.ctrl->lm_ticket, a.n_cta)) return;
-  lm_final_merge(a);
-  if (threadIdx.x == 0) a.ctrl->lm_ticket = 0u;
+  if (!lm_team_arrives(a)) return;
+  lm_final_merge(a, kLmTeam);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -772,9 +771,10 @@ bool lmhead_tc2_params(int npad, int H, TcParams* tp, size_t* smem) {
 // kernels stream HBM side by side.  Its shared memory is what is left of
 // the SM's 228 KB after that CTA and the two per-CTA reservations, and must
 // exceed half the SM (so two LM-head CTAs never share one); TMEM stays within
-// 256 columns (R <= 128: one tile per buffer from 65 rows on) and registers
-// within 168 per thread.  The widest K stage (4, 2 or 1 boxes of 64) that
-// still fits two weight stages is taken.
+// 256 columns and registers within 168 per thread (R <= 64: at 128 rows the
+// attention beside the LM head cost more than running it before, 339 against
+// 270 us a batch-16 step at prefix 2048).  The widest K stage (4, 2 or 1
+// boxes of 64) that still fits two weight stages is taken.
 bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcParams* tp,
                       size_t* smem);
 
@@ -788,7 +788,7 @@ bool lmhead_tc_params(int R, int H, int rows_per_cta, size_t beside_smem, TcPara
   const bool shared = beside_smem > 0;
   int nch = 1;
   while (nch * 32 < R) nch *= 2;
-  if (nch > (shared ? 4 : 8)) return false;
+  if (nch > (shared ? 2 : 8)) return false;
   tp->npad = nch * 32;
   // Tiles per TMEM buffer: about half a CTA's range, so each X chunk serves
   // several weight tiles and the epilogue of one group hides under the next
@@ -888,6 +888,7 @@ cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem
                              bool after_producer) {
   TcParams tp;
   size_t smem = 0;
+  if (a.n_cta > kLmTeam * kLmMaxTeams) return cudaErrorInvalidValue;  // team tickets
   // From 129 rows on (full form): CTA pairs sharing each X chunk.  At 256
   // rows (7B vocabulary) 327 us a pass against 348 us for one CTA; at 128
   // rows the pair measured no faster (232 against 228 us) and the one-CTA
