@@ -12,9 +12,10 @@
 // takes its own, so the split follows the actual lengths and a CTA produces
 // at most two partial results (its first and last item); items it covers
 // whole are written out directly.  Per chunk:
-//   warp 0   TMA: K and V [64 keys x 128] as one 32 KB stage (four 8 KB boxes,
-//            128-byte swizzle, one barrier) through a STAGES-deep ring; Q of
-//            each item by a 3D box (d, head group, positions);
+//   warp 0   TMA: K and V [64 keys x 128] into one 32 KB stage (four 8 KB
+//            boxes, 128-byte swizzle) of a STAGES-deep ring, a barrier pair
+//            per half: S frees the K half, P V the V half; Q of each item by
+//            a 3D box (d, head group, positions);
 //   warp 1   tcgen05.mma: S = Q K^T (M 128, N 64, K 128) into one of two TMEM
 //            S buffers, then, one chunk behind, O += P V (M 128, N 128, K 64)
 //            with P read from TMEM and V MN-major from shared memory, into
@@ -79,6 +80,7 @@ struct TcArgs {
   float2* part_ml;        // [2 * n_cta][128]
   int inline_merge;       // the last CTA to finish a row of an item merges it
   int merge_wide;         // merge kernel: lanes over partials (many per item)
+  int v_lag;              // V loads issued this many chunks behind K (0 or 1)
   int q_region;           // bytes between the two d-halves of the Q buffer
 };
 
@@ -87,7 +89,8 @@ struct Maps {
 };
 
 struct Smem {
-  uint64_t kv_full[kMaxStages], kv_empty[kMaxStages];
+  uint64_t k_full[kMaxStages], k_empty[kMaxStages];  // K half of a stage: free after S
+  uint64_t v_full[kMaxStages], v_empty[kMaxStages];  // V half: free after P V
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[kSB], s_empty[kSB];   // S ready / S and its P free again
   uint64_t p_full[kSB];                 // P written into TMEM
@@ -358,8 +361,10 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&S.kv_full[i], 1);
-      mbar_init(&S.kv_empty[i], 1);
+      mbar_init(&S.k_full[i], 1);
+      mbar_init(&S.k_empty[i], 1);
+      mbar_init(&S.v_full[i], 1);
+      mbar_init(&S.v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.q_full[i], 1);
@@ -437,47 +442,71 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
 
   if (c_begin < c_end && warp == 0) {
     // -------------------------------------------------------------- TMA
-    // One 32 KB stage per chunk (K and V, four boxes, one barrier): the TMA
-    // engine streams far faster with few large stages than many small ones.
+    // A stage holds one chunk's K and V (16 KB each, two 8 KB boxes), with a
+    // barrier per half: S = Q K^T releases the K half, P V the V half, so the
+    // next K streams in while this chunk's softmax still runs.  Issue order
+    // K(j), V(j - v_lag).  With 128-row tiles (compute-heavy) v_lag = 1: K's
+    // slot frees (S(j - STAGES) done) before V's does, so K does not wait
+    // behind V's slot (PrefixCache 42.7 -> 37.8 us); streaming decode keeps
+    // each chunk's K and V together (v_lag = 0), V on time for its P V.
     if (lane == 0) {
       const int n_my = (int)(c_end - c_begin);
+      const int lag = a.v_lag;
       int q_i = 0, prev_x = -1;
-      Cursor c = locate(cb, nc, a.B, c_begin);
-      for (int i = 0; i < n_my && !failed; ++i, advance(c, nc, per_seq)) {
-        const int x = c.b * per_seq + c.it;
-        const int kvh = c.it / a.n_rt, rt = c.it % a.n_rt;
-        const int slot = i % STAGES;
-        if (!mbar_wait(&S.kv_empty[slot], ((i / STAGES) & 1) ^ 1)) { failed = true; break; }
-        const ChunkInfo ci = chunk_info(c.j, lp[c.b], ls[c.b], a.D);
-        const int bk = c.b * a.Hkv + kvh;
-        const CUtensorMap* mk = ci.seg == 0 ? &maps.kp : (ci.seg == 1 ? &maps.kb : &maps.ks);
-        const CUtensorMap* mv = ci.seg == 0 ? &maps.vp : (ci.seg == 1 ? &maps.vb : &maps.vs);
-        const int row = ci.seg == 0 ? bk * a.cap_p + ci.key0
-                                    : (ci.seg == 1 ? bk * a.D + ci.key0 : bk * a.cap_s + ci.key0);
-        uint8_t* dst = kv_smem + slot * kKVSlot;
-        mbar_arrive_expect_tx(&S.kv_full[slot], kKVSlot);
-        tma_load_2d(dst, mk, 0, row, &S.kv_full[slot]);
-        tma_load_2d(dst + kKVRegion, mk, 64, row, &S.kv_full[slot]);
-        tma_load_2d(dst + 2 * kKVRegion, mv, 0, row, &S.kv_full[slot]);
-        tma_load_2d(dst + 3 * kKVRegion, mv, 64, row, &S.kv_full[slot]);
-        // A new item's Q goes after its first K/V, so that load overlaps the
-        // wait for the previous item's last S to release the Q buffer.
-        if (x != prev_x) {
-          const int qb = q_i % kQBufs;
-          if (!mbar_wait(&S.q_empty[qb], ((q_i / kQBufs) & 1) ^ 1)) { failed = true; break; }
-          mbar_arrive_expect_tx(&S.q_full[qb], 2u * 128u * (uint32_t)rows_full);
-          const int z = c.b * a.q_len + rt * a.qpt;
-          tma_load_3d(q_smem + qb * 2 * a.q_region, &maps.q, 0, kvh * a.group, z,
-                      &S.q_full[qb]);
-          tma_load_3d(q_smem + qb * 2 * a.q_region + a.q_region, &maps.q, 64, kvh * a.group, z,
-                      &S.q_full[qb]);
-          ++q_i;
-          prev_x = x;
+      Cursor ck = locate(cb, nc, a.B, c_begin), cv = ck;
+      for (int j = 0; j < n_my + lag && !failed; ++j) {
+        if (j < n_my) {
+          const int x = ck.b * per_seq + ck.it;
+          const int kvh = ck.it / a.n_rt, rt = ck.it % a.n_rt;
+          const int slot = j % STAGES;
+          if (!mbar_wait(&S.k_empty[slot], ((j / STAGES) & 1) ^ 1)) { failed = true; break; }
+          const ChunkInfo ci = chunk_info(ck.j, lp[ck.b], ls[ck.b], a.D);
+          const int bk = ck.b * a.Hkv + kvh;
+          const CUtensorMap* mk = ci.seg == 0 ? &maps.kp : (ci.seg == 1 ? &maps.kb : &maps.ks);
+          const int row = ci.seg == 0 ? bk * a.cap_p + ci.key0
+                                      : (ci.seg == 1 ? bk * a.D + ci.key0 : bk * a.cap_s + ci.key0);
+          uint8_t* dst = kv_smem + slot * kKVSlot;
+          mbar_arrive_expect_tx(&S.k_full[slot], 2 * kKVRegion);
+          tma_load_2d(dst, mk, 0, row, &S.k_full[slot]);
+          tma_load_2d(dst + kKVRegion, mk, 64, row, &S.k_full[slot]);
+          // A new item's Q goes after its first K, so that load overlaps the
+          // wait for the previous item's last S to release the Q buffer.
+          if (x != prev_x) {
+            const int qb = q_i % kQBufs;
+            if (!mbar_wait(&S.q_empty[qb], ((q_i / kQBufs) & 1) ^ 1)) { failed = true; break; }
+            mbar_arrive_expect_tx(&S.q_full[qb], 2u * 128u * (uint32_t)rows_full);
+            const int z = ck.b * a.q_len + rt * a.qpt;
+            tma_load_3d(q_smem + qb * 2 * a.q_region, &maps.q, 0, kvh * a.group, z,
+                        &S.q_full[qb]);
+            tma_load_3d(q_smem + qb * 2 * a.q_region + a.q_region, &maps.q, 64, kvh * a.group, z,
+                        &S.q_full[qb]);
+            ++q_i;
+            prev_x = x;
+          }
+          advance(ck, nc, per_seq);
+        }
+        if (j >= lag) {
+          const int i = j - lag;
+          const int kvh = cv.it / a.n_rt;
+          const int slot = i % STAGES;
+          if (!mbar_wait(&S.v_empty[slot], ((i / STAGES) & 1) ^ 1)) { failed = true; break; }
+          const ChunkInfo ci = chunk_info(cv.j, lp[cv.b], ls[cv.b], a.D);
+          const int bk = cv.b * a.Hkv + kvh;
+          const CUtensorMap* mv = ci.seg == 0 ? &maps.vp : (ci.seg == 1 ? &maps.vb : &maps.vs);
+          const int row = ci.seg == 0 ? bk * a.cap_p + ci.key0
+                                      : (ci.seg == 1 ? bk * a.D + ci.key0 : bk * a.cap_s + ci.key0);
+          uint8_t* dst = kv_smem + slot * kKVSlot + 2 * kKVRegion;
+          mbar_arrive_expect_tx(&S.v_full[slot], 2 * kKVRegion);
+          tma_load_2d(dst, mv, 0, row, &S.v_full[slot]);
+          tma_load_2d(dst + kKVRegion, mv, 64, row, &S.v_full[slot]);
+          advance(cv, nc, per_seq);
         }
       }
       // Drain: every load issued has landed before this CTA can exit.
-      for (int m = max(0, n_my - STAGES); m < n_my; ++m)
-        if (!mbar_wait(&S.kv_full[m % STAGES], (m / STAGES) & 1)) failed = true;
+      for (int m = max(0, n_my - STAGES); m < n_my; ++m) {
+        if (!mbar_wait(&S.k_full[m % STAGES], (m / STAGES) & 1)) failed = true;
+        if (!mbar_wait(&S.v_full[m % STAGES], (m / STAGES) & 1)) failed = true;
+      }
       for (int m = max(0, q_i - kQBufs); m < q_i; ++m)
         if (!mbar_wait(&S.q_full[m % kQBufs], (m / kQBufs) & 1)) failed = true;
     }
@@ -500,7 +529,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
           const bool first = x != prev_xs;
           const int slot = is % STAGES, sb = is % kSB;
           bool ready = first ? mbar_test(&S.q_full[q_s % kQBufs], (q_s / kQBufs) & 1) : true;
-          ready = ready && mbar_test(&S.kv_full[slot], (is / STAGES) & 1) &&
+          ready = ready && mbar_test(&S.k_full[slot], (is / STAGES) & 1) &&
                   mbar_test(&S.s_empty[sb], ((is / kSB) & 1) ^ 1);
           if (ready) {
             if (first) {
@@ -519,6 +548,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
                        desc_k_sw128(k_base + (k >> 2) * kKVRegion + (k & 3) * 32), id_s,
                        k ? 1u : 0u);
             mma_commit(&S.s_full[sb]);
+            mma_commit(&S.k_empty[slot]);
             if (last) mma_commit(&S.q_empty[qb]);
             advance(cs, nc, per_seq);
             ++is;
@@ -529,7 +559,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
           const int x = cp.b * per_seq + cp.it;
           const bool first = x != prev_xp;
           const int pb = ip % kSB, vslot = ip % STAGES;
-          bool ready = mbar_test(&S.p_full[pb], (ip / kSB) & 1);
+          bool ready = mbar_test(&S.p_full[pb], (ip / kSB) & 1) &&
+                       mbar_test(&S.v_full[vslot], (ip / STAGES) & 1);
           if (first) ready = ready && mbar_test(&S.o_empty[0], (o_i & 1) ^ 1);
           if (ready) {
             if (first) prev_xp = x;
@@ -542,7 +573,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
             for (int k = 0; k < kCh / 16; ++k)  // 16 keys = 8 packed columns of P
               mma_bf16_ts(d_o, p_tmem + k * 8, desc_mn_sw128(v_base + k * 2048, kKVRegion, 1024),
                           id_pv, (first && k == 0) ? 0u : 1u);
-            mma_commit(&S.kv_empty[vslot]);
+            mma_commit(&S.v_empty[vslot]);
             mma_commit(&S.s_empty[pb]);
             if (last) {
               mma_commit(&S.o_full[0]);
@@ -1066,6 +1097,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   t.part_ml = part_ml;
   t.inline_merge = beside_prior ? 1 : 0;
   t.merge_wide = 0;
+  t.v_lag = qpt * a.group > 64 ? 1 : 0;
   t.q_region = q_region_for(qpt * a.group);
   // Beside the LM head: one K/V stage, so the SM's remaining shared memory
   // goes to that kernel's weight ring.

@@ -444,10 +444,12 @@ LARGE_BATCH = dict(batch=40, n_q_heads=8, n_kv_heads=2, head_dim=128, block_size
                    w_scale=8.0, dtype="bf16", masked=(1, 8))
 
 
-def test_fused_step_with_two_lm_passes():
+@pytest.mark.parametrize("shift", [1, 0])
+def test_fused_step_with_two_lm_passes(shift):
     """A fused step with 320 LM-head rows (passes of 256 and 64 rows, each
-    committing its own sequences) against the oracle, bit-exact commits."""
-    case, ref, _ = cases.parity_case("large_batch", 0, cfg=LARGE_BATCH)
+    committing its own sequences) against the oracle, bit-exact commits,
+    with and without the token-shift gather before the LM head."""
+    case, ref, _ = cases.parity_case("large_batch", 0, cfg=dict(LARGE_BATCH, shift=shift))
     gh.compare_step(case, gh.run_denoise_step(case), ref)
 
 
