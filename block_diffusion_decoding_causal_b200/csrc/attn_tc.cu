@@ -910,6 +910,10 @@ __global__ void __launch_bounds__(256, 3)
 attn_merge_rows_kernel(const TcArgs a) {
   __shared__ int cb[kMaxSeq + 1];
   __shared__ int nc[kMaxSeq];
+  // The step's LM head, launched behind this grid when its rows do not come
+  // from the attention, may start on the SM room these CTAs leave; it
+  // touches nothing this grid reads or writes.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_seq = a.Hkv * a.n_rt;
   if (warp == 0) {

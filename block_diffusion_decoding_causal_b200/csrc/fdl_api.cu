@@ -540,10 +540,15 @@ int fdl_denoise_step(const fdl_step_cfg* cfg, const void* q, const void* k_pre,
                          len_suf, out, ws, s, true);
       return rc != FDL_OK ? rc : ok();
     }
+    // Too many rows for the shared form: the gather (already launched), the
+    // attention and its merge, then the LM head as a programmatic dependent
+    // of the merge, streaming the weight from the rows gathered before the
+    // attention began while the merge still runs.
     rc = run_attention(c, p, dual, q, k_pre, v_pre, len_pre, k_blk, v_blk, k_suf, v_suf,
                        len_suf, out, ws, s);
     if (rc != FDL_OK) return rc;
-    rc = run_lmhead_passes(a, c, p, s);
+    a.rows_ready = 1;
+    rc = run_lmhead_passes(a, c, p, s, true);
     return rc != FDL_OK ? rc : ok();
   }
 

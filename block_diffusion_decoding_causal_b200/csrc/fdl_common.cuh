@@ -115,6 +115,9 @@ struct LmArgs {
   int n_cta;
   int rows_per_cta;          // vocab rows per CTA (multiple of 16)
   int w_packed;              // w in the tiled layout of fdl_lmhead_pack_weight
+  int rows_ready;            // tensor-core LM head: the rows were in place before
+                             // its programmatic predecessor began, so it reads
+                             // them without waiting for that grid
   // fused commit (when commit != 0)
   int commit;
   int32_t* block_tokens;

@@ -175,7 +175,9 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
       tma_prefetch_desc(&tm_x);
       const uint64_t pol_w = policy_evict_first();
       int ia = 0, ib = 0;
-      bool x_ready = false;  // the kernel before this one (the gather) finished
+      // The kernel before this one (the gather) finished, or the rows were
+      // in place before that kernel began.
+      bool x_ready = a.rows_ready != 0;
       auto load_x = [&](int kc) {
         if (!x_ready) {
           asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -455,7 +457,7 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
       const uint64_t pol_x = policy_evict_last();
       // The rows may come from the kernel launched just before this one (the
       // token-shift gather, programmatic launch); without one this returns.
-      asm volatile("griddepcontrol.wait;" ::: "memory");
+      if (!a.rows_ready) asm volatile("griddepcontrol.wait;" ::: "memory");
       int ia = 0, ib = 0;
       for (int g = 0; g < n_groups && !failed; ++g) {
         const int t0 = g * G, t1 = min(n_tiles, t0 + G);
