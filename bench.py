@@ -953,7 +953,8 @@ def sweep_leg(torch, fdl, synth, stream, timed, world, steps, peaks, w8, seed,
                               == c["mask_id"]).sum())
                 for i in range(3):
                     step(i)
-                s_us = rounds_us(timed, step, steps, reps, world)
+                with ClockSampler(_gpu_id(torch)) as clk:
+                    s_us = rounds_us(timed, step, steps, reps, world)
                 s_bytes = a_bytes + lm_bytes + (2 * B * c["q_len"] * c["hidden"] * 2)
                 points.append({
                     "batch": B, "prefix": P, "scale": sc,
@@ -968,7 +969,8 @@ def sweep_leg(torch, fdl, synth, stream, timed, world, steps, peaks, w8, seed,
                     "step": {"us": spread(s_us),
                              "positions_per_s": B * c["q_len"] / statistics.median(s_us) * 1e6,
                              "frac_hbm": s_bytes / statistics.median(s_us) / 1e3
-                             / peaks["hbm_gbs"]},
+                             / peaks["hbm_gbs"],
+                             "clocks": clk.summary()},
                     "masked_in_unit": masked,
                     "committed_per_step": int(n_c.sum()),
                     "committed_per_sequence": (n_c.float().mean().item()),
