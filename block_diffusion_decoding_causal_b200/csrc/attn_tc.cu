@@ -25,11 +25,11 @@
 //            grows by more than 2^8), P = exp2(S - m) as bf16 written back
 //            over its S columns, and the item epilogue.
 // Partial results (unnormalised O, m, l) go to the workspace.  Alone on the
-// GPU (two CTAs per SM, two stages each) a small merge kernel, launched as a
-// programmatic dependent of this grid, combines them.  Beside the LM head
-// (one CTA per SM, one stage, leaving the SM's other room to that kernel)
-// the thread that writes a row's last partial merges the row itself.
-// No thread waits on another CTA.
+// GPU (two CTAs per SM, three stages each where they fit, else two) a
+// grid-stride merge kernel, launched as a programmatic dependent of this
+// grid, combines them.  Beside the LM head (one CTA per SM, one stage,
+// leaving the SM's other room to that kernel) the thread that writes a row's
+// last partial merges the row itself.  No thread waits on another CTA.
 #include <cudaTypedefs.h>
 
 #include <mutex>

@@ -1,5 +1,6 @@
-// Last-CTA merge of the LM-head partials, confidence/token output and the
-// fused commit.  Shared by the CUDA-core and the tensor-core LM-head kernels.
+// Merge of the LM-head partials (by the last CTA to arrive, or in two levels
+// by teams of CTAs), confidence/token output and the fused commit.  Shared
+// by the CUDA-core and the tensor-core LM-head kernels.
 #pragma once
 
 #include "fdl_common.cuh"
