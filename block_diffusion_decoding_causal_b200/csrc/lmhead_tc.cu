@@ -44,6 +44,7 @@ constexpr int kTileM = 128;                 // vocab rows per MMA tile
 constexpr int kKChunk = 64;                 // bf16 per 128-byte row
 constexpr int kStageA = kTileM * kKChunk * 2;  // 16 KB
 constexpr int kBoxPart = 16;                // rows per box of a partial tile
+constexpr int kTail = 16;                   // short last tile of the CTA-pair form
 constexpr int kThreads = 192;
 constexpr unsigned kDevTimeout = FDL_DEV_TIMEOUT;
 
@@ -387,20 +388,34 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
 //   empty_a / empty_b in each CTA: the MMA commits to both;
 //   acc_full          in each CTA: the MMA commits to both;
 //   acc_empty         on the even CTA: both CTAs' epilogue threads arrive.
+// Short last tile.  A range of 128 k + t rows with 0 < t <= kTail (t = 16
+// at the Qwen2.5 vocabulary over 148 CTAs) would spend a whole M = 256 tile
+// of MMAs on t rows.  Instead the t rows of each CTA ride along with the
+// first tile with the operands swapped: A = the X chunk already staged (this
+// CTA's 128 X rows), B = the two CTAs' t-row weight pieces (kTail rows each,
+// N = 2 kTail), D in the first 2 kTail columns of the second TMEM buffer,
+// which the first tile leaves free.  Lane = X row there, so the epilogue
+// folds those 2 kTail vocabulary entries into its own X rows' states, the
+// even CTA's entries before the odd CTA's; every (X row, vocabulary row)
+// pair is still counted once.  The MMA waits for those columns (tail_empty)
+// before the second tile.
 template <int NCH, int KSUB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
+                  const __grid_constant__ CUtensorMap tm_w_tail,
                   const __grid_constant__ CUtensorMap tm_x, const LmArgs a, const TcParams tp) {
   constexpr int NPAD = NCH * 32;
   constexpr int NH = NPAD / 2;                    // X rows this CTA stages
   constexpr int SA_BYTES = kStageA * KSUB;        // one A stage: 128 rows x 64*KSUB
+  constexpr int TAIL_BYTES = kTail * 128 * KSUB;  // short-tile rows of one A stage
+  constexpr int SA_STRIDE = SA_BYTES + TAIL_BYTES;
   constexpr int SB_BYTES = NH * 128 * KSUB;       // one B stage: NH rows x 64*KSUB
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int SA = tp.stages_a, SB = tp.stages_b;
   uint8_t* sa = smem;
-  uint8_t* sb = sa + SA * SA_BYTES;
+  uint8_t* sb = sa + SA * SA_STRIDE;
   uint64_t* full_a = reinterpret_cast<uint64_t*>(sb + SB * SB_BYTES);
   uint64_t* empty_a = full_a + SA;
   uint64_t* full_b = empty_a + SA;
@@ -408,8 +423,10 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
   uint64_t* acc_full = empty_b + SB;   // [2]
   uint64_t* acc_empty = acc_full + 2;  // [2]
   uint64_t* drain = acc_empty + 2;     // [1]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-  MSI* s_red = reinterpret_cast<MSI*>(tmem_holder + 4);  // [4][NPAD]
+  uint64_t* tail_empty = drain + 1;    // [1]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tail_empty + 1);
+  MSI* s_red = reinterpret_cast<MSI*>(tmem_holder + 4);  // [4][NPAD], then [NH] short tile
+  static_assert((4 * NPAD + NH) * sizeof(MSI) <= red_bytes(NPAD), "epilogue states fit");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -419,7 +436,10 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
   // The pair steps through the same number of tiles: the larger range's.
   const int pair0 = (blockIdx.x & ~1) * a.rows_per_cta;
   const int pair_rows = max(0, min(a.V, pair0 + a.rows_per_cta) - pair0);
-  const int n_tiles = (pair_rows + kTileM - 1) / kTileM;
+  // Short last tile folded into the first one (same decision in both CTAs).
+  const int t_rows = pair_rows % kTileM;
+  const bool fold = pair_rows > kTileM && t_rows > 0 && t_rows <= kTail;
+  const int n_tiles = fold ? pair_rows / kTileM : (pair_rows + kTileM - 1) / kTileM;
   const int G = tp.group;
   const int n_groups = (n_tiles + G - 1) / G;
   const int KC = a.H / (kKChunk * KSUB);
@@ -439,6 +459,7 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
       mbar_init(&acc_empty[i], 256);
     }
     mbar_init(drain, 1);
+    mbar_init(tail_empty, 256);
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc_pair(tmem_holder, tp.tmem_cols);
@@ -452,6 +473,7 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
     // ------------------------------------------------------ TMA producer
     if (lane == 0 && n_tiles > 0) {
       tma_prefetch_desc(&tm_w_full);
+      tma_prefetch_desc(&tm_w_tail);
       tma_prefetch_desc(&tm_x);
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
@@ -475,12 +497,31 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
           }
           for (int t = t0; t < t1; ++t) {
             const int slot_a = ia % SA;
+            const bool with_tail = fold && t == 0;
             if (!mbar_wait(&empty_a[slot_a], ((ia / SA) & 1) ^ 1)) { failed = true; break; }
-            if (leader) mbar_arrive_expect_tx(&full_a[slot_a], 2 * SA_BYTES);
+            if (leader)
+              mbar_arrive_expect_tx(&full_a[slot_a],
+                                    2 * (SA_BYTES + (with_tail ? TAIL_BYTES : 0)));
             const uint32_t bar = mapa_shared(smem_u32(&full_a[slot_a]), 0u);
             const int row0 = v0 + t * kTileM;
             const int rt = max(0, min(kTileM, v1 - row0));  // rows of the tile (packed layout)
-            uint8_t* dst = sa + slot_a * SA_BYTES;
+            uint8_t* dst = sa + slot_a * SA_STRIDE;
+            if (with_tail) {
+              // This CTA's short-tile rows (a full kTail box; rows past its
+              // range read the next chunk's pieces or zeros, masked later).
+              const int trow0 = v0 + n_tiles * kTileM;
+              const int trt = max(0, min(kTileM, v1 - trow0));
+#pragma unroll
+              for (int u = 0; u < KSUB; ++u) {
+                const int kk = kc * KSUB + u;
+                if (a.w_packed)
+                  tma_load_2d_pair(dst + SA_BYTES + u * kTail * 128, &tm_w_tail, 0,
+                                   trow0 * KCT + kk * trt, bar, pol_w);
+                else
+                  tma_load_2d_pair(dst + SA_BYTES + u * kTail * 128, &tm_w_tail, kk * kKChunk,
+                                   trow0, bar, pol_w);
+              }
+            }
 #pragma unroll
             for (int u = 0; u < KSUB; ++u) {
               const int kk = kc * KSUB + u;
@@ -514,11 +555,13 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
     // ------------------------------------------- MMA issuer (even CTA)
     if (leader && lane == 0 && n_tiles > 0) {
       const uint32_t idesc = idesc_bf16_f32(2 * kTileM, NPAD);
+      const uint32_t idesc_tail = idesc_bf16_f32(2 * kTileM, 2 * kTail);
       int ia = 0, ib = 0;
       for (int g = 0; g < n_groups && !failed; ++g) {
         const int buf = tp.nbuf == 2 ? (g & 1) : 0;
         const uint32_t ph = tp.nbuf == 2 ? ((g >> 1) & 1) : (g & 1);
         if (!mbar_wait(&acc_empty[buf], ph ^ 1)) { failed = true; break; }
+        if (fold && g == 1 && !mbar_wait(tail_empty, 0)) { failed = true; break; }
         tc_fence_after();
         const int t0 = g * G, t1 = min(n_tiles, t0 + G);
         for (int kc = 0; kc < KC && !failed; ++kc) {
@@ -530,8 +573,18 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
             const int slot_a = ia % SA;
             if (!mbar_wait(&full_a[slot_a], (ia / SA) & 1)) { failed = true; break; }
             tc_fence_after();
-            const uint32_t a_base = smem_u32(sa + slot_a * SA_BYTES);
+            const uint32_t a_base = smem_u32(sa + slot_a * SA_STRIDE);
             const uint32_t d = tmem + (uint32_t)((buf * G + (t - t0)) * NPAD);
+            if (fold && t == 0) {
+              // Short tile, operands swapped: X rows x (kTail + kTail) rows.
+#pragma unroll
+              for (int u = 0; u < KSUB; ++u)
+#pragma unroll
+                for (int k = 0; k < kKChunk / 16; ++k)
+                  mma_bf16_pair(tmem + (uint32_t)NPAD, desc_k_sw128(b_base + u * NH * 128 + k * 32),
+                                desc_k_sw128(a_base + SA_BYTES + u * kTail * 128 + k * 32),
+                                idesc_tail, (kc | u | k) != 0 ? 1u : 0u);
+            }
 #pragma unroll
             for (int u = 0; u < KSUB; ++u)
 #pragma unroll
@@ -559,11 +612,31 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
     MSI st[NCH];
 #pragma unroll
     for (int c = 0; c < NCH; ++c) st[c] = msi_empty();
+    MSI st_tail = msi_empty();  // X row rank * NH + q * 32 + lane, short-tile entries
     for (int g = 0; g < n_groups; ++g) {
       const int buf = tp.nbuf == 2 ? (g & 1) : 0;
       const uint32_t ph = tp.nbuf == 2 ? ((g >> 1) & 1) : (g & 1);
       if (!mbar_wait(&acc_full[buf], ph)) { failed = true; break; }
       tc_fence_after();
+      if (fold && g == 0) {
+        // Columns j < kTail: the even CTA's short-tile rows, j >= kTail the
+        // odd CTA's, each in increasing vocabulary order.
+        uint32_t r[32];
+        static_assert(2 * kTail == 32, "one 32-column load holds the short tile");
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)NPAD, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c0 = (blockIdx.x & ~1) + h;
+          const int tv0 = c0 * a.rows_per_cta + n_tiles * kTileM;
+          const int tv1 = min(a.V, c0 * a.rows_per_cta + a.rows_per_cta);
+#pragma unroll
+          for (int j = 0; j < kTail; ++j)
+            if (tv0 + j < tv1) msi_push(st_tail, __uint_as_float(r[h * kTail + j]), tv0 + j);
+        }
+        tc_fence_before();
+        mbar_arrive_cluster(mapa_shared(smem_u32(tail_empty), 0u));
+      }
       const int t0 = g * G, t1 = min(n_tiles, t0 + G);
       for (int t = t0; t < t1; ++t) {
         const int vbase = v0 + t * kTileM + q * 32;
@@ -592,11 +665,15 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
     named_barrier_epilogue();
 #pragma unroll
     for (int c = 0; c < NCH; ++c) s_red[q * NPAD + c * 32 + lane] = st[c];
+    MSI* s_tail = s_red + 4 * NPAD;  // [NH], this CTA's X rows
+    s_tail[q * 32 + lane] = st_tail;
     named_barrier_epilogue();
     for (int col = threadIdx.x - 64; col < NPAD; col += 128) {
       MSI m = s_red[col];
 #pragma unroll
       for (int j = 1; j < 4; ++j) m = msi_merge(m, s_red[j * NPAD + col]);
+      const int xl = col - (int)rank * NH;
+      if (xl >= 0 && xl < NH) m = msi_merge(m, s_tail[xl]);
       if (col < a.R) {
         Partial p;
         p.m = m.m;
@@ -710,8 +787,9 @@ cudaError_t launch_nch(const CUtensorMap& wf, const CUtensorMap& wp, const CUten
 }
 
 template <int NCH, int KSUB>
-cudaError_t launch_pair(const CUtensorMap& wf, const CUtensorMap& x, const LmArgs& a,
-                        const TcParams& tp, size_t smem, cudaStream_t s, bool after_producer) {
+cudaError_t launch_pair(const CUtensorMap& wf, const CUtensorMap& wt, const CUtensorMap& x,
+                        const LmArgs& a, const TcParams& tp, size_t smem, cudaStream_t s,
+                        bool after_producer) {
   auto k = lmhead_tc2_kernel<NCH, KSUB>;
   static std::mutex mu;
   static size_t smem_set[64] = {};
@@ -737,30 +815,36 @@ cudaError_t launch_pair(const CUtensorMap& wf, const CUtensorMap& x, const LmArg
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = after_producer ? 1 : 0;
-  return cudaLaunchKernelEx(&lc, k, wf, x, a, tp);
+  return cudaLaunchKernelEx(&lc, k, wf, wt, x, a, tp);
 }
 
 // Ring shapes of the CTA-pair form (256 padded rows, full form): two-box K
-// stages (32 KB weight stages; X stages of half the rows), one tile per TMEM
-// buffer, two buffers, about 192 KB of rings.  (Other shapes measured at 256
-// rows: 3 + 3 stages 327 us; 4 weight + 2 X stages 350 us; two tiles per
-// buffer sharing each X chunk 334 us; a single X stage 490-560 us.)
+// stages (32 KB weight stages, each with room for the short tile's 2 x 2 KB;
+// X stages of half the rows), one tile per TMEM buffer, two buffers, about
+// 204 KB of rings.  With the short tile folded into the first one the 7B
+// vocabulary takes eight tiles per CTA instead of nine: 287 -> 275 us a pass
+// at 256 rows on one box.  (Other shapes measured at 256 rows, before the
+// fold: 3 + 3 stages 327 us; 4 weight + 2 X stages 350 us; 4 + 3 stages with
+// the epilogue reducing in registers to make room, no faster than 3 + 3;
+// two tiles per buffer sharing each X chunk 334 us; a single X stage
+// 490-560 us.)
 bool lmhead_tc2_params(int npad, int H, TcParams* tp, size_t* smem) {
   if (npad != 256) return false;
   if ((H / kKChunk) % 2 != 0) return false;
   tp->npad = npad;
   tp->ksub = 2;
   tp->nbuf = 2;
-  tp->group = npad == 128 ? 2 : 1;
+  tp->group = 1;
   tp->tmem_cols = 512;
-  const size_t a_stage = (size_t)kStageA * 2;
+  const size_t a_stage = (size_t)kStageA * 2 + (size_t)kTail * 128 * 2;  // + short-tile rows
   const size_t b_stage = (size_t)(npad / 2) * 128 * 2;
-  tp->stages_b = npad == 128 ? 4 : 3;
-  tp->stages_a = npad == 128 ? 4 : 3;
-  const size_t bars = 8 * (size_t)(2 * tp->stages_a + 2 * tp->stages_b + 5) + 16;
+  tp->stages_b = 3;
+  tp->stages_a = 3;
+  const size_t bars = 8 * (size_t)(2 * tp->stages_a + 2 * tp->stages_b + 6) + 16;
   *smem = 1024 + (size_t)tp->stages_a * a_stage + (size_t)tp->stages_b * b_stage + bars +
           red_bytes(npad);
-  return *smem <= 227 * 1024;
+  // Dynamic plus static (the final merge's row scratch) within 227 KB.
+  return *smem + kMaxRows * 8 + 64 <= 227 * 1024;
 }
 
 }  // namespace
@@ -897,15 +981,16 @@ cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem
   // form stays.
   if (beside_smem == 0 && a.R > 128 && a.R <= 256 &&
       lmhead_tc2_params(256, a.H, &tp, &smem)) {
-    CUtensorMap wf, x;
+    CUtensorMap wf, wt, x;
     const uint64_t w_inner = a.w_packed ? kKChunk : a.H;
     const uint64_t w_outer = a.w_packed ? (uint64_t)a.V * (a.H / kKChunk) : a.V;
     if (!make_map(&wf, a.w, w_inner, w_outer, kKChunk, kTileM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+        !make_map(&wt, a.w, w_inner, w_outer, kKChunk, kTail, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
         !make_map(&x, a.rows, a.H, a.R, kKChunk, tp.npad / 2, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
       return cudaErrorInvalidValue;
     LmArgs ap = a;
     ap.n_cta = (a.n_cta + 1) & ~1;  // whole pairs; a spare CTA reports an empty range
-    return launch_pair<8, 2>(wf, x, ap, tp, smem, s, after_producer);
+    return launch_pair<8, 2>(wf, wt, x, ap, tp, smem, s, after_producer);
   }
   if (!lmhead_tc_params(a.R, a.H, a.rows_per_cta, beside_smem, &tp, &smem))
     return cudaErrorInvalidValue;

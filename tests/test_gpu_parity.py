@@ -240,14 +240,18 @@ def test_llada_dualcache_step_more_seeds(seed, regime):
 
 @pytest.mark.parametrize("R,V,H", [(1, 5000, 64), (32, 5000, 448), (33, 33000, 128),
                                    (128, 20000, 256), (256, 7001, 64), (8, 151936, 1536),
-                                   (256, 152064, 256), (200, 152064, 128)])
+                                   (256, 152064, 256), (200, 152064, 128),
+                                   (256, 152885, 256), (144, 21000, 128)])
 def test_lmhead_shapes_against_oracle(R, V, H):
     """Every N padding (32..256), partial vocab tiles (5000 / 148 CTAs = 48
-    rows each), ragged vocab ends and several K depths; at the 7B vocabulary
-    with N = 256, nine tiles per CTA in groups of two sharing one TMEM
-    buffer, the last group a single 16-row tile.  Tokens must match
-    wherever the oracle's top-2 logit gap exceeds 1e-3 (fp32 accumulation
-    error is ~1e-5 at these sizes); confidences within 1e-3 relative."""
+    rows each), ragged vocab ends and several K depths.  From 129 rows the
+    CTA pairs: at the 7B vocabulary 1040 rows per CTA, eight full tiles and
+    a 16-row short tile folded into the first one (operands swapped); at
+    V = 152885 the last pair's odd CTA holds 5 rows (its short-tile and most
+    of its tile rows masked); at V = 21000, 144 rows per CTA, one full tile
+    and the folded one.  Tokens must match wherever the oracle's top-2 logit
+    gap exceeds 1e-3 (fp32 accumulation error is ~1e-5 at these sizes);
+    confidences within 1e-3 relative."""
     g = torch.Generator().manual_seed(R * 7 + V + H)
     rows = torch.randn((R, H), generator=g).to(torch.bfloat16)
     w = (torch.randn((V, H), generator=g) * (8.0 / H ** 0.5)).to(torch.bfloat16)
