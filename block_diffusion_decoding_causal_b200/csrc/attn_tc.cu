@@ -81,6 +81,8 @@ struct TcArgs {
   int inline_merge;       // the last CTA to finish a row of an item merges it
   int merge_wide;         // merge kernel: lanes over partials (many per item)
   int v_lag;              // V loads issued this many chunks behind K (0 or 1)
+  int wait_inputs;        // programmatic launch: wait for the previous grid
+                          // after the prologue, before any input is read
   int q_region;           // bytes between the two d-halves of the Q buffer
 };
 
@@ -382,7 +384,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   }
   // Sequence table from the device-resident lengths: warp 0 reads 32
   // lengths at a time and prefix-sums the chunk counts with shuffles.
-  if (warp == 0) {
+  auto build_table = [&]() {
     int run = 0;
     for (int b0 = 0; b0 < a.B; b0 += 32) {
       const int b = b0 + lane;
@@ -417,7 +419,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
       run += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) cb[a.B] = run;
-  }
+  };
+  // Without a wait its length reads overlap the rest of the prologue.
+  if (!a.wait_inputs && warp == 0) build_table();
   // Padding rows of the Q halves are never written by TMA: zero them once.
   const int q_rows = a.q_region / 128;
   for (int t = threadIdx.x; t < kQBufs * 2 * (q_rows - rows_full) * 8; t += kThreads) {
@@ -433,6 +437,14 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem;
+  // Launched as a programmatic dependent of whatever ran before (a stand-
+  // alone call): everything above overlapped that grid's tail; from here on
+  // inputs are read and the workspace written, so wait for it to finish.
+  if (a.wait_inputs) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (warp == 0) build_table();
+    __syncthreads();
+  }
 
   const long long T = cb[a.B];
   const int n = a.n_cta;
@@ -801,7 +813,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, const TcArgs a) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // When launched beside the step's LM head, finish only after it did, so
   // that this grid's completion (which the merge waits for) covers both.
-  // Without a programmatic predecessor this returns at once.
+  // Alone (the wait after the prologue already returned) or without a
+  // programmatic predecessor this returns at once.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
@@ -1108,6 +1121,17 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
   t.inline_merge = beside_prior ? 1 : 0;
   t.merge_wide = 0;
   t.v_lag = qpt * a.group > 64 ? 1 : 0;
+  // One sequence and one CTA per item (the PrefixCache shape): every item
+  // has the same chunks, each CTA's range is exactly one item and there is
+  // nothing to merge.
+  const bool no_merge = !beside_prior && a.B == 1 && n_cta == n_items_all;
+  // Programmatic launch.  Beside the LM head the attention reads nothing
+  // that kernel writes and starts at once.  Alone it waits for its
+  // predecessor after the prologue, so a call's launch and prologue overlap
+  // the previous call's merge: 0.7-1.8 us a call at batch 1-16 (batch 4,
+  // prefix 8192: 25.7 -> 24.0-24.3 us); the same time as before at the
+  // PrefixCache shape, whose predecessor has no merge to hide behind.
+  t.wait_inputs = beside_prior ? 0 : 1;
   t.q_region = q_region_for(qpt * a.group);
   // Beside the LM head: one K/V stage, so the SM's remaining shared memory
   // goes to that kernel's weight ring.
@@ -1127,14 +1151,12 @@ cudaError_t launch_attn_tc(const AttnArgs& a, float* part_o, float2* part_ml,
     mc.dynamicSmemBytes = smem;
     mc.stream = s;
     mc.attrs = attr;
-    mc.numAttrs = beside_prior ? 1 : 0;
+    mc.numAttrs = 1;
     e = cudaLaunchKernelEx(&mc, kern, maps, t);
     if (e != cudaSuccess) return e;
   }
   if (beside_prior) return cudaSuccess;  // merged inside the kernel
-  // One sequence and one CTA per item: all its items have the same chunks,
-  // so each CTA's range is exactly one item and there is nothing to merge.
-  if (a.B == 1 && n_cta == n_items_all) return cudaGetLastError();
+  if (no_merge) return cudaGetLastError();
   // The merge: up to three CTAs per SM, eight warps each, one (item, row)
   // task per warp at a time, or one (item, row, column quarter) with lanes
   // over the partials when an item has about 40 or more of them (batch 1 at
