@@ -47,6 +47,11 @@ __global__ void gather_rows_kernel(const uint4* src, const uint4* h_prev,
   // The LM head launched behind this kernel may start its weight stream now;
   // it waits for this grid before reading the rows.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // Launched as a programmatic dependent of the previous step (whose last
+  // grid, the attention, completes only after that step's LM head, the
+  // reader of `rows`): its launch overlapped that step; wait for it before
+  // reading the inputs or overwriting the rows.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const size_t n = (size_t)B * q_len * vec_per_row;
   for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < n;
        t += (size_t)gridDim.x * blockDim.x) {
@@ -96,10 +101,21 @@ cudaError_t launch_gather_rows(const void* src, const void* h_prev, void* rows,
   const size_t n = (size_t)B * q_len * vec_per_row;
   const int threads = 256;
   const int blocks = (int)((n + threads - 1) / threads);
-  gather_rows_kernel<<<blocks, threads, 0, s>>>(
-      static_cast<const uint4*>(src), static_cast<const uint4*>(h_prev),
-      static_cast<uint4*>(rows), B, q_len, vec_per_row, shift);
-  return cudaGetLastError();
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(blocks, 1, 1);
+  lc.blockDim = dim3(threads, 1, 1);
+  lc.dynamicSmemBytes = 0;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&lc, gather_rows_kernel,
+                                           static_cast<const uint4*>(src),
+                                           static_cast<const uint4*>(h_prev),
+                                           static_cast<uint4*>(rows), B, q_len, vec_per_row, shift);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace fdl
