@@ -183,7 +183,7 @@ int run_lmhead_passes(const LmArgs& a, const fdl_step_cfg& c, const Plan& p, cud
                       bool after_gather = false) {
   if (a.R <= p.lm_pass_rows) return run_lmhead(a, c, s, 0, after_gather);
   const size_t row_bytes = (size_t)c.hidden * p.elem;
-  for (int r0 = 0; r0 < a.R; r0 += p.lm_pass_rows) {
+  auto pass_args = [&](int r0) {
     LmArgs pa = a;
     const int b0 = r0 / c.q_len;
     pa.R = a.R - r0 < p.lm_pass_rows ? a.R - r0 : p.lm_pass_rows;
@@ -199,8 +199,30 @@ int run_lmhead_passes(const LmArgs& a, const fdl_step_cfg& c, const Plan& p, cud
       pa.n_committed = a.n_committed + b0;
       pa.n_masked_left = a.n_masked_left + b0;
     }
-    const int rc = run_lmhead(pa, c, s, 0, after_gather && r0 == 0);
+    return pa;
+  };
+  bool first = true;
+  for (int r0 = 0; r0 < a.R;) {
+    const LmArgs pa = pass_args(r0);
+    const int r1 = r0 + pa.R;
+    if (c.dtype == FDL_BF16 && r1 < a.R && p.lm_part_regions >= 2) {
+      // Two passes of the CTA-pair form in one launch, the second with its
+      // own partial region and ticket set.
+      LmArgs pb = pass_args(r1);
+      pb.part = a.part + (size_t)kLmMaxCTAs * p.lm_pass_rows;
+      pb.slot = 1;
+      if (lmhead_tc_two_pass_ok(pa, pb)) {
+        const cudaError_t e = launch_lmhead_tc_two_pass(pa, pb, s, after_gather && first);
+        if (e != cudaSuccess) return cuda_fail(e, "lm-head launch");
+        first = false;
+        r0 = r1 + pb.R;
+        continue;
+      }
+    }
+    const int rc = run_lmhead(pa, c, s, 0, after_gather && first);
     if (rc != FDL_OK) return rc;
+    first = false;
+    r0 = r1;
   }
   return FDL_OK;
 }

@@ -69,10 +69,12 @@ struct alignas(16) Partial {
 // Workspace control words (first 256 bytes of the workspace).
 constexpr int kLmTeam = 16;      // LM-head CTAs per first-level merge
 constexpr int kLmMaxTeams = 16;  // teams the control words count for
+// The LM head's tickets come in two sets (LmArgs::slot): one launch of the
+// CTA-pair form can run two passes, whose merges overlap.
 struct Control {
-  unsigned int status;                // FDL_DEV_* bits
-  unsigned int lm_ticket;             // LM-head last-CTA (or last-team) ticket
-  unsigned int lm_team[kLmMaxTeams];  // LM-head per-team tickets
+  unsigned int status;                   // FDL_DEV_* bits
+  unsigned int lm_ticket[2];             // LM-head last-CTA (or last-team) tickets
+  unsigned int lm_team[2][kLmMaxTeams];  // LM-head per-team tickets
 };
 
 // ----------------------------------------------------------------- attention
@@ -118,6 +120,7 @@ struct LmArgs {
   int rows_ready;            // tensor-core LM head: the rows were in place before
                              // its programmatic predecessor began, so it reads
                              // them without waiting for that grid
+  int slot;                  // ticket set in Control (0, or 1 for a launch's second pass)
   // fused commit (when commit != 0)
   int commit;
   int32_t* block_tokens;
@@ -283,6 +286,13 @@ cudaError_t launch_lmhead_simt(const LmArgs& a, fdl_dtype dt, cudaStream_t s);
 cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem = 0,
                              bool after_producer = false);
 bool lmhead_tc_shared_ok(const LmArgs& a, size_t beside_smem);
+// Two consecutive passes (129..256 rows each, full form) in one launch of
+// the CTA-pair form: b's partials in their own region and b.slot = 1, so
+// the first pass's merges run under the second pass's stream.  False: not
+// applicable (the caller launches the passes one by one).
+bool lmhead_tc_two_pass_ok(const LmArgs& a, const LmArgs& b);
+cudaError_t launch_lmhead_tc_two_pass(const LmArgs& a, const LmArgs& b, cudaStream_t s,
+                                      bool after_producer = false);
 // Rewrites the bf16 weight [V, H] into the tiled layout the LM head reads
 // when LmArgs::w_packed is set (see lmhead_tc.cu).
 cudaError_t launch_pack_weight(const void* w, void* out, int V, int H, int rows_per_cta,

@@ -30,6 +30,7 @@ struct Plan {
   bool step_ok;    // within the fused step's limits (LM head, commit sized)
   int R;           // LM-head rows = batch * q_len
   int lm_pass_rows;  // rows per LM-head pass: whole sequences, at most 256
+  int lm_part_regions;  // LM-head partial regions of kLmMaxCTAs x lm_pass_rows
   int elem;        // bytes per floating element
   int n_row_tiles;
   AttnSplit attn_plain, attn_dual;
@@ -152,8 +153,11 @@ inline bool make_plan(const fdl_step_cfg* c, Plan* p, std::string* why, bool ste
   // the fused step: sized only for configurations the step accepts.
   p->off_rows = off;
   off = align256(off + (size_t)p->elem * p->R * c->hidden);
+  // LM-head partials: one region per pass of a launch (two when the rows
+  // take more than one pass: the CTA-pair form runs two passes a launch).
   p->off_lm_part = off;
-  off = align256(off + 16 * (size_t)kLmMaxCTAs * p->lm_pass_rows);
+  p->lm_part_regions = p->R > p->lm_pass_rows ? 2 : 1;
+  off = align256(off + 16 * (size_t)kLmMaxCTAs * p->lm_pass_rows * p->lm_part_regions);
   p->off_attn = off;
   off = align256(off + (size_t)p->elem * p->R * c->n_q_heads * c->head_dim);
   // Tensor-core attention: at most two partials (first and last item) per CTA.

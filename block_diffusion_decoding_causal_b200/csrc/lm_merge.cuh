@@ -7,18 +7,34 @@
 
 namespace fdl {
 
+// The threads of a CTA that run a merge: all of them, or the tensor-core LM
+// head's four epilogue warps (threads 64..191, named barrier 1) while its
+// other warps already stream the next pass.
+struct CtaThreads {
+  __device__ static int rank() { return threadIdx.x; }
+  __device__ static int size() { return blockDim.x; }
+  __device__ static void sync() { __syncthreads(); }
+};
+struct EpilogueThreads {
+  __device__ static int rank() { return threadIdx.x - 64; }
+  __device__ static int size() { return 128; }
+  __device__ static void sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+};
+
 // "Last CTA to arrive" ticket: every CTA has written its partials; returns
 // true in exactly one CTA, after all other CTAs' writes are visible.  No
 // thread ever waits on another CTA.
+template <class G = CtaThreads>
 __device__ __forceinline__ bool last_cta_arrives(unsigned int* ticket,
                                                  unsigned int n_cta) {
   __shared__ int s_last;
   __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1u) == n_cta - 1u;
-  __syncthreads();
-  if (s_last) __threadfence();
-  return s_last != 0;
+  G::sync();
+  if (G::rank() == 0) s_last = atomicAdd(ticket, 1u) == n_cta - 1u;
+  G::sync();
+  const bool last = s_last != 0;
+  if (last) __threadfence();
+  return last;
 }
 
 // Row r's merge of n partials part[(first + j * stride) * R + r], j < n, in
@@ -50,14 +66,17 @@ __device__ __forceinline__ MSI lm_merge_sources(const Partial* part, int R, int 
 // The merges run one thread per row with all of a team's reads in flight, so
 // the tail after the last CTA is two short merges instead of one over every
 // CTA.  Each merger rearms its ticket.  No thread waits on another CTA.
+template <class G = CtaThreads>
 __device__ __forceinline__ bool lm_team_arrives(const LmArgs& a) {
   const int team = blockIdx.x / kLmTeam;
   const int first = team * kLmTeam;
   const int size = min(kLmTeam, a.n_cta - first);
   const int n_teams = (a.n_cta + kLmTeam - 1) / kLmTeam;
-  if (!last_cta_arrives(&a.ctrl->lm_team[team], (unsigned int)size)) return false;
-  if (threadIdx.x == 0) a.ctrl->lm_team[team] = 0u;
-  for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
+  unsigned int* team_ticket = &a.ctrl->lm_team[a.slot][team];
+  unsigned int* ticket = &a.ctrl->lm_ticket[a.slot];
+  if (!last_cta_arrives<G>(team_ticket, (unsigned int)size)) return false;
+  if (G::rank() == 0) *team_ticket = 0u;
+  for (int r = G::rank(); r < a.R; r += G::size()) {
     const MSI st = lm_merge_sources(a.part, a.R, r, first, 1, size);
     Partial p;
     p.m = st.m;
@@ -66,8 +85,8 @@ __device__ __forceinline__ bool lm_team_arrives(const LmArgs& a) {
     p.pad = 0;
     a.part[(size_t)first * a.R + r] = p;  // read above by this thread only
   }
-  if (!last_cta_arrives(&a.ctrl->lm_ticket, (unsigned int)n_teams)) return false;
-  if (threadIdx.x == 0) a.ctrl->lm_ticket = 0u;
+  if (!last_cta_arrives<G>(ticket, (unsigned int)n_teams)) return false;
+  if (G::rank() == 0) *ticket = 0u;
   return true;
 }
 
@@ -82,15 +101,16 @@ __device__ __forceinline__ bool lm_team_arrives(const LmArgs& a) {
 // before its ticket), its partials are stale: every row then reports
 // conf = -1 and tok = -1 and the commit selects nothing (block tokens kept,
 // counts written), until the caller reads and clears the status word.
+template <class G = CtaThreads>
 __device__ __forceinline__ void lm_final_merge(const LmArgs& a, int stride = 1) {
   __shared__ float s_conf[kMaxRows];
   __shared__ int s_tok[kMaxRows];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nw = blockDim.x >> 5;
+  const int warp = G::rank() >> 5, lane = threadIdx.x & 31;
+  const int nw = G::size() >> 5;
   const int n_src = (a.n_cta + stride - 1) / stride;
   const bool timed_out =
       (*reinterpret_cast<volatile unsigned int*>(&a.ctrl->status) & FDL_DEV_TIMEOUT) != 0u;
-  for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
+  for (int r = G::rank(); r < a.R; r += G::size()) {
     const MSI st = lm_merge_sources(a.part, a.R, r, 0, stride, n_src);
     bool act = true;
     if (a.row_active != nullptr) act = a.row_active[r] != 0;
@@ -107,7 +127,7 @@ __device__ __forceinline__ void lm_final_merge(const LmArgs& a, int stride = 1) 
     s_tok[r] = t;
   }
   if (!a.commit) return;
-  __syncthreads();
+  G::sync();
   for (int b = warp; b < a.B; b += nw) {
     const int base = b * a.q_len;
     if (timed_out) {

@@ -97,9 +97,9 @@ lmhead_simt_kernel(const LmArgs a) {
     }
     __syncthreads();
   }
-  if (!last_cta_arrives(&a.ctrl->lm_ticket, a.n_cta)) return;
+  if (!last_cta_arrives(&a.ctrl->lm_ticket[a.slot], a.n_cta)) return;
   lm_final_merge(a);
-  if (threadIdx.x == 0) a.ctrl->lm_ticket = 0u;
+  if (threadIdx.x == 0) a.ctrl->lm_ticket[a.slot] = 0u;
 }
 
 }  // namespace

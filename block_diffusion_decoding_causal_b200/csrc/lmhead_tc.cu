@@ -33,6 +33,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 namespace fdl {
@@ -399,11 +400,27 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w_full,
 // even CTA's entries before the odd CTA's; every (X row, vocabulary row)
 // pair is still counted once.  The MMA waits for those columns (tail_empty)
 // before the second tile.
+// Two passes in one launch (ps.n == 2: 257..512 rows as two groups of whole
+// sequences): the producer and the MMA go on from the first pass's last tile
+// to the second pass's first, with one count of TMEM buffers across both,
+// while the epilogue warps write the first pass's partials and run its
+// merges (its own ticket set) by themselves.  The last tile's epilogue and
+// the two merges of the first pass, about 25 us, then hide under the second
+// pass's MMAs, and one launch gap goes.
+struct XMaps {
+  CUtensorMap m[2];  // the X rows of each pass
+};
+struct LmPasses {
+  LmArgs p[2];  // outputs, partials and ticket set of each pass
+  int n;        // 1 or 2
+};
 template <int NCH, int KSUB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
                   const __grid_constant__ CUtensorMap tm_w_tail,
-                  const __grid_constant__ CUtensorMap tm_x, const LmArgs a, const TcParams tp) {
+                  const __grid_constant__ XMaps tm_x, const __grid_constant__ LmPasses ps,
+                  const TcParams tp) {
+  const LmArgs& a = ps.p[0];  // vocabulary, weight and control: the same in every pass
   constexpr int NPAD = NCH * 32;
   constexpr int NH = NPAD / 2;                    // X rows this CTA stages
   constexpr int SA_BYTES = kStageA * KSUB;        // one A stage: 128 rows x 64*KSUB
@@ -424,7 +441,8 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
   uint64_t* acc_empty = acc_full + 2;  // [2]
   uint64_t* drain = acc_empty + 2;     // [1]
   uint64_t* tail_empty = drain + 1;    // [1]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tail_empty + 1);
+  uint64_t* tail_free = tail_empty + 1;  // [1] next pass's short-tile columns read out
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tail_free + 1);
   MSI* s_red = reinterpret_cast<MSI*>(tmem_holder + 4);  // [4][NPAD], then [NH] short tile
   static_assert((4 * NPAD + NH) * sizeof(MSI) <= red_bytes(NPAD), "epilogue states fit");
 
@@ -460,6 +478,7 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
     }
     mbar_init(drain, 1);
     mbar_init(tail_empty, 256);
+    mbar_init(tail_free, 256);
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc_pair(tmem_holder, tp.tmem_cols);
@@ -474,13 +493,15 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
     if (lane == 0 && n_tiles > 0) {
       tma_prefetch_desc(&tm_w_full);
       tma_prefetch_desc(&tm_w_tail);
-      tma_prefetch_desc(&tm_x);
+      for (int pass = 0; pass < ps.n; ++pass) tma_prefetch_desc(&tm_x.m[pass]);
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
       // The rows may come from the kernel launched just before this one (the
       // token-shift gather, programmatic launch); without one this returns.
       if (!a.rows_ready) asm volatile("griddepcontrol.wait;" ::: "memory");
       int ia = 0, ib = 0;
+      for (int pass = 0; pass < ps.n && !failed; ++pass) {
+      const CUtensorMap* xm = &tm_x.m[pass];
       for (int g = 0; g < n_groups && !failed; ++g) {
         const int t0 = g * G, t1 = min(n_tiles, t0 + G);
         for (int kc = 0; kc < KC && !failed; ++kc) {
@@ -491,7 +512,7 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
             const uint32_t bar = mapa_shared(smem_u32(&full_b[slot_b]), 0u);
 #pragma unroll
             for (int u = 0; u < KSUB; ++u)
-              tma_load_2d_pair(sb + slot_b * SB_BYTES + u * NH * 128, &tm_x,
+              tma_load_2d_pair(sb + slot_b * SB_BYTES + u * NH * 128, xm,
                                (kc * KSUB + u) * kKChunk, (int)rank * NH, bar, pol_x);
             ++ib;
           }
@@ -535,6 +556,7 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
           }
         }
       }
+      }
       // Drain: every load of this CTA has landed before it can exit (the
       // even CTA's full barriers count both CTAs' bytes; the odd CTA waits
       // on its empty barriers, which the MMA releases only after the loads
@@ -557,11 +579,25 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
       const uint32_t idesc = idesc_bf16_f32(2 * kTileM, NPAD);
       const uint32_t idesc_tail = idesc_bf16_f32(2 * kTileM, 2 * kTail);
       int ia = 0, ib = 0;
-      for (int g = 0; g < n_groups && !failed; ++g) {
-        const int buf = tp.nbuf == 2 ? (g & 1) : 0;
-        const uint32_t ph = tp.nbuf == 2 ? ((g >> 1) & 1) : (g & 1);
+      int gg = 0;                        // groups over all passes: TMEM buffer gg & 1
+      int tail_buf = -1, tail_pass = 0;  // short-tile columns the epilogue still reads
+      for (int pass = 0; pass < ps.n && !failed; ++pass) {
+      for (int g = 0; g < n_groups && !failed; ++g, ++gg) {
+        const int buf = gg & 1;
+        const uint32_t ph = (gg >> 1) & 1;
         if (!mbar_wait(&acc_empty[buf], ph ^ 1)) { failed = true; break; }
-        if (fold && g == 1 && !mbar_wait(tail_empty, 0)) { failed = true; break; }
+        if (buf == tail_buf) {
+          if (!mbar_wait(tail_empty, (uint32_t)(tail_pass & 1))) { failed = true; break; }
+          tail_buf = -1;
+        }
+        const int tb = buf ^ 1;  // the short tile's columns: the start of the other buffer
+        if (fold && g == 0) {
+          // After the first pass that buffer holds the previous pass's last
+          // tile: the epilogue reads its first 32 columns first and says so.
+          if (pass > 0 && !mbar_wait(tail_free, (uint32_t)((pass - 1) & 1))) { failed = true; break; }
+          tail_buf = tb;
+          tail_pass = pass;
+        }
         tc_fence_after();
         const int t0 = g * G, t1 = min(n_tiles, t0 + G);
         for (int kc = 0; kc < KC && !failed; ++kc) {
@@ -581,7 +617,8 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
               for (int u = 0; u < KSUB; ++u)
 #pragma unroll
                 for (int k = 0; k < kKChunk / 16; ++k)
-                  mma_bf16_pair(tmem + (uint32_t)NPAD, desc_k_sw128(b_base + u * NH * 128 + k * 32),
+                  mma_bf16_pair(tmem + (uint32_t)(tb * NPAD),
+                                desc_k_sw128(b_base + u * NH * 128 + k * 32),
                                 desc_k_sw128(a_base + SA_BYTES + u * kTail * 128 + k * 32),
                                 idesc_tail, (kc | u | k) != 0 ? 1u : 0u);
             }
@@ -600,6 +637,7 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
         }
         mma_commit_pair(&acc_full[buf]);
       }
+      }
       mma_commit_pair_local(drain);
       if (!mbar_wait(drain, 0)) failed = true;
     }
@@ -609,13 +647,17 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
     float* tr = reinterpret_cast<float*>(s_red) + (warp - 2) * (32 * kTrStride);
     const uint32_t acc_empty_lead0 = mapa_shared(smem_u32(&acc_empty[0]), 0u);
     const uint32_t acc_empty_lead1 = mapa_shared(smem_u32(&acc_empty[1]), 0u);
+    const uint32_t tail_free_lead = mapa_shared(smem_u32(tail_free), 0u);
+    int gg = 0;
+    for (int pass = 0; pass < ps.n; ++pass) {
+    const LmArgs& ap = ps.p[pass];
     MSI st[NCH];
 #pragma unroll
     for (int c = 0; c < NCH; ++c) st[c] = msi_empty();
     MSI st_tail = msi_empty();  // X row rank * NH + q * 32 + lane, short-tile entries
-    for (int g = 0; g < n_groups; ++g) {
-      const int buf = tp.nbuf == 2 ? (g & 1) : 0;
-      const uint32_t ph = tp.nbuf == 2 ? ((g >> 1) & 1) : (g & 1);
+    for (int g = 0; g < n_groups && !failed; ++g, ++gg) {
+      const int buf = gg & 1;
+      const uint32_t ph = (gg >> 1) & 1;
       if (!mbar_wait(&acc_full[buf], ph)) { failed = true; break; }
       tc_fence_after();
       if (fold && g == 0) {
@@ -623,7 +665,7 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
         // odd CTA's, each in increasing vocabulary order.
         uint32_t r[32];
         static_assert(2 * kTail == 32, "one 32-column load holds the short tile");
-        tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)NPAD, r);
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((buf ^ 1) * NPAD), r);
         tmem_ld_wait();
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -638,6 +680,9 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
         mbar_arrive_cluster(mapa_shared(smem_u32(tail_empty), 0u));
       }
       const int t0 = g * G, t1 = min(n_tiles, t0 + G);
+      // The last group of a pass before a folding one: its first 32 columns
+      // are the next pass's short-tile columns.
+      const bool free_head = fold && g == n_groups - 1 && pass + 1 < ps.n;
       for (int t = t0; t < t1; ++t) {
         const int vbase = v0 + t * kTileM + q * 32;
         const int n_valid = min(32, v1 - vbase);  // same for the whole warp; may be <= 0
@@ -648,6 +693,10 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
                                  (uint32_t)((buf * G + (t - t0)) * NPAD + c * 32),
                              r);
           tmem_ld_wait();
+          if (c == 0 && free_head) {
+            tc_fence_before();
+            mbar_arrive_cluster(tail_free_lead);
+          }
           // Lane = vocabulary row in r; after the transpose lane j reads
           // column j, rows in increasing vocabulary order.
 #pragma unroll
@@ -674,14 +723,25 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
       for (int j = 1; j < 4; ++j) m = msi_merge(m, s_red[j * NPAD + col]);
       const int xl = col - (int)rank * NH;
       if (xl >= 0 && xl < NH) m = msi_merge(m, s_tail[xl]);
-      if (col < a.R) {
+      if (col < ap.R) {
         Partial p;
         p.m = m.m;
         p.s = m.s;
         p.i = m.i;
         p.pad = 0;
-        a.part[(size_t)blockIdx.x * a.R + col] = p;
+        ap.part[(size_t)blockIdx.x * ap.R + col] = p;
       }
+    }
+    // A pass before the last merges now, by the four epilogue warps alone
+    // while the others stream the next pass (their barriers also keep the
+    // transpose buffers, which share s_red, from being rewritten before
+    // every warp has read it); the last pass merges below with every
+    // thread.  Every CTA arrives on every pass, failed or not, so the
+    // tickets always complete and rearm.
+    if (pass + 1 < ps.n) {
+      if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
+      if (lm_team_arrives<EpilogueThreads>(ap)) lm_final_merge<EpilogueThreads>(ap, kLmTeam);
+    }
     }
   }
 
@@ -693,8 +753,8 @@ lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tm_w_full,
     tmem_dealloc_pair(tmem, tp.tmem_cols);
   }
   if (failed) atomicOr(&a.ctrl->status, kDevTimeout);
-  if (!lm_team_arrives(a)) return;
-  lm_final_merge(a, kLmTeam);
+  if (!lm_team_arrives(ps.p[ps.n - 1])) return;
+  lm_final_merge(ps.p[ps.n - 1], kLmTeam);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -787,9 +847,10 @@ cudaError_t launch_nch(const CUtensorMap& wf, const CUtensorMap& wp, const CUten
 }
 
 template <int NCH, int KSUB>
-cudaError_t launch_pair(const CUtensorMap& wf, const CUtensorMap& wt, const CUtensorMap& x,
-                        const LmArgs& a, const TcParams& tp, size_t smem, cudaStream_t s,
+cudaError_t launch_pair(const CUtensorMap& wf, const CUtensorMap& wt, const XMaps& x,
+                        const LmPasses& ps, const TcParams& tp, size_t smem, cudaStream_t s,
                         bool after_producer) {
+  const LmArgs& a = ps.p[0];
   auto k = lmhead_tc2_kernel<NCH, KSUB>;
   static std::mutex mu;
   static size_t smem_set[64] = {};
@@ -815,7 +876,7 @@ cudaError_t launch_pair(const CUtensorMap& wf, const CUtensorMap& wt, const CUte
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = after_producer ? 1 : 0;
-  return cudaLaunchKernelEx(&lc, k, wf, wt, x, a, tp);
+  return cudaLaunchKernelEx(&lc, k, wf, wt, x, ps, tp);
 }
 
 // Ring shapes of the CTA-pair form (256 padded rows, full form): two-box K
@@ -840,11 +901,12 @@ bool lmhead_tc2_params(int npad, int H, TcParams* tp, size_t* smem) {
   const size_t b_stage = (size_t)(npad / 2) * 128 * 2;
   tp->stages_b = 3;
   tp->stages_a = 3;
-  const size_t bars = 8 * (size_t)(2 * tp->stages_a + 2 * tp->stages_b + 6) + 16;
+  const size_t bars = 8 * (size_t)(2 * tp->stages_a + 2 * tp->stages_b + 7) + 16;
   *smem = 1024 + (size_t)tp->stages_a * a_stage + (size_t)tp->stages_b * b_stage + bars +
           red_bytes(npad);
-  // Dynamic plus static (the final merge's row scratch) within 227 KB.
-  return *smem + kMaxRows * 8 + 64 <= 227 * 1024;
+  // Dynamic plus static (the row scratch of the two final-merge forms, all
+  // threads and epilogue warps only) within 227 KB.
+  return *smem + 2 * kMaxRows * 8 + 64 <= 227 * 1024;
 }
 
 }  // namespace
@@ -970,6 +1032,55 @@ bool lmhead_tc_shared_ok(const LmArgs& a, size_t beside_smem) {
   return lmhead_tc_params(a.R, a.H, a.rows_per_cta, beside_smem, &tp, &smem);
 }
 
+// The CTA-pair form over ps.n passes (the tensor maps of the weight, its
+// short tiles and each pass's rows; whole pairs of CTAs, a spare CTA
+// reporting an empty range).
+static cudaError_t launch_pair_passes(LmPasses ps, const TcParams& tp, size_t smem,
+                                      cudaStream_t s, bool after_producer) {
+  const LmArgs& a = ps.p[0];
+  CUtensorMap wf, wt;
+  XMaps x;
+  memset(&x, 0, sizeof(x));
+  const uint64_t w_inner = a.w_packed ? kKChunk : a.H;
+  const uint64_t w_outer = a.w_packed ? (uint64_t)a.V * (a.H / kKChunk) : a.V;
+  if (!make_map(&wf, a.w, w_inner, w_outer, kKChunk, kTileM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+      !make_map(&wt, a.w, w_inner, w_outer, kKChunk, kTail, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+    return cudaErrorInvalidValue;
+  for (int i = 0; i < ps.n; ++i) {
+    if (!make_map(&x.m[i], ps.p[i].rows, a.H, ps.p[i].R, kKChunk, tp.npad / 2,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+      return cudaErrorInvalidValue;
+    ps.p[i].n_cta = (a.n_cta + 1) & ~1;
+  }
+  return launch_pair<8, 2>(wf, wt, x, ps, tp, smem, s, after_producer);
+}
+
+bool lmhead_tc_two_pass_ok(const LmArgs& a, const LmArgs& b) {
+  TcParams tp;
+  size_t smem = 0;
+  return a.R > 128 && a.R <= 256 && b.R > 128 && b.R <= 256 && a.H == b.H && a.V == b.V &&
+         a.w == b.w && a.n_cta == b.n_cta && a.rows_per_cta == b.rows_per_cta &&
+         a.w_packed == b.w_packed && a.ctrl == b.ctrl && a.part != b.part &&
+         a.n_cta <= kLmTeam * kLmMaxTeams && lmhead_tc2_params(256, a.H, &tp, &smem);
+}
+
+cudaError_t launch_lmhead_tc_two_pass(const LmArgs& a, const LmArgs& b, cudaStream_t s,
+                                      bool after_producer) {
+  TcParams tp;
+  size_t smem = 0;
+  if (!lmhead_tc_two_pass_ok(a, b) || !lmhead_tc2_params(256, a.H, &tp, &smem))
+    return cudaErrorInvalidValue;
+  LmPasses ps;
+  memset(&ps, 0, sizeof(ps));
+  ps.p[0] = a;
+  ps.p[0].slot = 0;
+  ps.p[1] = b;
+  ps.p[1].slot = 1;
+  ps.p[1].rows_ready = a.rows_ready;
+  ps.n = 2;
+  return launch_pair_passes(ps, tp, smem, s, after_producer);
+}
+
 cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem,
                              bool after_producer) {
   TcParams tp;
@@ -981,16 +1092,11 @@ cudaError_t launch_lmhead_tc(const LmArgs& a, cudaStream_t s, size_t beside_smem
   // form stays.
   if (beside_smem == 0 && a.R > 128 && a.R <= 256 &&
       lmhead_tc2_params(256, a.H, &tp, &smem)) {
-    CUtensorMap wf, wt, x;
-    const uint64_t w_inner = a.w_packed ? kKChunk : a.H;
-    const uint64_t w_outer = a.w_packed ? (uint64_t)a.V * (a.H / kKChunk) : a.V;
-    if (!make_map(&wf, a.w, w_inner, w_outer, kKChunk, kTileM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
-        !make_map(&wt, a.w, w_inner, w_outer, kKChunk, kTail, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
-        !make_map(&x, a.rows, a.H, a.R, kKChunk, tp.npad / 2, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
-      return cudaErrorInvalidValue;
-    LmArgs ap = a;
-    ap.n_cta = (a.n_cta + 1) & ~1;  // whole pairs; a spare CTA reports an empty range
-    return launch_pair<8, 2>(wf, wt, x, ap, tp, smem, s, after_producer);
+    LmPasses ps;
+    memset(&ps, 0, sizeof(ps));
+    ps.p[0] = a;
+    ps.n = 1;
+    return launch_pair_passes(ps, tp, smem, s, after_producer);
   }
   if (!lmhead_tc_params(a.R, a.H, a.rows_per_cta, beside_smem, &tp, &smem))
     return cudaErrorInvalidValue;

@@ -11,6 +11,7 @@ import pytest
 import torch
 
 from block_diffusion_decoding_causal_b200 import fdl, synth
+from oracle import step
 from tests import gpu_harness as gh
 
 pytestmark = pytest.mark.gpu
@@ -97,3 +98,34 @@ def test_fused_step_repeats_bit_for_bit():
         for k in ("tok", "committed", "n_committed", "n_masked_left", "block_tokens"):
             assert torch.equal(r[k], runs[0][k]), k
         assert r["status"] == 0
+
+
+@pytest.mark.parametrize("batch,prefix", [(4, 8192), (1, 8192), (4, 2048)])
+def test_attention_calls_back_to_back(batch, prefix):
+    """Consecutive standalone attention calls on one stream and one
+    workspace with no synchronisation between them.  Each launch is a
+    programmatic dependent of the previous call's merge kernel: it starts
+    during that merge and must wait for it before reading its lengths or
+    reusing the workspace's tickets and partial slots.  Three different
+    inputs (ragged prefix lengths), each output against the oracle; at
+    prefix 8192 batch 1 merges tens of partials per item (the wide merge),
+    batch 4 about twenty."""
+    outs, cases_ = [], []
+    c = dict(synth.sweep_config(batch, prefix), prefix=(prefix // 2, prefix))
+    for seed in (21, 22, 23):
+        case = synth.make_case("sweep", seed, cfg=c, draw_w=False)
+        cases_.append((case, fdl.make_cfg(case.cfg), gh.device_case(case)))
+    ws = fdl.workspace(cases_[0][1])  # same geometry; the unit offset differs
+    torch.cuda.synchronize()
+    for case, cfg, d in cases_:
+        out = torch.empty_like(d["q"])
+        fdl.block_attn(cfg, d["q"], d["k_pre"], d["v_pre"], d["len_pre"], d["k_blk"],
+                       d["v_blk"], out, ws)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert fdl.get_status(ws) == 0
+    for (case, _, _), out in zip(cases_, outs):
+        ref = step.attention_step(case.q, case.k_pre, case.v_pre, case.len_pre.numpy(),
+                                  case.prompt_len.numpy(), case.k_blk, case.v_blk,
+                                  case.cfg["q_off"])
+        gh.assert_close_scaled(out.double().cpu().numpy(), ref, 2e-2, "attn")
