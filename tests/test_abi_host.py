@@ -208,6 +208,17 @@ def test_step_rows_beyond_one_lm_pass_are_accepted_up_to_4096(L):
     assert rc == fdl.ERR_INVALID_ARG and "4096" in fdl.last_error()
 
 
+def test_rows_past_one_pass_get_a_second_partial_region(L):
+    """Past 256 LM-head rows the CTA-pair form runs two passes in one launch,
+    each with its own region of per-CTA partials (up to 4 x 148 CTAs x 256
+    rows x 16 bytes): crossing from 256 to 264 rows adds at least that much
+    workspace, while 8 more rows below one pass add little."""
+    region = 4 * 148 * 256 * 16
+    size = lambda b: L.fdl_workspace_size(ctypes.byref(_cfg(batch=b, q_len=8, q_off=0)))
+    assert size(33) - size(32) >= region
+    assert size(32) - size(31) < region // 4
+
+
 def test_wait_timeout_check_rejects_bad_arguments(L):
     rc = L.fdl_check_wait_timeout(None, 256, 1000000, None)
     assert rc == fdl.ERR_WORKSPACE
