@@ -377,6 +377,11 @@ def main():
     ms_per_step = t_step / args.steps * 1e3
     pos = world * B * q_len * args.steps
     value = pos / t_step
+    # The same K steps replayed from one CUDA graph (as a serving loop that
+    # captures its step runs them): reported beside the headline, which
+    # stays the back-to-back direct calls.
+    step_graph = graph_rounds_us(torch, stream, lambda i: step(sets[i % n_copies]),
+                                 args.steps, 3, world)
 
     # Dominant kernel: the fused LM head (weight stream), timed alone on the
     # same stream over K launches.
@@ -570,6 +575,10 @@ def main():
                                 / peaks["hbm_gbs"]}},
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": step_bytes / (t_step / args.steps) / 1e9,
                           "frac": step_bytes / (t_step / args.steps) / 1e9 / peaks["hbm_gbs"]},
+        "step_graph": {"us": spread(step_graph),
+                       "positions_per_s": world * B * q_len / statistics.median(step_graph) * 1e6,
+                       "frac_hbm": step_bytes / statistics.median(step_graph) / 1e3
+                       / peaks["hbm_gbs"]},
         "prefixcache": pc,
         "block_decode": blk,
         "lmhead_large_batch": lm_big,
