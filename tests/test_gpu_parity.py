@@ -416,11 +416,15 @@ def test_prefixcache_attn_against_oracle(B, Hq, Hkv, n, lens):
 
 # ---------------------------------------- more LM-head rows than one pass holds
 
-def test_lmhead_more_rows_than_one_pass():
+@pytest.mark.parametrize("V", [20000, 59200])
+def test_lmhead_more_rows_than_one_pass(V):
     """batch * q_len = 600 rows: passes of 256, 256 and 88 rows over the
-    weight, against the oracle (tokens where the top-2 gap exceeds 1e-3)."""
-    B, q_len, V, H = 75, 8, 20000, 256
-    g = torch.Generator().manual_seed(600)
+    weight (the first two in one launch of the CTA pairs), against the
+    oracle (tokens where the top-2 gap exceeds 1e-3).  V = 20000: one full
+    tile per CTA plus the folded short tile; V = 59200: three (an odd group
+    count, so the second pass starts on the other TMEM buffer)."""
+    B, q_len, H = 75, 8, 256
+    g = torch.Generator().manual_seed(600 + V)
     rows = torch.randn((B * q_len, H), generator=g).to(torch.bfloat16)
     w = (torch.randn((V, H), generator=g) * (8.0 / H ** 0.5)).to(torch.bfloat16)
     active = (torch.rand(B * q_len, generator=g) < 0.8).to(torch.uint8)
@@ -446,6 +450,19 @@ LARGE_BATCH = dict(batch=40, n_q_heads=8, n_kv_heads=2, head_dim=128, block_size
                    q_len=8, q_off=None, prefix=(100, 400), cap_prefix=400, suffix=0,
                    cap_suffix=0, hidden=256, vocab=5000, mask_id=4999, shift=1, tau=0.8,
                    w_scale=8.0, dtype="bf16", masked=(1, 8))
+
+
+@pytest.mark.parametrize("vocab", [5000, 59200])
+def test_fused_step_two_lm_passes_in_one_launch(vocab):
+    """400 LM-head rows (passes of 256 and 144, both on CTA pairs, in one
+    launch): the first pass commits its 32 sequences from the epilogue warps
+    while the second pass streams, the second its 18 after the main loop;
+    bit-exact commits against the oracle.  vocab 59200: three tiles per CTA
+    and the folded short tile in each pass."""
+    cfg = dict(LARGE_BATCH, batch=50, vocab=vocab, mask_id=vocab - 1)
+    case, ref, _ = cases.parity_case("large_batch", 0, cfg=cfg)
+    gh.compare_step(case, gh.run_denoise_step(case), ref)
+    gh.compare_step(case, gh.run_denoise_step(case, packed=True), ref)
 
 
 @pytest.mark.parametrize("shift", [1, 0])
