@@ -129,3 +129,36 @@ def test_attention_calls_back_to_back(batch, prefix):
                                   case.prompt_len.numpy(), case.k_blk, case.v_blk,
                                   case.cfg["q_off"])
         gh.assert_close_scaled(out.double().cpu().numpy(), ref, 2e-2, "attn")
+
+
+def test_two_pass_launch_matches_two_single_passes():
+    """512 rows (two passes of 256 in one launch of the CTA pairs, the first
+    pass's merges on a second ticket set under the second pass's stream)
+    return the very same bits as the two halves called one by one: the
+    arithmetic of each pass is unchanged by sharing a launch."""
+    c = dict(synth.CONFIGS["qwen7b"], batch=64, q_off=0)
+    V, H = c["vocab"], c["hidden"]
+    g = torch.Generator(device="cuda").manual_seed(512)
+    w_rm = (torch.randn((V, H), generator=g, device="cuda") * (8.0 / H ** 0.5)).to(torch.bfloat16)
+    cfg = fdl.make_cfg(c)
+    w = torch.empty_like(w_rm)
+    fdl.lmhead_pack_weight(cfg, w_rm, w)
+    del w_rm
+    rows = torch.randn((512, H), generator=g, device="cuda").to(torch.bfloat16)
+    cfg.w_layout = fdl.W_PACKED
+    conf = torch.empty(512, dtype=torch.float32, device="cuda")
+    tok = torch.empty(512, dtype=torch.int32, device="cuda")
+    ws = fdl.workspace(cfg)
+    fdl.lmhead_confidence(cfg, rows, w, None, conf, tok, ws)
+    half = fdl.make_cfg(dict(c, batch=32))
+    half.w_layout = fdl.W_PACKED
+    ws_h = fdl.workspace(half)
+    conf_h = torch.empty(512, dtype=torch.float32, device="cuda")
+    tok_h = torch.empty(512, dtype=torch.int32, device="cuda")
+    for r0 in (0, 256):
+        fdl.lmhead_confidence(half, rows[r0:r0 + 256], w, None, conf_h[r0:r0 + 256],
+                              tok_h[r0:r0 + 256], ws_h)
+    torch.cuda.synchronize()
+    assert torch.equal(tok.cpu(), tok_h.cpu())
+    assert torch.equal(conf.cpu().view(torch.int32), conf_h.cpu().view(torch.int32))
+    assert fdl.get_status(ws) == 0 and fdl.get_status(ws_h) == 0
